@@ -1,0 +1,116 @@
+"""Plant one plausible mistake at a time in the oracle (on the CPU) and check
+that the pins catch it.  This shows the pins are sensitive to dropped terms,
+wrong signs/indices and transposed operands."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention as A
+from tests import oracle_pins as P
+
+ALL_PREFILL_PINS = [
+    lambda: P.pin_golden_two_keys(A.attention_ref),
+    lambda: P.pin_golden_causal_uniform(A.attention_ref),
+    lambda: P.pin_identical_keys(A.attention_ref, True),
+    lambda: P.pin_identical_keys(A.attention_ref, False),
+    lambda: P.pin_causal_row0(A.attention_ref),
+    lambda: P.pin_bruteforce(A.attention_ref),
+    lambda: P.pin_sdpa(A.attention_ref),
+    lambda: P.pin_rows_sum_to_one(A.attention_probs_ref, True),
+]
+
+
+def _some_pin_fires(pins):
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            return True
+    return False
+
+
+MUTANTS = {
+    # causal mask in the wrong direction (future keys allowed, past masked)
+    "mask_flipped": ("_causal_mask_block",
+                     lambda row0, n, nk: (np.arange(nk)[None, :] < np.arange(row0, row0 + n)[:, None])),
+    # off-by-one: diagonal key masked
+    "mask_excludes_diag": ("_causal_mask_block",
+                           lambda row0, n, nk: (np.arange(nk)[None, :] >= np.arange(row0, row0 + n)[:, None])),
+    # scale dropped
+    "no_scale": ("_scores", lambda q, k, scale: q @ k.T),
+    # operands transposed (K Q^T instead of Q K^T) on square blocks
+    "transposed": ("_scores", lambda q, k, scale: scale * (k @ q.T) if q.shape == k.shape else scale * (q @ k.T)),
+    # GQA head mapping interleaved instead of grouped
+    "gqa_modulo": ("kv_head_of", lambda h, hq, hkv: h % hkv),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_prefill_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(A, attr, fn)
+    assert _some_pin_fires(ALL_PREFILL_PINS), f"no pin caught mutant {name}"
+
+
+def test_lse_base2_is_caught(monkeypatch):
+    orig = A._softmax_with_lse
+
+    def bad(s):
+        p, lse = orig(s)
+        return p, lse / math.log(2.0)
+    monkeypatch.setattr(A, "_softmax_with_lse", bad)
+    assert _some_pin_fires(ALL_PREFILL_PINS)
+
+
+def test_lse_missing_max_is_caught(monkeypatch):
+    orig = A._softmax_with_lse
+
+    def bad(s):
+        p, lse = orig(s)
+        m = np.max(s, axis=-1)
+        return p, lse - np.where(np.isfinite(m), m, 0.0)
+    monkeypatch.setattr(A, "_softmax_with_lse", bad)
+    assert _some_pin_fires(ALL_PREFILL_PINS)
+
+
+def _merge_uniform(o_parts, lse_parts):
+    o_parts = np.asarray(o_parts)
+    return o_parts.mean(axis=0), np.max(lse_parts, axis=0)
+
+
+def _merge_no_shift(o_parts, lse_parts):
+    w = np.exp(np.asarray(lse_parts))
+    return (w[..., None] * o_parts).sum(0) / w.sum(0)[..., None], np.log(w.sum(0))
+
+
+def _merge_wrong_lse(o_parts, lse_parts):
+    o, l = oracle.merge_states_ref(o_parts, lse_parts)
+    return o, np.max(lse_parts, axis=0)
+
+
+@pytest.mark.parametrize("bad", [_merge_uniform, _merge_no_shift, _merge_wrong_lse])
+def test_merge_mutant_is_caught(bad):
+    pins = [lambda: P.pin_golden_merge(bad),
+            lambda: P.pin_partition_merge(oracle.partial_state_ref, bad, oracle.attention_rows_ref)]
+    with np.errstate(all="ignore"):
+        assert _some_pin_fires(pins)
+
+
+def test_paged_walk_mutant_is_caught(monkeypatch):
+    """Reading slot t % page_size from page t // page_size of the *physical*
+    pool (ignoring the page table) must be caught."""
+    def bad_gather(k_pages, v_pages, row, seqlen, g, ps, layout="NHD"):
+        n = (seqlen + ps - 1) // ps
+        if layout == "NHD":
+            K = np.concatenate([k_pages[p, :, g] for p in range(n)])[:seqlen]
+            V = np.concatenate([v_pages[p, :, g] for p in range(n)])[:seqlen]
+        else:
+            K = np.concatenate([k_pages[p, g] for p in range(n)])[:seqlen]
+            V = np.concatenate([v_pages[p, g] for p in range(n)])[:seqlen]
+        return K, V
+    monkeypatch.setattr(A, "gather_paged_kv", bad_gather)
+    pins = [lambda: P.pin_golden_paged(A.paged_decode_ref),
+            lambda: P.pin_decode_walk(A.paged_decode_ref, A.partial_state_ref)]
+    assert _some_pin_fires(pins)

@@ -1,0 +1,341 @@
+"""Seeded synthetic inputs for exact attention (prefill and paged decode).
+
+This module is shared by the CPU oracle's tests, the GPU parity tests and
+``bench.py``.  It only draws random numbers, rounds them to bfloat16 and lays
+them out; it holds none of the attention arithmetic.
+
+Workload shapes follow the pages' problem statements:
+
+* prefill: packed ``[T, H, d]`` Q/K/V with ``cu_seqlens`` offsets (the FA
+  varlen form named on "FIA / FlashAttention", section 二 and 三);
+* decode: one query row per request over a KV cache stored in fixed-size pages
+  (64 tokens per page, "FlashAttention突破性架构", section 分页存储系统) addressed
+  through a logical-to-physical page table ("Flash Attention & Paged
+  Attention", section 2).
+
+Every tensor is produced as float32 draws from N(0, 1), rounded to bfloat16
+with round-to-nearest-even.  The ``*_bits`` arrays are the uint16 bit patterns
+that go to the device; ``as_f64`` gives the same values widened for the oracle.
+"""
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field
+
+import numpy as np
+
+PAGE_SIZE = 64
+
+
+# ---------------------------------------------------------------------------
+# bfloat16 helpers (bit manipulation only)
+# ---------------------------------------------------------------------------
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (round-to-nearest-even); uint16 bits."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    out = rounded.astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        out[nan] = 0x7FC0
+    return out
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def as_f64(b: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns -> float64 values (exact widening)."""
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+def _normal_bf16_bits(seed_seq: np.random.SeedSequence, shape, chunk_elems=1 << 24) -> np.ndarray:
+    """N(0,1) float32 draws rounded to bf16, filled in parallel chunks.
+
+    Each chunk draws from its own child of ``seed_seq`` so the result does not
+    depend on the number of worker threads.
+    """
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    nchunks = max(1, math.ceil(n / chunk_elems))
+    children = seed_seq.spawn(nchunks)
+
+    def fill(i):
+        lo = i * chunk_elems
+        hi = min(n, lo + chunk_elems)
+        g = np.random.Generator(np.random.PCG64(children[i]))
+        out[lo:hi] = f32_to_bf16_bits(g.standard_normal(hi - lo, dtype=np.float32))
+
+    workers = min(nchunks, os.cpu_count() or 1)
+    if workers <= 1:
+        for i in range(nchunks):
+            fill(i)
+    else:
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, range(nchunks)))
+    return out.reshape(shape)
+
+
+# ---------------------------------------------------------------------------
+# Prefill workloads
+# ---------------------------------------------------------------------------
+
+@dataclass
+class PrefillInputs:
+    name: str
+    q_bits: np.ndarray          # [T, Hq, d] uint16 (bf16)
+    k_bits: np.ndarray          # [T, Hkv, d]
+    v_bits: np.ndarray          # [T, Hkv, d]
+    cu_seqlens: np.ndarray      # [B+1] int32
+    causal: bool
+    scale: float
+    q_f32_unrounded: np.ndarray | None = None   # only kept for tiny cases
+
+    @property
+    def num_q_heads(self):
+        return self.q_bits.shape[1]
+
+    @property
+    def num_kv_heads(self):
+        return self.k_bits.shape[1]
+
+    @property
+    def head_dim(self):
+        return self.q_bits.shape[2]
+
+    @property
+    def seqlens(self):
+        return np.diff(self.cu_seqlens).astype(np.int64)
+
+    def causal_flops(self) -> float:
+        """Algorithmic FLOPs: 4*d*Hq per (query, allowed key) pair."""
+        L = self.seqlens
+        pairs = (L * (L + 1) // 2).sum() if self.causal else (L * L).sum()
+        return 4.0 * self.head_dim * self.num_q_heads * float(pairs)
+
+
+def make_prefill(seqlens, num_q_heads, num_kv_heads, head_dim, *, causal=True,
+                 scale=None, seed=0, name="prefill") -> PrefillInputs:
+    seqlens = np.asarray(seqlens, dtype=np.int64)
+    cu = np.zeros(len(seqlens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(seqlens)
+    T = int(cu[-1])
+    ss = np.random.SeedSequence(seed)
+    sq, sk, sv = ss.spawn(3)
+    q = _normal_bf16_bits(sq, (T, num_q_heads, head_dim))
+    k = _normal_bf16_bits(sk, (T, num_kv_heads, head_dim))
+    v = _normal_bf16_bits(sv, (T, num_kv_heads, head_dim))
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    return PrefillInputs(name, q, k, v, cu, causal, float(scale))
+
+
+def tiny_causal_prefill() -> PrefillInputs:
+    """Batch 1, 2 heads, 128 tokens, d=64, fp32 N(0,1) inputs, scale 1/sqrt(64).
+
+    The fp32 draws are rounded to bf16 before either side sees them; the
+    unrounded query is kept so tests can report the rounding effect.
+    """
+    g = np.random.default_rng(0)
+    T, H, d = 128, 2, 64
+    qf = g.standard_normal((T, H, d), dtype=np.float32)
+    kf = g.standard_normal((T, H, d), dtype=np.float32)
+    vf = g.standard_normal((T, H, d), dtype=np.float32)
+    cu = np.array([0, T], dtype=np.int32)
+    inp = PrefillInputs("tiny_causal_prefill", f32_to_bf16_bits(qf), f32_to_bf16_bits(kf),
+                        f32_to_bf16_bits(vf), cu, True, 1.0 / math.sqrt(64))
+    inp.q_f32_unrounded = qf
+    return inp
+
+
+def varlen_lengths(seed=1, batch=8, lo=512, hi=4096) -> np.ndarray:
+    return np.random.default_rng(seed).integers(lo, hi + 1, size=batch).astype(np.int64)
+
+
+def varlen_causal_prefill() -> PrefillInputs:
+    """8 sequences, lengths uniform in [512, 4096], 32 heads MHA, d=128, causal."""
+    return make_prefill(varlen_lengths(1), 32, 32, 128, causal=True, seed=1,
+                        name="varlen_causal_prefill")
+
+
+def long_gqa_prefill() -> PrefillInputs:
+    """One 32768-token sequence, 32 query heads sharing 8 KV heads, d=128, causal."""
+    return make_prefill([32768], 32, 8, 128, causal=True, seed=2, name="long_gqa_prefill")
+
+
+# ---------------------------------------------------------------------------
+# Paged decode workloads
+# ---------------------------------------------------------------------------
+
+@dataclass
+class DecodeInputs:
+    name: str
+    q_bits: np.ndarray            # [B, Hq, d]
+    k_pages_bits: np.ndarray      # NHD: [P, page, Hkv, d]; HND: [P, Hkv, page, d]
+    v_pages_bits: np.ndarray
+    block_table: np.ndarray       # [B, max_pages] int32 (unused slots = -1)
+    cache_seqlens: np.ndarray     # [B] int32
+    scale: float
+    layout: str = "NHD"
+    page_size: int = PAGE_SIZE
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def batch(self):
+        return self.q_bits.shape[0]
+
+    @property
+    def num_q_heads(self):
+        return self.q_bits.shape[1]
+
+    @property
+    def head_dim(self):
+        return self.q_bits.shape[2]
+
+    @property
+    def num_kv_heads(self):
+        return self.k_pages_bits.shape[2] if self.layout == "NHD" else self.k_pages_bits.shape[1]
+
+    @property
+    def num_pages(self):
+        return self.k_pages_bits.shape[0]
+
+    def strides(self):
+        """(page_stride, token_stride, head_stride) in elements."""
+        P, a, b, d = self.k_pages_bits.shape
+        if self.layout == "NHD":
+            return a * b * d, b * d, d
+        return a * b * d, d, b * d
+
+    def kv_bytes(self) -> float:
+        """Bytes of K and V the decode must read: every cached token once."""
+        return 2.0 * float(self.cache_seqlens.astype(np.int64).sum()) * self.num_kv_heads * self.head_dim * 2
+
+    def algorithmic_bytes(self) -> float:
+        """KV read once + q read + out/lse written + block_table entries used."""
+        B, Hq, d = self.q_bits.shape
+        pages_used = int(np.sum((self.cache_seqlens.astype(np.int64) + self.page_size - 1) // self.page_size))
+        return self.kv_bytes() + B * Hq * d * 2 * 2 + B * Hq * 4 + pages_used * 4 + B * 4
+
+
+def make_decode(cache_seqlens, num_q_heads, num_kv_heads, head_dim, *, seed=3,
+                page_size=PAGE_SIZE, layout="NHD", scale=None, extra_pages=0,
+                name="decode") -> DecodeInputs:
+    """Paged KV cache whose physical pages are a seeded random permutation.
+
+    Request b owns ceil(seqlen_b / page_size) logical pages; the physical page
+    for each logical page comes from a random permutation of the pool.  The pool
+    is drawn i.i.d. N(0,1), which is the same distribution as drawing each
+    request's logical K/V and scattering it.  ``extra_pages`` adds pool pages
+    that no request uses.
+    """
+    cache_seqlens = np.asarray(cache_seqlens, dtype=np.int64)
+    B = len(cache_seqlens)
+    npages = (cache_seqlens + page_size - 1) // page_size
+    total = int(npages.sum()) + int(extra_pages)
+    ss = np.random.SeedSequence(seed)
+    s_perm, s_q, s_k, s_v = ss.spawn(4)
+    perm = np.random.Generator(np.random.PCG64(s_perm)).permutation(total).astype(np.int32)
+    max_pages = int(max(1, npages.max()))
+    bt = np.full((B, max_pages), -1, dtype=np.int32)
+    off = 0
+    for b in range(B):
+        n = int(npages[b])
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    if layout == "NHD":
+        shape = (total, page_size, num_kv_heads, head_dim)
+    elif layout == "HND":
+        shape = (total, num_kv_heads, page_size, head_dim)
+    else:
+        raise ValueError(layout)
+    q = _normal_bf16_bits(s_q, (B, num_q_heads, head_dim))
+    kp = _normal_bf16_bits(s_k, shape)
+    vp = _normal_bf16_bits(s_v, shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    return DecodeInputs(name, q, kp, vp, bt, cache_seqlens.astype(np.int32), float(scale),
+                        layout, page_size)
+
+
+def paged_decode_batch() -> DecodeInputs:
+    """64 requests, cache lengths uniform in [1024, 32768], 32 q / 8 kv heads, d=128."""
+    lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=64)
+    return make_decode(lens, 32, 8, 128, seed=3, name="paged_decode_batch")
+
+
+def long_split_decode() -> DecodeInputs:
+    """4 requests of 131072 cached tokens, 32 heads MHA, d=128, shuffled pages."""
+    return make_decode([131072] * 4, 32, 32, 128, seed=4, name="long_split_decode")
+
+
+def ragged_split_decode() -> DecodeInputs:
+    """1 request at 131072 plus 63 at 2048 tokens, 32 heads MHA, d=128."""
+    return make_decode([131072] + [2048] * 63, 32, 32, 128, seed=5, name="ragged_split_decode")
+
+
+def relayout(inp: DecodeInputs, layout: str) -> DecodeInputs:
+    """Same cache contents in the other page layout (NHD <-> HND)."""
+    if layout == inp.layout:
+        return inp
+    kp = np.ascontiguousarray(np.swapaxes(inp.k_pages_bits, 1, 2))
+    vp = np.ascontiguousarray(np.swapaxes(inp.v_pages_bits, 1, 2))
+    return DecodeInputs(inp.name + "_" + layout, inp.q_bits, kp, vp, inp.block_table,
+                        inp.cache_seqlens, inp.scale, layout, inp.page_size, dict(inp.extra))
+
+
+def permute_pages(inp: DecodeInputs, seed: int) -> DecodeInputs:
+    """Move every physical page to a new random slot and rewrite the block table."""
+    P = inp.num_pages
+    perm = np.random.default_rng(seed).permutation(P).astype(np.int32)   # old -> new
+    kp = np.empty_like(inp.k_pages_bits)
+    vp = np.empty_like(inp.v_pages_bits)
+    kp[perm] = inp.k_pages_bits
+    vp[perm] = inp.v_pages_bits
+    bt = inp.block_table.copy()
+    used = bt >= 0
+    bt[used] = perm[bt[used]]
+    return DecodeInputs(inp.name + "_perm", inp.q_bits, kp, vp, bt, inp.cache_seqlens,
+                        inp.scale, inp.layout, inp.page_size, dict(inp.extra))
+
+
+BF16_NAN_BITS = 0x7FC0
+
+
+def poison_unused(inp: DecodeInputs) -> DecodeInputs:
+    """Fill every cache slot no request reads (page tails, unused pages) with NaN."""
+    kp = inp.k_pages_bits.copy()
+    vp = inp.v_pages_bits.copy()
+    P = inp.num_pages
+    ps = inp.page_size
+    valid = np.zeros((P, ps), dtype=bool)
+    for b in range(inp.batch):
+        L = int(inp.cache_seqlens[b])
+        for p in range((L + ps - 1) // ps):
+            phys = int(inp.block_table[b, p])
+            n = min(ps, L - p * ps)
+            valid[phys, :n] = True
+    inv = ~valid
+    if inp.layout == "NHD":
+        kp[inv] = BF16_NAN_BITS
+        vp[inv] = BF16_NAN_BITS
+    else:
+        kp.transpose(0, 2, 1, 3)[inv] = BF16_NAN_BITS
+        vp.transpose(0, 2, 1, 3)[inv] = BF16_NAN_BITS
+    return DecodeInputs(inp.name + "_poison", inp.q_bits, kp, vp, inp.block_table,
+                        inp.cache_seqlens, inp.scale, inp.layout, inp.page_size, dict(inp.extra))
+
+
+CONFIGS = {
+    "tiny_causal_prefill": tiny_causal_prefill,
+    "varlen_causal_prefill": varlen_causal_prefill,
+    "long_gqa_prefill": long_gqa_prefill,
+    "paged_decode_batch": paged_decode_batch,
+    "long_split_decode": long_split_decode,
+    "ragged_split_decode": ragged_split_decode,
+}
