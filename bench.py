@@ -1,0 +1,526 @@
+#!/usr/bin/env python3
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  1. causal varlen prefill (8 sequences, lengths U[512, 4096], 32 heads, d=128)
+     through fa_prefill, then
+  2. Flash-Decoding of a paged batch (64 requests, cache lengths U[1024, 32768],
+     32 q / 8 kv heads, d=128, shuffled 64-token pages) through fa_decode_plan's
+     plan and fa_decode_paged (split kernel + merge kernel).
+The line's ``value`` is the prefill throughput in TFLOP/s (causal algorithmic
+FLOPs); the decode half reports HBM GB/s under ``decode``.  ``--workload``
+selects a single configuration instead (one line for that configuration).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch under torch.distributed.run; every rank runs an independent
+replica of the step (no collective on the data path; "replicas only").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "causal prefill TFLOP/s and paged-decode HBM GB/s on 1 B200 vs roofline"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill"}
+DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- device inputs
+
+def _dev_bf16(bits, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def _dev_i32(a, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(np.asarray(a, dtype=np.int32))).to(device)
+
+
+class PrefillCase:
+    def __init__(self, inp: W.PrefillInputs, device):
+        import torch
+        self.inp = inp
+        self.q = _dev_bf16(inp.q_bits, device)
+        self.k = _dev_bf16(inp.k_bits, device)
+        self.v = _dev_bf16(inp.v_bits, device)
+        self.cu = _dev_i32(inp.cu_seqlens, device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=device)
+        self.flops = inp.causal_flops()
+        self.launches = -(-sum(-(-int(L) // 128) for L in inp.seqlens) // 2048)
+        # pinned host copies for the end-to-end leg
+        self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
+        self.h_k = torch.from_numpy(inp.k_bits.view(np.int16)).pin_memory()
+        self.h_v = torch.from_numpy(inp.v_bits.view(np.int16)).pin_memory()
+        self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def run(self):
+        import exact_attention_148_b200 as fa
+        fa.prefill(self.q, self.k, self.v, self.cu, causal=self.inp.causal, scale=self.inp.scale,
+                   out=self.out, lse=self.lse, cu_seqlens_host=self.inp.cu_seqlens)
+
+    def run_e2e(self):
+        """Host buffers in, host buffers out: H2D copies, the C-ABI call, D2H copies."""
+        import torch
+        self.q.view(torch.int16).copy_(self.h_q, non_blocking=True)
+        self.k.view(torch.int16).copy_(self.h_k, non_blocking=True)
+        self.v.view(torch.int16).copy_(self.h_v, non_blocking=True)
+        self.run()
+        self.h_out.copy_(self.out.view(torch.int16), non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def h2d_bytes(self):
+        return 2 * (self.inp.q_bits.size + self.inp.k_bits.size + self.inp.v_bits.size) + \
+            4 * self.inp.cu_seqlens.size
+
+    def d2h_bytes(self):
+        return 2 * self.inp.q_bits.size + 4 * self.lse.numel()
+
+    def describe(self):
+        i = self.inp
+        return {"workload": i.name, "batch": int(len(i.seqlens)), "seqlens_total": int(i.seqlens.sum()),
+                "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads,
+                "head_dim": i.head_dim, "causal": bool(i.causal),
+                "algorithmic_tflop": round(self.flops / 1e12, 4)}
+
+
+class DecodeCase:
+    def __init__(self, inp: W.DecodeInputs, device, num_splits=0):
+        import torch
+        import exact_attention_148_b200 as fa
+        self.inp = inp
+        self.q = _dev_bf16(inp.q_bits, device)
+        self.kp = _dev_bf16(inp.k_pages_bits, device)
+        self.vp = _dev_bf16(inp.v_pages_bits, device)
+        self.bt = _dev_i32(inp.block_table, device)
+        self.lens = _dev_i32(inp.cache_seqlens, device)
+        t0 = time.perf_counter()
+        self.plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=inp.num_q_heads,
+                                   num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
+                                   page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
+                                   num_splits=num_splits)
+        self.plan_ms = (time.perf_counter() - t0) * 1e3
+        self.ws = torch.empty(max(self.plan.workspace_bytes, 256), dtype=torch.uint8, device=device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=device)
+        self.bytes = inp.algorithmic_bytes()
+        self.launches = 1 + (1 if self.plan.info.max_splits > 1 else 0)
+        self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
+        self.h_k = torch.from_numpy(inp.k_pages_bits.view(np.int16)).pin_memory()
+        self.h_v = torch.from_numpy(inp.v_pages_bits.view(np.int16)).pin_memory()
+        self.h_bt = torch.from_numpy(inp.block_table).pin_memory()
+        self.h_lens = torch.from_numpy(inp.cache_seqlens).pin_memory()
+        self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def run(self):
+        import exact_attention_148_b200 as fa
+        fa.decode_paged(self.q, self.kp, self.vp, self.bt, self.lens, self.plan, layout=self.inp.layout,
+                        scale=self.inp.scale, out=self.out, lse=self.lse, workspace=self.ws)
+
+    def run_e2e(self):
+        import torch
+        self.q.view(torch.int16).copy_(self.h_q, non_blocking=True)
+        self.kp.view(torch.int16).copy_(self.h_k, non_blocking=True)
+        self.vp.view(torch.int16).copy_(self.h_v, non_blocking=True)
+        self.bt.copy_(self.h_bt, non_blocking=True)
+        self.lens.copy_(self.h_lens, non_blocking=True)
+        self.run()
+        self.h_out.copy_(self.out.view(torch.int16), non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def h2d_bytes(self):
+        i = self.inp
+        return 2 * (i.q_bits.size + i.k_pages_bits.size + i.v_pages_bits.size) + \
+            4 * (i.block_table.size + i.cache_seqlens.size)
+
+    def d2h_bytes(self):
+        return 2 * self.inp.q_bits.size + 4 * self.lse.numel()
+
+    def describe(self):
+        i = self.inp
+        info = self.plan.info
+        return {"workload": i.name, "batch": i.batch, "cache_tokens_total": int(i.cache_seqlens.sum()),
+                "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads, "head_dim": i.head_dim,
+                "page_size": i.page_size, "layout": i.layout, "chunk_tokens": info.chunk_tokens,
+                "max_splits": info.max_splits, "work_items": info.num_work_items,
+                "plan_ms": round(self.plan_ms, 3), "algorithmic_gb": round(self.bytes / 1e9, 4)}
+
+
+# ----------------------------------------------------------------------------- timing
+
+def time_cases(cases, steps, warmup, flush, dist_ctx, e2e=False):
+    """Per case: total device ms over `steps` timed steps (each case of a step
+    bracketed by its own CUDA events on the current stream; L2 flushed before
+    every step outside the events).  Returns (per-case ms list, total ms)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for c in cases:
+            (c.run_e2e if e2e else c.run)()
+    torch.cuda.synchronize()
+    if dist_ctx is not None:
+        dist_ctx.barrier()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in cases] for _ in range(steps)]
+    for s in range(steps):
+        flush.zero_()
+        for ci, c in enumerate(cases):
+            evs[s][ci][0].record(stream)
+            (c.run_e2e if e2e else c.run)()
+            evs[s][ci][1].record(stream)
+    torch.cuda.synchronize()
+    if dist_ctx is not None:
+        dist_ctx.barrier()
+    torch.cuda.synchronize()
+    per_case = [sum(evs[s][ci][0].elapsed_time(evs[s][ci][1]) for s in range(steps)) for ci in range(len(cases))]
+    if dist_ctx is not None:
+        per_case = dist_ctx.max_over_ranks(per_case)
+    return per_case
+
+
+class DistCtx:
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        self.dist = dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+        self.rank = dist.get_rank()
+        self.world = dist.get_world_size()
+        self.local = int(os.environ.get("LOCAL_RANK", 0))
+        torch.cuda.set_device(self.local)
+
+    def barrier(self):
+        self.dist.barrier()
+
+    def max_over_ranks(self, vals):
+        import torch
+        t = torch.tensor(vals, dtype=torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return t.tolist()
+
+    def close(self):
+        self.dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(inp: W.PrefillInputs, budget_s: float):
+    """Run the oracle on whole (sequence, head) blocks until about budget_s has
+    passed; returns (flops done, seconds, description)."""
+    import oracle
+    order = np.argsort(inp.seqlens)          # shortest sequences first
+    flops, secs, done = 0.0, 0.0, []
+    d = inp.head_dim
+    for b in order:
+        s0, s1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
+        L = s1 - s0
+        g = 0
+        q = W.as_f64(inp.q_bits[s0:s1, 0:1])
+        k = W.as_f64(inp.k_bits[s0:s1, g:g + 1])
+        v = W.as_f64(inp.v_bits[s0:s1, g:g + 1])
+        t0 = time.perf_counter()
+        oracle.attention_ref(q, k, v, [0, L], inp.causal, inp.scale)
+        secs += time.perf_counter() - t0
+        pairs = L * (L + 1) // 2 if inp.causal else L * L
+        flops += 4.0 * d * pairs
+        done.append(L)
+        if secs >= budget_s:
+            break
+    return flops, secs, f"oracle attention_ref on head 0 of sequences with lengths {done}"
+
+
+def oracle_decode_sample(inp: W.DecodeInputs, budget_s: float):
+    import oracle
+    flops_bytes, secs, rows = 0.0, 0.0, []
+    G = inp.num_q_heads // inp.num_kv_heads
+    for b in range(inp.batch):
+        rws = [(b, h) for h in range(0, inp.num_q_heads, G)][:2]   # two kv heads' first q head
+        t0 = time.perf_counter()
+        oracle.paged_decode_rows_ref(inp.q_bits, inp.k_pages_bits, inp.v_pages_bits, inp.block_table,
+                                     inp.cache_seqlens, inp.scale, rws, inp.page_size, inp.layout,
+                                     to_f64=W.as_f64)
+        secs += time.perf_counter() - t0
+        flops_bytes += len(rws) * 2.0 * int(inp.cache_seqlens[b]) * inp.head_dim * 2
+        rows.append(b)
+        if secs >= budget_s:
+            break
+    return flops_bytes, secs, f"oracle paged_decode_rows_ref, 2 kv heads of requests {rows}"
+
+
+# ----------------------------------------------------------------------------- main
+
+def build_cases(workload, device, num_splits):
+    if workload == "default":
+        return [PrefillCase(W.varlen_causal_prefill(), device), DecodeCase(W.paged_decode_batch(), device)]
+    if workload in PREFILL_WORKLOADS:
+        return [PrefillCase(W.CONFIGS[workload](), device)]
+    if workload in DECODE_WORKLOADS:
+        return [DecodeCase(W.CONFIGS[workload](), device, num_splits)]
+    raise SystemExit(f"unknown workload {workload}")
+
+
+def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=None):
+    if kind == "tensor":
+        achieved = algorithmic / (ms_per_launch * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "frac_of_spec": round(achieved / SPEC_PEAKS["bf16_tflops"], 4)}
+    achieved = algorithmic / (ms_per_launch * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": f"{peak_src} HBM copy", "frac_of_spec": round(achieved / SPEC_PEAKS["hbm_gbs"], 4)}
+
+
+def run_ours(args):
+    import torch
+    import exact_attention_148_b200 as fa  # noqa: F401  (fails loudly if the library is missing)
+    fa.library()
+    dist_ctx = DistCtx() if args.gpus > 1 else None
+    rank = dist_ctx.rank if dist_ctx else 0
+    device = torch.device("cuda", dist_ctx.local if dist_ctx else 0)
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+    cases = build_cases(args.workload, device, args.num_splits)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler.start()
+    per_case = time_cases(cases, args.steps, args.warmup, flush, dist_ctx)
+    clocks = sampler.stop()
+    status = fa.device_status(clear=True)
+
+    e2e_case = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 5))
+        e2e_case = time_cases(cases, e2e_steps, 1, flush, dist_ctx, e2e=True)
+        e2e_case = [x / e2e_steps for x in e2e_case]
+
+    N = args.gpus
+    ms_case = [x / args.steps for x in per_case]
+    ms_step = sum(ms_case)
+    line = {"metric": METRIC}
+    launches = sum(c.launches for c in cases) * args.steps
+    main = cases[0]
+    if isinstance(main, PrefillCase):
+        value = N * main.flops / (ms_case[0] * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        rl = roofline_entry("tensor", main.flops, ms_case[0] / main.launches, peaks, peak_src)
+    else:
+        value = N * main.bytes / (ms_case[0] * 1e-3) / 1e9
+        unit = "GB/s"
+        rl = roofline_entry("hbm", main.bytes, ms_case[0], peaks, peak_src)
+    line.update({"value": round(value, 3), "unit": unit, "n_gpus": N, "steps": args.steps,
+                 "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                 "data": "synthetic (seeded N(0,1) rounded to bf16; see workloads/)"})
+    cfg = {"workload": " + ".join(c.inp.name for c in cases),
+           "l2": "flushed before every step (256 MiB write), outside the timed events; "
+                 "inputs also exceed L2",
+           "parallelism": f"replicas x{N}" if N > 1 else "single GPU"}
+    for i, c in enumerate(cases):
+        cfg["prefill" if isinstance(c, PrefillCase) else "decode"] = c.describe()
+    line["config"] = cfg
+    line["roofline"] = rl
+    if len(cases) > 1:
+        dc = cases[1]
+        line["decode"] = {"value": round(N * dc.bytes / (ms_case[1] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                          "ms": round(ms_case[1], 4),
+                          "roofline": roofline_entry("hbm", dc.bytes, ms_case[1], peaks, peak_src),
+                          "timed_over": "fa_decode_paged call (split kernel + merge kernel)"}
+        line["prefill_ms"] = round(ms_case[0], 4)
+    if e2e_case is not None:
+        if isinstance(main, PrefillCase):
+            e2e_v = N * main.flops / (e2e_case[0] * 1e-3) / 1e12
+        else:
+            e2e_v = N * main.bytes / (e2e_case[0] * 1e-3) / 1e9
+        line["e2e"] = {"value": round(e2e_v, 3), "unit": unit,
+                       "h2d_bytes_per_step": int(sum(c.h2d_bytes() for c in cases)),
+                       "d2h_bytes_per_step": int(sum(c.d2h_bytes() for c in cases)),
+                       "ms_per_step": round(sum(e2e_case), 3),
+                       "path": "pinned host -> device copies, C-ABI calls, device -> pinned host copies"}
+    line["gpu_launches"] = int(launches)
+    line["clocks"] = clocks
+    line["device_status"] = status
+    if rank == 0 and N == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(main, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_ctx is not None:
+        dist_ctx.close()
+
+
+def cpu_baseline(case, budget):
+    threads = blas_threads()
+    if isinstance(case, PrefillCase):
+        work, secs, desc = oracle_prefill_sample(case.inp, budget)
+        val, unit = work / secs / 1e12, "TFLOP/s"
+    else:
+        work, secs, desc = oracle_decode_sample(case.inp, budget)
+        val, unit = work / secs / 1e9, "GB/s"
+    return {"value": val, "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": f"{desc}; {secs:.1f} s of CPU time"}
+
+
+def run_reference(args):
+    """The oracle, as it stands, timed on the host cores on a bounded sample
+    of the same workload (rank 0 only; other ranks exit without work)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    main = args.workload
+    if main == "default":
+        inp = W.varlen_causal_prefill()
+        is_prefill = True
+    elif main in PREFILL_WORKLOADS:
+        inp = W.CONFIGS[main]()
+        is_prefill = True
+    else:
+        inp = W.CONFIGS[main]()
+        is_prefill = False
+    per_step = max(1.0, args.cpu_budget / max(1, args.steps))
+    fn = oracle_prefill_sample if is_prefill else oracle_decode_sample
+    for _ in range(args.warmup and 1):
+        fn(inp, 0.0)
+    work, secs = 0.0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        w, s, desc = fn(inp, per_step)
+        work += w
+        secs += s
+    if is_prefill:
+        value, unit = work / secs / 1e12, "TFLOP/s"
+    else:
+        value, unit = work / secs / 1e9, "GB/s"
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) rounded to bf16; see workloads/)",
+            "config": {"workload": inp.name if not (main == "default") else
+                       "varlen_causal_prefill + paged_decode_batch (prefill half sampled)"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=int(os.environ.get("WORLD_SIZE", "1")))
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="default",
+                    help="default | " + " | ".join(sorted(PREFILL_WORKLOADS | DECODE_WORKLOADS)))
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

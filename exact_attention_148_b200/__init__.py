@@ -1,0 +1,310 @@
+"""exact_attention_148_b200 — B200 (sm_100a) exact attention forward.
+
+Thin Python binding over the C ABI in ``include/exact_attention.h``: it only
+marshals arguments (device pointers, sizes, the current CUDA stream) into
+``libexact_attention.so``; every step of the computation runs in that
+library's CUDA kernels.  PyTorch provides device memory and streams.
+
+There is no CPU fallback: if the shared library is missing, or a tensor is not
+a CUDA tensor, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+__all__ = [
+    "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
+    "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
+]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG_DIR, "libexact_attention.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = -1
+FA_ERR_UNSUPPORTED = -2
+FA_ERR_WORKSPACE = -3
+FA_ERR_CUDA = -4
+FA_ERR_TIMEOUT = -5
+FA_ERR_PLAN_MISMATCH = -6
+FA_ERR_BAD_PAGE = -7
+
+EXPORTED_SYMBOLS = [
+    "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
+    "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
+]
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = f"{what}: {strerror(status)} ({status})"
+        if status == FA_ERR_CUDA:
+            msg += f", cuda error {library().fa_last_cuda_error()}"
+        super().__init__(msg)
+
+
+class _PlanInfo(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("page_size", ctypes.c_int), ("max_pages_per_seq", ctypes.c_int),
+        ("chunk_tokens", ctypes.c_int), ("max_splits", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
+        ("num_work_items", ctypes.c_int), ("max_seqlen", ctypes.c_int),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load the in-tree shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(lib_path):
+        raise RuntimeError(f"{lib_path} is missing; build it with "
+                           "`python -m exact_attention_148_b200._build`")
+    L = ctypes.CDLL(lib_path)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    L.fa_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp]
+    L.fa_prefill.restype = i32
+    L.fa_decode_plan.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                 ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t)]
+    L.fa_decode_plan.restype = i32
+    L.fa_plan_get_info.argtypes = [vp, ctypes.POINTER(_PlanInfo)]
+    L.fa_plan_get_info.restype = i32
+    L.fa_plan_free.argtypes = [vp]
+    L.fa_plan_free.restype = None
+    L.fa_decode_paged.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, f32, vp, vp, vp,
+                                  ctypes.c_size_t, vp]
+    L.fa_decode_paged.restype = i32
+    L.fa_merge_states.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    L.fa_merge_states.restype = i32
+    L.fa_strerror.argtypes = [i32]
+    L.fa_strerror.restype = ctypes.c_char_p
+    L.fa_last_cuda_error.argtypes = []
+    L.fa_last_cuda_error.restype = i32
+    L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(i32), i32]
+    L.fa_get_device_status.restype = i32
+    L.fa_version.argtypes = []
+    L.fa_version.restype = i32
+    _lib = L
+    return L
+
+
+def strerror(status: int) -> str:
+    return library().fa_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("exact_attention_148_b200 runs on CUDA tensors only "
+                             "(no CPU fallback)")
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _scale_arg(scale):
+    return float("nan") if scale is None else float(scale)
+
+
+# ----------------------------------------------------------------------------- prefill
+
+def prefill(q, k, v, cu_seqlens, *, causal: bool = True, scale: float | None = None,
+            out=None, lse=None, cu_seqlens_host=None, return_lse: bool = True, stream=None):
+    """Exact attention over packed variable-length sequences.
+
+    q [T, Hq, d], k/v [T, Hkv, d] bf16 CUDA tensors (contiguous); cu_seqlens
+    [B+1] int32 CUDA tensor.  Returns (out [T, Hq, d] bf16, lse [T, Hq] fp32 or
+    None).  ``cu_seqlens_host`` (a sequence of ints / numpy array) avoids a
+    device-to-host copy of the offsets.
+    """
+    torch = _torch()
+    _require_cuda(q, k, v, cu_seqlens, out, lse)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous 3-D bfloat16 tensor")
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu().numpy()
+    cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+    batch = len(cu_h) - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    st = library().fa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                              cu_h.ctypes.data_as(ctypes.c_void_p), batch, Hq, Hkv, d,
+                              1 if causal else 0, _scale_arg(scale), _ptr(out), _ptr(lse),
+                              _stream_ptr(stream))
+    _check(st, "fa_prefill")
+    return out, lse
+
+
+# ----------------------------------------------------------------------------- decode
+
+@dataclass
+class PlanInfo:
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    page_size: int
+    max_pages_per_seq: int
+    chunk_tokens: int
+    max_splits: int
+    heads_per_cta: int
+    num_work_items: int
+    max_seqlen: int
+    workspace_bytes: int
+
+
+class DecodePlan:
+    """Host-side split plan (owns an ``fa_plan``; freed with the object)."""
+
+    def __init__(self, handle: ctypes.c_void_p, workspace_bytes: int):
+        self._h = handle
+        self.workspace_bytes = int(workspace_bytes)
+        info = _PlanInfo()
+        _check(library().fa_plan_get_info(self._h, ctypes.byref(info)), "fa_plan_get_info")
+        self.info = PlanInfo(**{f: getattr(info, f) for f, _ in _PlanInfo._fields_})
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            library().fa_plan_free(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def decode_plan(cache_seqlens_host, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                page_size: int = 64, max_pages_per_seq: int, num_sms: int | None = None,
+                num_splits: int = 0) -> DecodePlan:
+    """Plan the split of every request's cached context (host only, no GPU needed
+    when ``num_sms`` is given)."""
+    lens = np.ascontiguousarray(np.asarray(cache_seqlens_host, dtype=np.int32))
+    if num_sms is None:
+        torch = _torch()
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    h = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    st = library().fa_decode_plan(lens.ctypes.data_as(ctypes.c_void_p), len(lens), num_q_heads,
+                                  num_kv_heads, head_dim, page_size, max_pages_per_seq, num_sms,
+                                  num_splits, ctypes.byref(h), ctypes.byref(ws))
+    _check(st, "fa_decode_plan")
+    return DecodePlan(h, ws.value)
+
+
+def page_strides(k_pages, layout: str):
+    """(page_stride, token_stride, head_stride) in elements for NHD / HND pools."""
+    P, a, b, d = k_pages.shape
+    if layout == "NHD":     # [P, page, Hkv, d]
+        return a * b * d, b * d, d
+    if layout == "HND":     # [P, Hkv, page, d]
+        return a * b * d, d, b * d
+    raise ValueError(layout)
+
+
+def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePlan, *,
+                 layout: str = "NHD", scale: float | None = None, out=None, lse=None,
+                 workspace=None, return_lse: bool = True, stream=None):
+    """One query token per request against a paged KV cache (Flash-Decoding).
+
+    q [B, Hq, d] bf16; k_pages/v_pages [P, page, Hkv, d] (NHD) or
+    [P, Hkv, page, d] (HND) bf16; block_table [B, max_pages] int32;
+    cache_seqlens [B] int32 (device).  Returns (out, lse).
+    """
+    torch = _torch()
+    _require_cuda(q, k_pages, v_pages, block_table, cache_seqlens, out, lse, workspace)
+    if k_pages.dtype != torch.bfloat16 or v_pages.dtype != torch.bfloat16 or q.dtype != torch.bfloat16:
+        raise ValueError("q, k_pages and v_pages must be bfloat16")
+    if not (k_pages.is_contiguous() and v_pages.is_contiguous() and q.is_contiguous()
+            and block_table.is_contiguous()):
+        raise ValueError("tensors must be contiguous")
+    if k_pages.shape != v_pages.shape:
+        raise ValueError("k_pages and v_pages must have the same shape")
+    B, Hq, d = q.shape
+    ps, ts, hs = page_strides(k_pages, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None and plan.workspace_bytes > 0:
+        workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
+    st = library().fa_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(block_table),
+        _ptr(cache_seqlens), plan.handle, _scale_arg(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(st, "fa_decode_paged")
+    return out, lse
+
+
+def merge_states(o_parts, lse_parts, *, out=None, lse=None, stream=None):
+    """Merge states by LSE.  o_parts [S, rows, H, d] fp32, lse_parts [S, rows, H] fp32."""
+    torch = _torch()
+    _require_cuda(o_parts, lse_parts, out, lse)
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise ValueError("o_parts and lse_parts must be float32")
+    if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
+        raise ValueError("o_parts and lse_parts must be contiguous")
+    S, R, H, d = o_parts.shape
+    if out is None:
+        out = torch.empty((R, H, d), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((R, H), dtype=torch.float32, device=o_parts.device)
+    st = library().fa_merge_states(_ptr(o_parts), _ptr(lse_parts), S, R, H, d, _ptr(out), _ptr(lse),
+                                   _stream_ptr(stream))
+    _check(st, "fa_merge_states")
+    return out, lse
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    """Synchronise and return (optionally clear) the device status word."""
+    v = ctypes.c_int(0)
+    _check(library().fa_get_device_status(_stream_ptr(stream), ctypes.byref(v), 1 if clear else 0),
+           "fa_get_device_status")
+    return v.value
+
+
+def version() -> int:
+    return library().fa_version()
+
+
+def default_scale(head_dim: int) -> float:
+    return 1.0 / math.sqrt(head_dim)

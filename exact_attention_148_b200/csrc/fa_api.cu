@@ -1,0 +1,395 @@
+// C ABI of the exact-attention library: argument validation, tensor-map
+// construction, tile scheduling and kernel launches (declared in
+// include/exact_attention.h).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "../../include/exact_attention.h"
+#include "decode_sm100.cuh"
+#include "planner.h"
+#include "prefill_sm100.cuh"
+
+#define FA_API extern "C" __attribute__((visibility("default")))
+
+struct fa_plan {
+  fa::DecodePlan p;
+};
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(int code) {
+  t_last_cuda_error = code;
+  return FA_ERR_CUDA;
+}
+
+#define FA_CUDA_CHECK(expr)                          \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) return cuda_fail(e_);     \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+               const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                  strides_bytes, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(static_cast<int>(r) + 10000);
+  return FA_OK;
+}
+
+// cudaFuncSetAttribute once per (kernel, device).
+int ensure_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = 0;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& kv : done)
+    if (kv.first == kernel && kv.second == dev) return FA_OK;
+  FA_CUDA_CHECK(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done.emplace_back(kernel, dev);
+  return FA_OK;
+}
+
+float resolve_scale(float scale, int head_dim) {
+  return std::isnan(scale) ? 1.0f / std::sqrt(static_cast<float>(head_dim)) : scale;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------- prefill
+template <int D>
+int launch_prefill(fa::PrefillParams& prm, const std::vector<uint32_t>& tiles, int num_q_heads,
+                   cudaStream_t stream) {
+  using C = fa::PrefillCfg<D>;
+  auto kernel = fa::fa_prefill_kernel<D>;
+  int st = ensure_smem(reinterpret_cast<const void*>(kernel), C::SMEM_BYTES);
+  if (st != FA_OK) return st;
+  for (size_t off = 0; off < tiles.size(); off += fa::kPrefillMaxTiles) {
+    const int n = static_cast<int>(std::min<size_t>(fa::kPrefillMaxTiles, tiles.size() - off));
+    std::memcpy(prm.tiles, tiles.data() + off, n * sizeof(uint32_t));
+    prm.num_tiles = n;
+    dim3 grid(num_q_heads, n);
+    kernel<<<grid, fa::kPrefillThreads, C::SMEM_BYTES, stream>>>(prm);
+    FA_CUDA_CHECK(cudaGetLastError());
+  }
+  return FA_OK;
+}
+
+// ---------------------------------------------------------------------------- decode
+template <int D, int GC>
+int launch_decode_split(const fa::DecodeParams& prm, dim3 grid, cudaStream_t stream) {
+  using C = fa::DecodeCfg<D, GC>;
+  auto kernel = fa::fa_decode_split_kernel<D, GC>;
+  int st = ensure_smem(reinterpret_cast<const void*>(kernel), C::SMEM_BYTES);
+  if (st != FA_OK) return st;
+  kernel<<<grid, fa::kDecodeThreads, C::SMEM_BYTES, stream>>>(prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}
+
+template <int D>
+int dispatch_decode_gc(int gc, const fa::DecodeParams& prm, dim3 grid, cudaStream_t stream) {
+  switch (gc) {
+    case 1: return launch_decode_split<D, 1>(prm, grid, stream);
+    case 2: return launch_decode_split<D, 2>(prm, grid, stream);
+    case 4: return launch_decode_split<D, 4>(prm, grid, stream);
+    case 8: return launch_decode_split<D, 8>(prm, grid, stream);
+  }
+  return FA_ERR_UNSUPPORTED;
+}
+
+int launch_merge(const fa::MergeParams& mp, int head_dim, cudaStream_t stream) {
+  const int rows = mp.rows * mp.num_heads;
+  dim3 grid((rows + 3) / 4);
+  if (head_dim == 128)
+    fa::fa_merge_kernel<128><<<grid, 128, 0, stream>>>(mp);
+  else
+    fa::fa_merge_kernel<64><<<grid, 128, 0, stream>>>(mp);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}
+
+}  // namespace
+
+// ============================================================================ API
+
+FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
+                      const int32_t* cu_seqlens_host, int batch, int num_q_heads, int num_kv_heads,
+                      int head_dim, int causal, float scale, void* out, float* lse, void* stream) {
+  if (!q || !k || !v || !cu_seqlens_dev || !cu_seqlens_host || !out) return FA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || num_q_heads < 1 || num_kv_heads < 1 ||
+      num_q_heads > 65535 || num_q_heads % num_kv_heads != 0)
+    return FA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4) || !aligned(cu_seqlens_dev, 4))
+    return FA_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, head_dim);
+  if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
+  if (cu_seqlens_host[0] != 0) return FA_ERR_INVALID_ARG;
+  std::vector<std::pair<int, uint32_t>> work;   // (cost, entry)
+  for (int b = 0; b < batch; ++b) {
+    const int64_t L = static_cast<int64_t>(cu_seqlens_host[b + 1]) - cu_seqlens_host[b];
+    if (L < 1) return FA_ERR_INVALID_ARG;
+    const int64_t ntiles = (L + 127) / 128;
+    if (ntiles > 65535) return FA_ERR_UNSUPPORTED;
+    for (int t = 0; t < ntiles; ++t)
+      work.emplace_back(causal ? t + 1 : static_cast<int>(ntiles),
+                        (static_cast<uint32_t>(b) << 16) | static_cast<uint32_t>(t));
+  }
+  const int64_t T = cu_seqlens_host[batch];
+  if (T * num_q_heads * head_dim >= (int64_t{1} << 40)) return FA_ERR_UNSUPPORTED;
+  // Heaviest tiles first so the block scheduler's greedy fill ends with short
+  // tiles (longest-processing-time order); ties keep sequence/tile order.
+  std::stable_sort(work.begin(), work.end(),
+                   [](const auto& a, const auto& b) { return a.first > b.first; });
+  std::vector<uint32_t> tiles(work.size());
+  for (size_t i = 0; i < work.size(); ++i) tiles[i] = work[i].second;
+
+  static thread_local fa::PrefillParams prm;   // ~8.6 KB; kept off the stack
+  std::memset(&prm, 0, sizeof(prm));
+  const cuuint32_t box[3] = {64, 1, 128};
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                                static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                   static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+    int st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),
+                                static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                   static_cast<cuuint64_t>(num_kv_heads) * head_dim * 2};
+    int st = encode_map(&prm.tm_k, k, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+    st = encode_map(&prm.tm_v, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.cu_seqlens = cu_seqlens_dev;
+  prm.num_q_heads = num_q_heads;
+  prm.group = num_q_heads / num_kv_heads;
+  prm.causal = causal ? 1 : 0;
+  prm.scale_log2 = scale * kLog2e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128) return launch_prefill<128>(prm, tiles, num_q_heads, s);
+  return launch_prefill<64>(prm, tiles, num_q_heads, s);
+}
+
+FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                          int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                          int num_sms, int num_splits_override, fa_plan** plan_out,
+                          size_t* workspace_bytes) {
+  if (plan_out == nullptr) return FA_ERR_INVALID_ARG;
+  *plan_out = nullptr;
+  fa::DecodePlan p;
+  int st = fa::make_decode_plan(cache_seqlens_host, batch, num_q_heads, num_kv_heads, head_dim,
+                                page_size, max_pages_per_seq, num_sms, num_splits_override, &p);
+  if (st != FA_OK) return st;
+  fa_plan* plan = new (std::nothrow) fa_plan;
+  if (plan == nullptr) return FA_ERR_INVALID_ARG;
+  plan->p = std::move(p);
+  *plan_out = plan;
+  if (workspace_bytes) *workspace_bytes = plan->p.workspace_bytes;
+  return FA_OK;
+}
+
+FA_API int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info) {
+  if (plan == nullptr || info == nullptr || plan->p.magic != fa::kPlanMagic) return FA_ERR_INVALID_ARG;
+  const auto& p = plan->p;
+  info->batch = p.batch;
+  info->num_q_heads = p.num_q_heads;
+  info->num_kv_heads = p.num_kv_heads;
+  info->head_dim = p.head_dim;
+  info->page_size = p.page_size;
+  info->max_pages_per_seq = p.max_pages_per_seq;
+  info->chunk_tokens = p.chunk_tokens;
+  info->max_splits = p.max_splits;
+  info->heads_per_cta = p.heads_per_cta;
+  info->num_work_items = p.num_work_items;
+  info->max_seqlen = p.max_seqlen;
+  info->workspace_bytes = p.workspace_bytes;
+  return FA_OK;
+}
+
+FA_API void fa_plan_free(fa_plan* plan) {
+  if (plan != nullptr) {
+    plan->p.magic = 0;
+    delete plan;
+  }
+}
+
+FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                           int64_t page_stride, int64_t token_stride, int64_t head_stride,
+                           const int32_t* block_table, const int32_t* cache_seqlens_dev,
+                           const fa_plan* plan, float scale, void* out, float* lse, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (plan == nullptr || plan->p.magic != fa::kPlanMagic) return FA_ERR_INVALID_ARG;
+  const fa::DecodePlan& pl = plan->p;
+  if (!q || !k_pages || !v_pages || !block_table || !cache_seqlens_dev || !out)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4) || !aligned(block_table, 4) || !aligned(cache_seqlens_dev, 4))
+    return FA_ERR_INVALID_ARG;
+  if (num_pages < 1 || num_pages > INT32_MAX) return FA_ERR_INVALID_ARG;
+  if (page_stride <= 0 || token_stride <= 0 || head_stride <= 0 || page_stride % 8 ||
+      token_stride % 8 || head_stride % 8)
+    return FA_ERR_INVALID_ARG;
+  if (pl.workspace_bytes > 0) {
+    if (workspace == nullptr || !aligned(workspace, 256)) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < pl.workspace_bytes) return FA_ERR_WORKSPACE;
+  }
+  scale = resolve_scale(scale, pl.head_dim);
+  if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
+
+  static thread_local fa::DecodeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  // 4-D map over the pool: dim 0 = d (contiguous); dims 1..3 = token slot,
+  // kv head, page, ordered by increasing stride.
+  struct Dim { int64_t stride; int64_t extent; int role; };   // role 0 token, 1 head, 2 page
+  Dim dd[3] = {{token_stride, pl.page_size, 0}, {head_stride, pl.num_kv_heads, 1},
+               {page_stride, num_pages, 2}};
+  std::sort(dd, dd + 3, [](const Dim& a, const Dim& b) { return a.stride < b.stride; });
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(pl.head_dim), 0, 0, 0};
+  cuuint64_t strides[3];
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(pl.head_dim), 1, 1, 1};
+  for (int i = 0; i < 3; ++i) {
+    dims[i + 1] = static_cast<cuuint64_t>(dd[i].extent);
+    strides[i] = static_cast<cuuint64_t>(dd[i].stride) * 2;
+    if (dd[i].role == 0) box[i + 1] = fa::kDecodePage;
+    if (dd[i].role == 1) prm.head_coord = i + 1;
+    if (dd[i].role == 2) prm.page_coord = i + 1;
+  }
+  int st = encode_map(&prm.tm_k, k_pages, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != FA_OK) return st;
+  st = encode_map(&prm.tm_v, v_pages, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != FA_OK) return st;
+
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.block_table = block_table;
+  prm.cache_seqlens = cache_seqlens_dev;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.ws_o = pl.workspace_bytes ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.ws_o_offset)
+                                : nullptr;
+  prm.ws_lse = pl.workspace_bytes
+                   ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.ws_lse_offset)
+                   : nullptr;
+  prm.batch = pl.batch;
+  prm.num_q_heads = pl.num_q_heads;
+  prm.group = pl.group;
+  prm.subgroups = pl.subgroups;
+  prm.max_pages = pl.max_pages_per_seq;
+  prm.num_pages = static_cast<int>(num_pages);
+  prm.chunk_tokens = pl.chunk_tokens;
+  prm.max_splits = pl.max_splits;
+  prm.scale_log2 = scale * kLog2e;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(pl.max_splits, pl.num_kv_heads * pl.subgroups, pl.batch);
+  st = pl.head_dim == 128 ? dispatch_decode_gc<128>(pl.heads_per_cta, prm, grid, s)
+                          : dispatch_decode_gc<64>(pl.heads_per_cta, prm, grid, s);
+  if (st != FA_OK) return st;
+  if (pl.max_splits > 1) {
+    fa::MergeParams mp;
+    mp.o_parts = prm.ws_o;
+    mp.lse_parts = prm.ws_lse;
+    mp.out = prm.out;
+    mp.lse = lse;
+    mp.cache_seqlens = cache_seqlens_dev;
+    mp.num_states = pl.max_splits;
+    mp.rows = pl.batch;
+    mp.num_heads = pl.num_q_heads;
+    mp.chunk_tokens = pl.chunk_tokens;
+    mp.max_pages = pl.max_pages_per_seq;
+    st = launch_merge(mp, pl.head_dim, s);
+  }
+  return st;
+}
+
+FA_API int fa_merge_states(const float* o_parts, const float* lse_parts, int num_states, int rows,
+                           int num_heads, int head_dim, void* out, float* lse, void* stream) {
+  if (!o_parts || !lse_parts || !out) return FA_ERR_INVALID_ARG;
+  if (num_states < 1 || rows < 1 || num_heads < 1) return FA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(rows) * num_heads > INT32_MAX / 4) return FA_ERR_UNSUPPORTED;
+  fa::MergeParams mp;
+  mp.o_parts = o_parts;
+  mp.lse_parts = lse_parts;
+  mp.out = static_cast<__nv_bfloat16*>(out);
+  mp.lse = lse;
+  mp.cache_seqlens = nullptr;
+  mp.num_states = num_states;
+  mp.rows = rows;
+  mp.num_heads = num_heads;
+  mp.chunk_tokens = 1;
+  mp.max_pages = 0;
+  return launch_merge(mp, head_dim, static_cast<cudaStream_t>(stream));
+}
+
+FA_API const char* fa_strerror(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_WORKSPACE: return "workspace too small";
+    case FA_ERR_CUDA: return "CUDA call failed";
+    case FA_ERR_TIMEOUT: return "device wait timed out";
+    case FA_ERR_PLAN_MISMATCH: return "plan does not cover the call";
+    case FA_ERR_BAD_PAGE: return "block_table entry outside the page pool";
+  }
+  return "unknown status";
+}
+
+FA_API int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+FA_API int fa_get_device_status(void* stream, int* status_host, int clear) {
+  if (status_host == nullptr) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FA_CUDA_CHECK(cudaStreamSynchronize(s));
+  int v = 0;
+  FA_CUDA_CHECK(cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(int)));
+  if (clear) {
+    const int zero = 0;
+    FA_CUDA_CHECK(cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(int)));
+  }
+  *status_host = v;
+  return FA_OK;
+}
+
+FA_API int fa_version(void) { return 100; }

@@ -1,0 +1,40 @@
+// Host-side decode planner: chooses how each request's cached context is split
+// across CTAs (Flash-Decoding's split along the sequence, sized from the SM
+// count as the "plan" stage of wsisp.com "FIA / FlashAttention", section 二
+// describes: preprocess the variable lengths, balance the load, assign blocks).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <vector>
+
+namespace fa {
+
+constexpr uint32_t kPlanMagic = 0xFA148D0Cu;
+constexpr int kMaxSplits = 128;
+constexpr int kMinChunkTokens = 512;
+constexpr int kDecodeCtasPerSm = 2;
+constexpr int kItemsPerSlot = 8;   // target work items per resident CTA slot
+
+struct DecodePlan {
+  uint32_t magic = kPlanMagic;
+  int batch = 0, num_q_heads = 0, num_kv_heads = 0, head_dim = 0;
+  int page_size = 0, max_pages_per_seq = 0, num_sms = 0;
+  int group = 1;          // Hq / Hkv
+  int heads_per_cta = 1;  // GC: largest of 8, 4, 2, 1 dividing the group
+  int subgroups = 1;      // group / GC
+  int chunk_tokens = 0;
+  int max_splits = 1;
+  int max_seqlen = 0;
+  int num_work_items = 0;
+  size_t ws_o_offset = 0, ws_lse_offset = 0, workspace_bytes = 0;
+  std::vector<int32_t> seqlens;   // planned cache lengths
+};
+
+// Returns an fa_status.  Pure host code (no CUDA calls).
+int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                     int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                     int num_sms, int num_splits_override, DecodePlan* plan);
+
+}  // namespace fa

@@ -1,0 +1,188 @@
+/*
+ * exact_attention.h — C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * What is computed (wsisp.com "FIA / FlashAttention", section 一):
+ *     O = softmax(Q K^T * scale) V,   LSE = ln sum_j exp(scale * q.k_j)   per query row,
+ * by tiling with an online softmax so the score matrix never reaches HBM
+ * (cloud.baidu.com "FasterTransformer与FlashAttention的联系与区别", section 三,
+ * tiling pseudocode; niuteng5618.github.io "Flash Attention & Paged Attention",
+ * section 1).  Decode follows Flash-Decoding over a paged KV cache (same page,
+ * section "FA对decode阶段的影响" and section 2): the cached context of each request
+ * is split across SMs, each split emits a partial (O_i, LSE_i), and a light
+ * merge kernel reduces them.  The plan/run split follows wsisp.com, sections 二
+ * and 四 (plan does load balancing, run executes).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_host are host memory; every other pointer is device
+ *     memory on the current CUDA device.  The caller owns all memory,
+ *     including the decode workspace; the library never allocates device
+ *     memory.  The only library-owned object is the host-side fa_plan.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns (2 bytes per element).
+ *   - Device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is only enqueued; nothing synchronises the host, so a run can be
+ *     captured into a CUDA graph after its inputs' host-side shape data is fixed.
+ *   - Every function returns an fa_status.  Arguments are validated on the host
+ *     before any launch; on error nothing is enqueued.  FA_ERR_CUDA means a CUDA
+ *     runtime call failed (fa_last_cuda_error() gives the cudaError_t value).
+ *   - A kernel that finds bad device-side data (a page id outside the pool, a
+ *     cache length beyond what its plan covers) or a wait that exceeds its
+ *     bound records a code in a per-device status word; read it with
+ *     fa_get_device_status().  Kernels never trap.
+ */
+#ifndef EXACT_ATTENTION_H_
+#define EXACT_ATTENTION_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, bad size or count */
+  FA_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. head_dim 96) */
+  FA_ERR_WORKSPACE = -3,     /* decode workspace smaller than the plan needs */
+  FA_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = -5,       /* (device status) a bounded wait gave up */
+  FA_ERR_PLAN_MISMATCH = -6, /* plan does not match the call's shapes, or a
+                                device cache length exceeds what it covers */
+  FA_ERR_BAD_PAGE = -7       /* (device status) block_table entry outside the pool */
+} fa_status;
+
+/* Opaque host-side decode plan, created by fa_decode_plan, freed by fa_plan_free. */
+typedef struct fa_plan fa_plan;
+
+/* Read-only view of a plan (for tests and tools). */
+typedef struct {
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int page_size;
+  int max_pages_per_seq;
+  int chunk_tokens;      /* keys per split; a multiple of page_size */
+  int max_splits;        /* splits of the longest planned request */
+  int heads_per_cta;     /* query heads of one kv head packed into a CTA */
+  int num_work_items;    /* non-empty (request, kv-head group, split) items */
+  int max_seqlen;        /* longest planned cache length */
+  size_t workspace_bytes;
+} fa_plan_info;
+
+/*
+ * fa_prefill — causal or full exact attention over packed variable-length
+ * sequences (FA's varlen prefill: wsisp.com "FIA / FlashAttention", sections
+ * 一, 二 and 四; causal=True as in its API example).
+ *
+ *   q    [T, Hq,  d] bf16, row-major (token, head, dim), T = cu_seqlens[batch]
+ *   k, v [T, Hkv, d] bf16, same layout
+ *   cu_seqlens_dev  [batch+1] int32 device; cu_seqlens_host the same values
+ *                   on the host (used to build the tile schedule)
+ *   Query head h reads kv head h / (Hq/Hkv) (GQA/MQA when Hkv < Hq).
+ *   causal != 0: key j is visible to query i of the same sequence iff j <= i.
+ *   scale: score multiplier; NaN means 1/sqrt(d).  Must be > 0 otherwise.
+ *   out  [T, Hq, d] bf16 (written); lse [T, Hq] fp32 natural-log LSE, or NULL.
+ * Supported: d in {64, 128}; Hq % Hkv == 0; each sequence length >= 1;
+ * T < 2^31 / (Hq*d).  Output rows of different sequences never mix.
+ */
+int fa_prefill(const void* q, const void* k, const void* v,
+               const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host, int batch,
+               int num_q_heads, int num_kv_heads, int head_dim, int causal, float scale,
+               void* out, float* lse, void* stream);
+
+/*
+ * fa_decode_plan — host-only split and load-balance planning for paged
+ * decode (the "plan" stage: wsisp.com "FIA / FlashAttention", section 二;
+ * Flash-Decoding's split along the context: niuteng5618.github.io, section
+ * "FA对decode阶段的影响"; num_splits as a hardware knob: rt2005.com
+ * "FlashAttention突破性架构", section 分块矩阵乘法的并行优化).
+ *
+ *   cache_seqlens_host [batch] int32: cached tokens per request (0 allowed).
+ *   page_size: tokens per KV page (64 supported).
+ *   max_pages_per_seq: columns of block_table; each cache length must be
+ *                      <= max_pages_per_seq * page_size (cache overflow check,
+ *                      rt2005.com section 故障诊断与性能监控).
+ *   num_sms: SM count of the target GPU (148 on B200); sizes the splits.
+ *   num_splits_override: 0 = automatic; S > 0 caps every request at S splits
+ *                        (chunk = ceil(max_seqlen / S) rounded up to a page).
+ * On success *plan_out owns a new plan and *workspace_bytes is the device
+ * workspace fa_decode_paged needs (0 when no request is split).
+ * The plan stays valid for later calls whose device cache lengths are not
+ * longer than the planned maximum split coverage (max_splits*chunk_tokens).
+ */
+int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                   int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                   int num_sms, int num_splits_override, fa_plan** plan_out,
+                   size_t* workspace_bytes);
+
+int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info);
+void fa_plan_free(fa_plan* plan);
+
+/*
+ * fa_decode_paged — one query token per request against its paged KV cache
+ * (the "run" stage; Flash-Decoding split kernel + LSE merge kernel).
+ *
+ *   q [batch, Hq, d] bf16.
+ *   k_pages, v_pages: a pool of num_pages pages of page_size tokens; element
+ *       (page p, slot t, kv head g, dim c) is at
+ *       p*page_stride + t*token_stride + g*head_stride + c   (elements).
+ *       NHD layout [P, page, Hkv, d]: strides (page*Hkv*d, Hkv*d, d);
+ *       HND layout [P, Hkv, page, d]: strides (Hkv*page*d, d, page*d).
+ *       All strides must be multiples of 8 elements.
+ *   block_table [batch, max_pages_per_seq] int32: physical page of each
+ *       logical page; entries past a request's last page are never read.
+ *   cache_seqlens_dev [batch] int32 (device copy of the planned lengths, or
+ *       shorter/equal lengths at later steps).
+ *   scale: NaN means 1/sqrt(d).
+ *   out [batch, Hq, d] bf16; lse [batch, Hq] fp32 (or NULL).
+ *   workspace: >= the plan's workspace_bytes, 256-byte aligned (may be NULL
+ *       when that is 0).  It holds the split partials; its contents need no
+ *       initialisation and are dead after the call.
+ * A request with cache length 0 gets O = 0 and LSE = -inf.
+ * The result depends only on logical token order, never on which physical
+ * pages hold them (permuting the pool and the table gives identical bits).
+ */
+int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                    int64_t page_stride, int64_t token_stride, int64_t head_stride,
+                    const int32_t* block_table, const int32_t* cache_seqlens_dev,
+                    const fa_plan* plan, float scale, void* out, float* lse,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_merge_states — combine partial attention states by their LSE (the light
+ * reduction kernel of Flash-Decoding: niuteng5618.github.io, section
+ * "FA对decode阶段的影响", step 4).
+ *
+ *   o_parts   [num_states, rows, num_heads, d] fp32 (each state normalised)
+ *   lse_parts [num_states, rows, num_heads]    fp32 natural-log LSE; -inf marks
+ *             an empty state (zero weight)
+ *   out [rows, num_heads, d] bf16 = sum_i w_i O_i / sum_i w_i, w_i = e^{LSE_i - max}
+ *   lse [rows, num_heads] fp32 = max + ln sum_i w_i, or NULL.
+ * All-empty rows give O = 0, LSE = -inf.  d in {64, 128}; num_states >= 1.
+ */
+int fa_merge_states(const float* o_parts, const float* lse_parts, int num_states, int rows,
+                    int num_heads, int head_dim, void* out, float* lse, void* stream);
+
+/* Human-readable text for an fa_status value (static storage). */
+const char* fa_strerror(int status);
+
+/* cudaError_t of the last failed CUDA call made by this library in this thread. */
+int fa_last_cuda_error(void);
+
+/*
+ * Device status word of the current device: synchronises `stream`, copies the
+ * word into *status_host (FA_OK when no kernel recorded a problem) and clears
+ * it when clear != 0.
+ */
+int fa_get_device_status(void* stream, int* status_host, int clear);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_H_ */

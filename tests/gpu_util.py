@@ -1,0 +1,78 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device
+and compare results with the oracle under the stated tolerances."""
+from __future__ import annotations
+
+import numpy as np
+
+import workloads as W
+
+# Tolerances for bf16 inputs/outputs with fp32 accumulation against the fp64
+# oracle (O max-abs, O mean-abs, LSE abs).
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+LSE_ABS = 1e-3
+
+
+def to_dev_bf16(bits: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_dev_i32(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(np.asarray(a, dtype=np.int32))).cuda()
+
+
+def bf16_to_f64(t) -> np.ndarray:
+    import torch
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    """Assert the bf16/fp32 GPU result matches the fp64 oracle; returns errors."""
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    assert o_gpu.shape == o_ref.shape, (o_gpu.shape, o_ref.shape)
+    assert np.isfinite(o_gpu).all(), f"{what}: non-finite output"
+    err = np.abs(o_gpu - o_ref)
+    mx, mean = float(err.max()), float(err.mean())
+    assert mx <= O_MAX_ABS, f"{what}: O max-abs {mx:.3e} > {O_MAX_ABS}"
+    assert mean <= O_MEAN_ABS, f"{what}: O mean-abs {mean:.3e} > {O_MEAN_ABS}"
+    lerr = 0.0
+    if lse_ref is not None:
+        lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+        lse_ref = np.asarray(lse_ref, dtype=np.float64)
+        both_inf = np.isneginf(lse_gpu) & np.isneginf(lse_ref)
+        d = np.where(both_inf, 0.0, np.abs(lse_gpu - lse_ref))
+        lerr = float(np.nanmax(d)) if d.size else 0.0
+        assert not np.isnan(d).any(), f"{what}: NaN LSE"
+        assert lerr <= LSE_ABS, f"{what}: LSE abs {lerr:.3e} > {LSE_ABS}"
+    return mx, mean, lerr
+
+
+def prefill_on_gpu(inp: W.PrefillInputs, **kw):
+    import exact_attention_148_b200 as fa
+    q, k, v = (to_dev_bf16(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    cu = to_dev_i32(inp.cu_seqlens)
+    return fa.prefill(q, k, v, cu, causal=inp.causal, scale=inp.scale,
+                      cu_seqlens_host=inp.cu_seqlens, **kw)
+
+
+def decode_on_gpu(inp: W.DecodeInputs, num_splits=0, plan=None, dev=None, **kw):
+    import exact_attention_148_b200 as fa
+    if dev is None:
+        dev = decode_device_inputs(inp)
+    if plan is None:
+        plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=inp.num_q_heads,
+                              num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
+                              page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
+                              num_splits=num_splits)
+    out, lse = fa.decode_paged(dev["q"], dev["k"], dev["v"], dev["bt"], dev["lens"], plan,
+                               layout=inp.layout, scale=inp.scale, **kw)
+    return out, lse, plan
+
+
+def decode_device_inputs(inp: W.DecodeInputs):
+    return dict(q=to_dev_bf16(inp.q_bits), k=to_dev_bf16(inp.k_pages_bits),
+                v=to_dev_bf16(inp.v_pages_bits), bt=to_dev_i32(inp.block_table),
+                lens=to_dev_i32(inp.cache_seqlens))

@@ -1,0 +1,171 @@
+"""GPU parity of the paged Flash-Decoding path against the fp64 oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from tests.gpu_util import (bf16_to_f64, compare, decode_device_inputs, decode_on_gpu, to_dev_i32)
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_rows(inp, rows):
+    return oracle.paged_decode_rows_ref(inp.q_bits, inp.k_pages_bits, inp.v_pages_bits,
+                                        inp.block_table, inp.cache_seqlens, inp.scale, rows,
+                                        inp.page_size, inp.layout, to_f64=W.as_f64)
+
+
+def check_all_rows(inp, num_splits=0, what=""):
+    out, lse, plan = decode_on_gpu(inp, num_splits)
+    rows = [(b, h) for b in range(inp.batch) for h in range(inp.num_q_heads)]
+    o_ref, l_ref = oracle_rows(inp, rows)
+    compare(bf16_to_f64(out).reshape(-1, inp.head_dim), lse.cpu().numpy().reshape(-1), o_ref, l_ref,
+            what)
+    return out, lse, plan
+
+
+def check_sampled(inp, rows, num_splits=0, what="", dev=None):
+    out, lse, plan = decode_on_gpu(inp, num_splits, dev=dev)
+    o_ref, l_ref = oracle_rows(inp, rows)
+    bi = np.array([r[0] for r in rows])
+    hi = np.array([r[1] for r in rows])
+    o = out.float().cpu().numpy()[bi, hi].astype(np.float64)
+    l = lse.cpu().numpy()[bi, hi]
+    compare(o, l, o_ref, l_ref, what)
+    return plan
+
+
+SMALL_LENS = [1, 63, 64, 65, 1000, 4097]
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 2, 3, 16])
+def test_small_batch_all_rows(num_splits):
+    inp = W.make_decode(SMALL_LENS, 8, 2, 128, seed=200)
+    check_all_rows(inp, num_splits, f"small decode splits={num_splits}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (8, 2), (16, 2), (32, 2), (6, 2), (12, 2), (8, 1)])
+def test_group_sizes(d, hq, hkv):
+    inp = W.make_decode([70, 1500, 129], hq, hkv, d, seed=300 + d + hq * 7 + hkv)
+    check_all_rows(inp, 0, f"decode d={d} hq={hq} hkv={hkv}")
+    check_all_rows(inp, 5, f"decode d={d} hq={hq} hkv={hkv} 5 splits")
+
+
+@pytest.mark.parametrize("s", [1, 2, 4, 7, 8, 16, 32, 64])
+def test_num_splits_sweep(s):
+    inp = W.make_decode([8192 + 777, 4096], 4, 4, 128, seed=400)
+    check_all_rows(inp, s, f"splits={s}")
+
+
+def test_layouts_are_bit_identical():
+    import torch
+    inp = W.make_decode(SMALL_LENS, 8, 2, 128, seed=500)
+    a = decode_on_gpu(inp, 3)
+    b = decode_on_gpu(W.relayout(inp, "HND"), 3)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 4])
+def test_page_permutation_is_bit_identical(num_splits):
+    import torch
+    inp = W.make_decode(SMALL_LENS, 8, 2, 128, seed=600, extra_pages=5)
+    a = decode_on_gpu(inp, num_splits)
+    for seed in (1, 2):
+        b = decode_on_gpu(W.permute_pages(inp, seed), num_splits)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_unused_slots_poisoned_with_nan():
+    import torch
+    inp = W.make_decode(SMALL_LENS, 8, 2, 128, seed=700, extra_pages=3)
+    a = decode_on_gpu(inp, 2)
+    b = decode_on_gpu(W.poison_unused(inp), 2)
+    assert torch.isfinite(b[0].float()).all()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_zero_length_request():
+    import torch
+    inp = W.make_decode([0, 100, 0], 4, 2, 128, seed=800)
+    out, lse, _ = decode_on_gpu(inp, 0)
+    assert torch.all(out[0] == 0) and torch.all(out[2] == 0)
+    assert torch.all(torch.isneginf(lse[0])) and torch.all(torch.isneginf(lse[2]))
+    rows = [(1, h) for h in range(4)]
+    o_ref, l_ref = oracle_rows(inp, rows)
+    compare(bf16_to_f64(out[1]), lse[1].cpu().numpy(), o_ref, l_ref, "zero-length batch")
+
+
+def test_isolation_between_requests():
+    import torch
+    inp = W.make_decode([300, 700], 4, 4, 128, seed=900)
+    dev = decode_device_inputs(inp)
+    a = decode_on_gpu(inp, 2, dev=dev)
+    # overwrite request 0's pages
+    for p in inp.block_table[0][:5]:
+        dev["k"][int(p)] = 1.0
+        dev["v"][int(p)] = -1.0
+    b = decode_on_gpu(inp, 2, dev=dev)
+    assert torch.equal(a[0][1], b[0][1]) and torch.equal(a[1][1], b[1][1])
+    assert not torch.equal(a[0][0], b[0][0])
+
+
+def test_deterministic():
+    import torch
+    inp = W.make_decode(SMALL_LENS, 8, 2, 128, seed=1000)
+    dev = decode_device_inputs(inp)
+    a = decode_on_gpu(inp, 3, dev=dev)
+    b = decode_on_gpu(inp, 3, dev=dev)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_bad_page_id_is_reported_not_faulted():
+    import exact_attention_148_b200 as fa
+    inp = W.make_decode([200], 4, 4, 128, seed=1100)
+    fa.device_status(clear=True)
+    bt = inp.block_table.copy()
+    bt[0, 1] = inp.num_pages + 3          # outside the pool: reads as zeros
+    bad = W.DecodeInputs(inp.name, inp.q_bits, inp.k_pages_bits, inp.v_pages_bits, bt,
+                         inp.cache_seqlens, inp.scale, inp.layout, inp.page_size)
+    out, lse, _ = decode_on_gpu(bad, 1)
+    assert fa.device_status(clear=True) == fa.FA_ERR_BAD_PAGE
+    assert np.isfinite(out.float().cpu().numpy()).all()
+    decode_on_gpu(inp, 1)
+    assert fa.device_status(clear=True) == 0
+
+
+def test_longer_cache_than_planned_is_reported():
+    import exact_attention_148_b200 as fa
+    inp = W.make_decode([640, 64], 4, 4, 128, seed=1200)
+    plan = fa.decode_plan([128, 64], num_q_heads=4, num_kv_heads=4, head_dim=128,
+                          max_pages_per_seq=inp.block_table.shape[1], num_splits=1)
+    fa.device_status(clear=True)
+    decode_on_gpu(inp, plan=plan)
+    assert fa.device_status(clear=True) == fa.FA_ERR_PLAN_MISMATCH
+
+
+def _sample(inp, n, seed):
+    g = np.random.default_rng(seed)
+    rows = {(int(np.argmax(inp.cache_seqlens)), 0), (int(np.argmin(inp.cache_seqlens)), inp.num_q_heads - 1)}
+    while len(rows) < n:
+        rows.add((int(g.integers(inp.batch)), int(g.integers(inp.num_q_heads))))
+    return sorted(rows)
+
+
+def test_paged_decode_batch_config_sampled():
+    inp = W.paged_decode_batch()
+    check_sampled(inp, _sample(inp, 96, 3), 0, "paged decode batch (64 req, 32q/8kv)")
+
+
+def test_long_split_decode_config_sampled():
+    inp = W.long_split_decode()
+    dev = decode_device_inputs(inp)
+    rows = _sample(inp, 24, 4)
+    for s in (0, 1, 8, 64):
+        check_sampled(inp, rows, s, f"long split decode splits={s}", dev=dev)
+
+
+def test_ragged_split_decode_config_sampled():
+    inp = W.ragged_split_decode()
+    rows = [(0, h) for h in (0, 7, 31)] + _sample(inp, 24, 5)
+    check_sampled(inp, sorted(set(rows)), 0, "ragged split decode")

@@ -1,0 +1,125 @@
+"""GPU parity of fa_prefill against the fp64 oracle (run on a B200)."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from tests.gpu_util import bf16_to_f64, compare, prefill_on_gpu, to_dev_bf16, to_dev_i32
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_full(inp):
+    return oracle.attention_ref(W.as_f64(inp.q_bits), W.as_f64(inp.k_bits), W.as_f64(inp.v_bits),
+                                inp.cu_seqlens, inp.causal, inp.scale)
+
+
+def check_full(inp, what):
+    out, lse = prefill_on_gpu(inp)
+    o_ref, l_ref = oracle_full(inp)
+    return compare(bf16_to_f64(out), lse.cpu().numpy(), o_ref, l_ref, what)
+
+
+def sample_rows(inp, n, seed):
+    """Random (token, head) rows plus every sequence's first and last rows."""
+    g = np.random.default_rng(seed)
+    T = int(inp.cu_seqlens[-1])
+    H = inp.num_q_heads
+    rows = set()
+    for b in range(len(inp.cu_seqlens) - 1):
+        for t in (int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1]) - 1):
+            rows.add((t, int(g.integers(H))))
+    while len(rows) < n:
+        rows.add((int(g.integers(T)), int(g.integers(H))))
+    return sorted(rows)
+
+
+def check_sampled(inp, n, seed, what):
+    out, lse = prefill_on_gpu(inp)
+    rows = sample_rows(inp, n, seed)
+    q = W.bf16_bits_to_f32(inp.q_bits)
+    k = W.bf16_bits_to_f32(inp.k_bits)
+    v = W.bf16_bits_to_f32(inp.v_bits)
+    o_ref, l_ref = oracle.attention_rows_ref(q, k, v, inp.cu_seqlens, inp.causal, inp.scale, rows)
+    idx_t = np.array([r[0] for r in rows])
+    idx_h = np.array([r[1] for r in rows])
+    o = out.float().cpu().numpy()[idx_t, idx_h].astype(np.float64)
+    l = lse.cpu().numpy()[idx_t, idx_h]
+    return compare(o, l, o_ref, l_ref, what)
+
+
+def test_tiny_causal_prefill():
+    check_full(W.tiny_causal_prefill(), "tiny causal prefill")
+
+
+RAGGED = [1, 127, 128, 129, 300, 513]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 1), (8, 2)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_small_varlen(d, hq, hkv, causal):
+    inp = W.make_prefill(RAGGED, hq, hkv, d, causal=causal, seed=100 + d + hq + hkv)
+    check_full(inp, f"varlen d={d} hq={hq} hkv={hkv} causal={causal}")
+
+
+def test_explicit_scale_and_single_token():
+    inp = W.make_prefill([1], 2, 2, 128, causal=True, scale=0.3, seed=7)
+    check_full(inp, "single token")
+    inp = W.make_prefill([700, 1], 2, 2, 64, causal=False, scale=0.05, seed=8)
+    check_full(inp, "non-causal explicit scale")
+
+
+def test_multi_tile_long_sequence():
+    inp = W.make_prefill([2048 + 77], 4, 2, 128, causal=True, seed=11)
+    check_full(inp, "2125-token causal GQA")
+
+
+def test_varlen_config_sampled():
+    inp = W.varlen_causal_prefill()
+    check_sampled(inp, 1024, 1, "varlen causal prefill (8 seqs, 32 heads)")
+
+
+def test_long_gqa_config_sampled():
+    inp = W.long_gqa_prefill()
+    check_sampled(inp, 512, 2, "32K GQA causal prefill")
+
+
+def test_sequences_are_isolated():
+    """Changing one sequence's tokens leaves every other sequence bit-identical."""
+    import torch
+    inp = W.make_prefill([300, 200, 129], 4, 2, 128, causal=True, seed=21)
+    out1, lse1 = prefill_on_gpu(inp)
+    inp2 = W.make_prefill([300, 200, 129], 4, 2, 128, causal=True, seed=21)
+    s0, s1 = int(inp.cu_seqlens[1]), int(inp.cu_seqlens[2])
+    g = np.random.default_rng(5)
+    for arr in (inp2.q_bits, inp2.k_bits, inp2.v_bits):
+        arr[s0:s1] = W.f32_to_bf16_bits(g.standard_normal(arr[s0:s1].shape).astype(np.float32))
+    out2, lse2 = prefill_on_gpu(inp2)
+    keep = np.r_[0:s0, s1:int(inp.cu_seqlens[-1])]
+    assert torch.equal(out1[keep], out2[keep])
+    assert torch.equal(lse1[keep], lse2[keep])
+    assert not torch.equal(out1[s0:s1], out2[s0:s1])
+
+
+def test_deterministic():
+    import torch
+    inp = W.make_prefill([1000, 333], 8, 2, 128, causal=True, seed=31)
+    a = prefill_on_gpu(inp)
+    b = prefill_on_gpu(inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_without_lse_matches():
+    import torch
+    inp = W.make_prefill([257], 2, 2, 128, causal=True, seed=41)
+    a, _ = prefill_on_gpu(inp)
+    b, none = prefill_on_gpu(inp, return_lse=False)
+    assert none is None and torch.equal(a, b)
+
+
+def test_device_status_clean_after_prefill():
+    import exact_attention_148_b200 as fa
+    inp = W.make_prefill([129], 2, 2, 64, causal=True, seed=51)
+    prefill_on_gpu(inp)
+    assert fa.device_status() == 0

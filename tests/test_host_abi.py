@@ -1,0 +1,210 @@
+"""Host-side checks of the C ABI library (no GPU needed).
+
+The library must load, export every function include/exact_attention.h
+declares, and its host-only parts (planner, argument validation that fails
+before any CUDA call) must behave as documented.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import exact_attention_148_b200 as fa
+from exact_attention_148_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "exact_attention.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return fa.library()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_api():
+    fns = header_functions()
+    for name in ["fa_prefill", "fa_decode_plan", "fa_decode_paged", "fa_merge_states",
+                 "fa_plan_free", "fa_strerror", "fa_get_device_status"]:
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), f"{name} declared in the header but not exported"
+    assert sorted(header_functions()) == sorted(fa.EXPORTED_SYMBOLS)
+
+
+def test_only_api_symbols_are_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path], capture_output=True, text=True).stdout
+    names = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    fa_names = {n for n in names if n.startswith("fa_")}
+    assert fa_names == set(header_functions())
+
+
+def test_version_and_strerror(lib):
+    assert fa.version() == 100
+    assert fa.strerror(0) == "ok"
+    assert "workspace" in fa.strerror(-3)
+    assert fa.strerror(12345) == "unknown status"
+
+
+def _plan(lens, hq=32, hkv=8, d=128, max_pages=None, num_sms=148, splits=0):
+    lens = np.asarray(lens, dtype=np.int32)
+    if max_pages is None:
+        max_pages = max(1, int(np.max((lens + 63) // 64)))
+    return fa.decode_plan(lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                          max_pages_per_seq=max_pages, num_sms=num_sms, num_splits=splits)
+
+
+def _splits(L, chunk):
+    return max(1, -(-int(L) // chunk))
+
+
+@pytest.mark.parametrize("lens", [[1024, 32768, 5000, 64], [131072] * 4, [131072] + [2048] * 63,
+                                  [0, 0, 7], [1], list(range(1, 300, 7))])
+def test_plan_covers_every_key_once(lib, lens):
+    p = _plan(lens)
+    info = p.info
+    assert info.chunk_tokens % 64 == 0 and info.chunk_tokens >= 64
+    assert info.max_splits == max(1, max(_splits(L, info.chunk_tokens) for L in lens))
+    for L in lens:
+        # splits [s*chunk, min(L, (s+1)*chunk)) tile [0, L) exactly, no overlap
+        n = _splits(L, info.chunk_tokens)
+        covered = []
+        for s in range(n):
+            lo, hi = s * info.chunk_tokens, min(L, (s + 1) * info.chunk_tokens)
+            assert lo < hi or L == 0
+            covered.extend(range(lo, hi))
+        assert covered == list(range(L))
+    units = info.num_kv_heads * (info.num_q_heads // info.num_kv_heads // info.heads_per_cta)
+    assert info.num_work_items == units * sum(_splits(L, info.chunk_tokens) for L in lens)
+
+
+def test_plan_workspace_size(lib):
+    p = _plan([131072] * 4, hq=32, hkv=32, splits=16)
+    i = p.info
+    assert i.max_splits == 16
+    rows = 4 * 32
+    o_bytes = 16 * rows * 128 * 4
+    lse_bytes = 16 * rows * 4
+    assert p.workspace_bytes >= o_bytes + lse_bytes
+    assert p.workspace_bytes % 256 == 0
+    assert p.workspace_bytes < o_bytes + lse_bytes + 512
+    # no split -> no workspace
+    q = _plan([100, 200], splits=1)
+    assert q.info.max_splits == 1 and q.workspace_bytes == 0
+
+
+@pytest.mark.parametrize("s", [1, 2, 3, 4, 7, 8, 16, 32, 64])
+def test_plan_override_caps_splits(lib, s):
+    p = _plan([131072] * 4, hq=32, hkv=32, splits=s)
+    assert p.info.max_splits <= s
+    if 2048 % s == 0:
+        assert p.info.max_splits == s
+
+
+def test_plan_is_deterministic(lib):
+    lens = np.random.default_rng(3).integers(1024, 32769, size=64)
+    a = _plan(lens).info
+    b = _plan(lens).info
+    assert a == b
+
+
+def test_plan_heads_per_cta(lib):
+    assert _plan([100], hq=32, hkv=8).info.heads_per_cta == 4
+    assert _plan([100], hq=32, hkv=32).info.heads_per_cta == 1
+    assert _plan([100], hq=32, hkv=2).info.heads_per_cta == 8     # 16 per kv head -> 2 CTAs
+    assert _plan([100], hq=12, hkv=4).info.heads_per_cta == 1     # group 3
+    assert _plan([100], hq=12, hkv=2).info.heads_per_cta == 2     # group 6
+
+
+def test_plan_rejects_cache_overflow(lib):
+    with pytest.raises(fa.FAError) as e:
+        _plan([65], max_pages=1)
+    assert e.value.status == fa.FA_ERR_INVALID_ARG
+    with pytest.raises(fa.FAError):
+        _plan([-1], max_pages=1)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(hq=30, hkv=8), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(num_sms=0), fa.FA_ERR_INVALID_ARG),
+])
+def test_plan_rejects_bad_shapes(lib, kw, status):
+    with pytest.raises(fa.FAError) as e:
+        _plan([100], **kw)
+    assert e.value.status == status
+
+
+def test_plan_rejects_other_page_sizes(lib):
+    lens = np.array([100], dtype=np.int32)
+    with pytest.raises(fa.FAError) as e:
+        fa.decode_plan(lens, num_q_heads=4, num_kv_heads=4, head_dim=128, page_size=16,
+                       max_pages_per_seq=8, num_sms=148)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_prefill_validation_before_any_cuda_call(lib):
+    cu = np.array([0, 128], dtype=np.int32)
+    cuh = cu.ctypes.data_as(ctypes.c_void_p)
+    A = 0x10000   # never dereferenced: validation fails first
+    call = lambda q=A, hq=4, hkv=4, d=128, scale=float("nan"), cuh=cuh, out=A, k=A: lib.fa_prefill(
+        _fake(q), _fake(k), _fake(A), _fake(A), cuh, 1, hq, hkv, d, 1, scale, _fake(out), None, None)
+    assert call(q=0) == fa.FA_ERR_INVALID_ARG
+    assert call(q=A + 2) == fa.FA_ERR_INVALID_ARG                 # misaligned
+    assert call(hq=6, hkv=4) == fa.FA_ERR_INVALID_ARG              # Hq % Hkv
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(scale=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == fa.FA_ERR_INVALID_ARG
+    bad = np.array([0, 0], dtype=np.int32)                          # empty sequence
+    assert call(cuh=bad.ctypes.data_as(ctypes.c_void_p)) == fa.FA_ERR_INVALID_ARG
+    bad2 = np.array([5, 10], dtype=np.int32)                        # must start at 0
+    assert call(cuh=bad2.ctypes.data_as(ctypes.c_void_p)) == fa.FA_ERR_INVALID_ARG
+
+
+def test_decode_validation_before_any_cuda_call(lib):
+    p = _plan([1000, 3000], hq=8, hkv=2, splits=4)
+    assert p.workspace_bytes > 0
+    A = 0x10000
+    def call(ws=A, ws_bytes=None, q=A, strides=(64 * 2 * 128, 2 * 128, 128), npages=100, plan=p.handle):
+        return lib.fa_decode_paged(_fake(q), _fake(A), _fake(A), npages, *strides, _fake(A), _fake(A),
+                                   plan, float("nan"), _fake(A), None, _fake(ws),
+                                   p.workspace_bytes if ws_bytes is None else ws_bytes, None)
+    assert call(ws_bytes=p.workspace_bytes - 1) == fa.FA_ERR_WORKSPACE
+    assert call(ws=0) == fa.FA_ERR_INVALID_ARG
+    assert call(ws=A + 16) == fa.FA_ERR_INVALID_ARG                  # workspace not 256-aligned
+    assert call(q=A + 8) == fa.FA_ERR_INVALID_ARG
+    assert call(strides=(64 * 2 * 128, 2 * 128, 100)) == fa.FA_ERR_INVALID_ARG
+    assert call(npages=0) == fa.FA_ERR_INVALID_ARG
+    assert call(plan=None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_merge_validation_before_any_cuda_call(lib):
+    A = 0x10000
+    f = lambda S=2, d=128, o=A: lib.fa_merge_states(_fake(o), _fake(A), S, 4, 2, d, _fake(A), None, None)
+    assert f(S=0) == fa.FA_ERR_INVALID_ARG
+    assert f(d=32) == fa.FA_ERR_UNSUPPORTED
+    assert f(o=A + 4) == fa.FA_ERR_INVALID_ARG
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(128, 2, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 128], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.prefill(q, q, q, cu)
