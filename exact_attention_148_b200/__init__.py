@@ -19,7 +19,7 @@ import numpy as np
 
 __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
-    "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
+    "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +37,11 @@ FA_ERR_BAD_PAGE = -7
 EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
+    "fa_decode_paged_static",
 ]
+
+# Size of the library's static decode scratch (FA_STATIC_SCRATCH_BYTES).
+STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class FAError(RuntimeError):
@@ -94,6 +98,8 @@ def library() -> ctypes.CDLL:
     L.fa_get_device_status.restype = i32
     L.fa_version.argtypes = []
     L.fa_version.restype = i32
+    L.fa_decode_paged_static.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, f32, vp, vp, vp]
+    L.fa_decode_paged_static.restype = i32
     _lib = L
     return L
 
@@ -272,6 +278,29 @@ def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePl
         _ptr(cache_seqlens), plan.handle, _scale_arg(scale), _ptr(out), _ptr(lse), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(st, "fa_decode_paged")
+    return out, lse
+
+
+def decode_paged_static(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePlan, *,
+                        layout: str = "NHD", scale: float | None = None, out=None, lse=None,
+                        return_lse: bool = True, stream=None):
+    """``decode_paged`` without a workspace, for callers that cannot allocate
+    device memory: the split partials use the library's static 16 MiB device
+    scratch (``STATIC_SCRATCH_BYTES``), shared by every call on a device, so
+    calls that overlap on the GPU race and must be ordered by the caller.
+    Pass preallocated ``out`` (and ``lse``) to keep the call allocation-free."""
+    torch = _torch()
+    _require_cuda(q, k_pages, v_pages, block_table, cache_seqlens, out, lse)
+    B, Hq, d = q.shape
+    ps, ts, hs = page_strides(k_pages, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = library().fa_decode_paged_static(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(block_table),
+        _ptr(cache_seqlens), plan.handle, _scale_arg(scale), _ptr(out), _ptr(lse), _stream_ptr(stream))
+    _check(st, "fa_decode_paged_static")
     return out, lse
 
 

@@ -393,3 +393,53 @@ FA_API int fa_get_device_status(void* stream, int* status_host, int clear) {
 }
 
 FA_API int fa_version(void) { return 100; }
+
+// ============================================================================
+// Scratch-free decode (fa_decode_paged_static): the split partials go to a
+// fixed static device array instead of a caller workspace, for callers that
+// cannot allocate device memory.  Host code must not use the array's name as a
+// device address; its address is looked up once per device below.
+namespace {
+
+constexpr size_t kStaticScratchBytes = FA_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 128;
+
+// Device address of g_static_scratch on the current device, looked up with
+// cudaGetSymbolAddress the first time each device asks and cached after that.
+int static_scratch_address(void** addr_out) {
+  int dev = 0;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    addr[dev] = ptr;
+  }
+  *addr_out = addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+FA_API int fa_decode_paged_static(const void* q, const void* k_pages, const void* v_pages,
+                                  int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                                  int64_t head_stride, const int32_t* block_table,
+                                  const int32_t* cache_seqlens_dev, const fa_plan* plan, float scale,
+                                  void* out, float* lse, void* stream) {
+  if (plan == nullptr || plan->p.magic != fa::kPlanMagic) return FA_ERR_INVALID_ARG;
+  if (plan->p.workspace_bytes > kStaticScratchBytes) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (plan->p.workspace_bytes > 0) {
+    const int st = static_scratch_address(&scratch);
+    if (st != FA_OK) return st;
+  }
+  return fa_decode_paged(q, k_pages, v_pages, num_pages, page_stride, token_stride, head_stride,
+                         block_table, cache_seqlens_dev, plan, scale, out, lse, scratch,
+                         kStaticScratchBytes, stream);
+}

@@ -151,6 +151,40 @@ int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, int
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_decode_paged_static — fa_decode_paged for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that may not call cudaMalloc: extensions hosted inside a framework that owns
+ * every byte of device memory through its own allocator and gives plugins no
+ * way to allocate, serving loops that must not pay for cudaMalloc/cudaFree
+ * (which can synchronise the device and stall other work), and processes
+ * whose device-memory budget is fixed at start-up.
+ *
+ * Same arguments and results as fa_decode_paged, minus the workspace: the
+ * split partials live in one file-scope static device array of
+ * FA_STATIC_SCRATCH_BYTES (16 MiB) inside this library.  Every GPU that loads
+ * the library holds that array until the process exits.  The caller still
+ * passes all inputs and outputs.
+ *   - A plan whose workspace_bytes exceeds FA_STATIC_SCRATCH_BYTES is rejected
+ *     with FA_ERR_WORKSPACE before anything is enqueued.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array, which keeps whatever the last
+ *     call left in it.  Nothing in it needs to start at zero: every partial the
+ *     merge reads is written earlier in the same call.  Calls that overlap on
+ *     the GPU (for example on two streams at once) race on the array; the
+ *     caller must order them.
+ */
+#define FA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int fa_decode_paged_static(const void* q, const void* k_pages, const void* v_pages,
+                           int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                           int64_t head_stride, const int32_t* block_table,
+                           const int32_t* cache_seqlens_dev, const fa_plan* plan, float scale,
+                           void* out, float* lse, void* stream);
+
+/*
  * fa_merge_states — combine partial attention states by their LSE (the light
  * reduction kernel of Flash-Decoding: niuteng5618.github.io, section
  * "FA对decode阶段的影响", step 4).
