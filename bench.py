@@ -40,7 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill"}
-DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode"}
+DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode",
+                    "paged_decode_batch16"}
 
 
 def load_peaks():

@@ -269,6 +269,13 @@ def paged_decode_batch() -> DecodeInputs:
     return make_decode(lens, 32, 8, 128, seed=3, name="paged_decode_batch")
 
 
+def paged_decode_batch16() -> DecodeInputs:
+    """Profiling-sized variant of the paged batch (16 requests, ~1 GB of KV):
+    same length distribution and heads, small enough for multi-pass ncu."""
+    lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=16)
+    return make_decode(lens, 32, 8, 128, seed=13, name="paged_decode_batch16")
+
+
 def long_split_decode() -> DecodeInputs:
     """4 requests of 131072 cached tokens, 32 heads MHA, d=128, shuffled pages."""
     return make_decode([131072] * 4, 32, 32, 128, seed=4, name="long_split_decode")
@@ -336,6 +343,7 @@ CONFIGS = {
     "varlen_causal_prefill": varlen_causal_prefill,
     "long_gqa_prefill": long_gqa_prefill,
     "paged_decode_batch": paged_decode_batch,
+    "paged_decode_batch16": paged_decode_batch16,
     "long_split_decode": long_split_decode,
     "ragged_split_decode": ragged_split_decode,
 }
