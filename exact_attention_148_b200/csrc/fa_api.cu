@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -15,7 +16,7 @@
 #include "../../include/exact_attention.h"
 #include "decode_sm100.cuh"
 #include "planner.h"
-#include "prefill_sm100.cuh"
+#include "prefill_pp_sm100.cuh"
 
 #define FA_API extern "C" __attribute__((visibility("default")))
 
@@ -87,19 +88,27 @@ float resolve_scale(float scale, int head_dim) {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------- prefill
+// groups: (sequence << 16 | kv head, number of CTAs) in launch order.
 template <int D>
-int launch_prefill(fa::PrefillParams& prm, const std::vector<uint32_t>& tiles, int num_q_heads,
+int launch_prefill(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t, int>>& groups,
                    cudaStream_t stream) {
-  using C = fa::PrefillCfg<D>;
-  auto kernel = fa::fa_prefill_kernel<D>;
-  int st = ensure_smem(reinterpret_cast<const void*>(kernel), C::SMEM_BYTES);
+  constexpr int kSmem = fa::PrefillPPCfg<D>::SMEM_BYTES;
+  constexpr int kThreads = fa::kPrefillPPThreads;
+  auto kernel = fa::fa_prefill_pp_kernel<D>;
+  int st = ensure_smem(reinterpret_cast<const void*>(kernel), kSmem);
   if (st != FA_OK) return st;
-  for (size_t off = 0; off < tiles.size(); off += fa::kPrefillMaxTiles) {
-    const int n = static_cast<int>(std::min<size_t>(fa::kPrefillMaxTiles, tiles.size() - off));
-    std::memcpy(prm.tiles, tiles.data() + off, n * sizeof(uint32_t));
-    prm.num_tiles = n;
-    dim3 grid(num_q_heads, n);
-    kernel<<<grid, fa::kPrefillThreads, C::SMEM_BYTES, stream>>>(prm);
+  for (size_t off = 0; off < groups.size(); off += fa::kPrefillMaxGroups) {
+    const int n = static_cast<int>(std::min<size_t>(fa::kPrefillMaxGroups, groups.size() - off));
+    int64_t total = 0;
+    for (int i = 0; i < n; ++i) {
+      prm.group_start[i] = static_cast<int>(total);
+      prm.group_id[i] = groups[off + i].first;
+      total += groups[off + i].second;
+    }
+    if (total > INT32_MAX) return FA_ERR_UNSUPPORTED;
+    prm.group_start[n] = static_cast<int>(total);
+    prm.num_groups = n;
+    kernel<<<static_cast<unsigned>(total), kThreads, kSmem, stream>>>(prm);
     FA_CUDA_CHECK(cudaGetLastError());
   }
   return FA_OK;
@@ -157,26 +166,33 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
   scale = resolve_scale(scale, head_dim);
   if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
   if (cu_seqlens_host[0] != 0) return FA_ERR_INVALID_ARG;
-  std::vector<std::pair<int, uint32_t>> work;   // (cost, entry)
+  if (num_kv_heads > 65535) return FA_ERR_UNSUPPORTED;
+  // Sequences longest first (their groups carry the most work); each sequence
+  // contributes one group of ceil(L/128) * (Hq/Hkv) CTAs per kv head.
+  std::vector<std::pair<int64_t, int>> by_len;   // (length, sequence)
   for (int b = 0; b < batch; ++b) {
     const int64_t L = static_cast<int64_t>(cu_seqlens_host[b + 1]) - cu_seqlens_host[b];
     if (L < 1) return FA_ERR_INVALID_ARG;
-    const int64_t ntiles = (L + 127) / 128;
-    if (ntiles > 65535) return FA_ERR_UNSUPPORTED;
-    for (int t = 0; t < ntiles; ++t)
-      work.emplace_back(causal ? t + 1 : static_cast<int>(ntiles),
-                        (static_cast<uint32_t>(b) << 16) | static_cast<uint32_t>(t));
+    if ((L + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;
+    by_len.emplace_back(L, b);
   }
   const int64_t T = cu_seqlens_host[batch];
   if (T * num_q_heads * head_dim >= (int64_t{1} << 40)) return FA_ERR_UNSUPPORTED;
-  // Heaviest tiles first so the block scheduler's greedy fill ends with short
-  // tiles (longest-processing-time order); ties keep sequence/tile order.
-  std::stable_sort(work.begin(), work.end(),
+  std::stable_sort(by_len.begin(), by_len.end(),
                    [](const auto& a, const auto& b) { return a.first > b.first; });
-  std::vector<uint32_t> tiles(work.size());
-  for (size_t i = 0; i < work.size(); ++i) tiles[i] = work[i].second;
+  const int group = num_q_heads / num_kv_heads;
+  std::vector<std::pair<uint32_t, int>> groups;
+  groups.reserve(static_cast<size_t>(batch) * num_kv_heads);
+  for (const auto& e : by_len) {
+    const int ntiles = static_cast<int>((e.first + 127) / 128);
+    // A CTA takes two heads of the group at one q tile when the group is
+    // even, else two consecutive q tiles of one head.
+    const int ctas = (group % 2 == 0) ? ntiles * (group / 2) : ((ntiles + 1) / 2) * group;
+    for (int g = 0; g < num_kv_heads; ++g)
+      groups.emplace_back((static_cast<uint32_t>(e.second) << 16) | static_cast<uint32_t>(g), ctas);
+  }
 
-  static thread_local fa::PrefillParams prm;   // ~8.6 KB; kept off the stack
+  static thread_local fa::PrefillParams prm;   // ~17 KB; kept off the stack
   std::memset(&prm, 0, sizeof(prm));
   const cuuint32_t box[3] = {64, 1, 128};
   {
@@ -201,12 +217,11 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_dev;
   prm.num_q_heads = num_q_heads;
-  prm.group = num_q_heads / num_kv_heads;
+  prm.group = group;
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (head_dim == 128) return launch_prefill<128>(prm, tiles, num_q_heads, s);
-  return launch_prefill<64>(prm, tiles, num_q_heads, s);
+  return head_dim == 128 ? launch_prefill<128>(prm, groups, s) : launch_prefill<64>(prm, groups, s);
 }
 
 FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,

@@ -1,0 +1,450 @@
+// Ping-pong exact-attention prefill for sm_100a: two 128-row query tiles per
+// CTA share every K/V tile, and two softmax warpgroups take turns with the
+// tensor core.
+//
+// Roles (10 warps):
+//   warps 0-3  softmax + epilogue of slot 0 (thread r owns TMEM lane r)
+//   warps 4-7  softmax + epilogue of slot 1
+//   warp  8    TMA producer: both Q tiles once, then K_0, V_0, K_1, V_1, ...
+//              through one ring of NS shared-memory slots
+//   warp  9    tcgen05 MMA issuer, order per key tile j:
+//                PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
+//              so the tensor core computes one slot's P V and next scores
+//              while the other slot's softmax warpgroup exponentiates.
+// A slot is two query heads of one kv head at the same rows when the GQA
+// group is even, otherwise two consecutive 128-row tiles of one head; either
+// way both slots read the same K/V tiles, which are loaded once per CTA.
+//
+// The per-tile math is the tiling + online softmax of cloud.baidu.com
+// "FasterTransformer与FlashAttention的联系与区别", section 三 (load a K/V block, score
+// it, update running max and normaliser, accumulate the output), on tcgen05
+// tensor cores with accumulators in tensor memory; nothing of size N x N
+// reaches HBM.  S lives in TMEM, P (bf16) is written over S and fed to the PV
+// MMA straight from TMEM (TS form, V as the MN-major B operand in SMEM),
+// base-2 exponentials with a reference maximum that is only raised when a tile
+// exceeds it by more than 8 (a factor 256), which keeps O / l exact while
+// skipping most O rescales.
+//
+// Exponentials go to the MUFU unit (ex2.approx).  Optionally (compile-time
+// FA_PREFILL_POLY_MASK) some 32-column chunks of every 128, on tiles without
+// masking, are computed on the FMA and ALU pipes instead, as
+// 2^x = 2^n * p(f), n = round(x), f = x - n in [-1/2, 1/2] (Cody & Waite
+// argument reduction), with a degree-3 minimax polynomial p fitted by the Remez
+// exchange algorithm (relative error 7.5e-5, see tools/fit_exp2_poly.py), far
+// below the 2^-9 rounding P gets when it is stored as bf16.  The rounding uses
+// the float adder (adding 1.5*2^23 leaves round(x) in the low mantissa bits)
+// and 2^n is added straight into the exponent field, so no instruction of this
+// path runs on the MUFU/conversion (XU) pipe that ex2.approx uses.
+#pragma once
+
+#include "ptx_sm100.cuh"
+
+namespace fa {
+
+constexpr int kPrefillMaxGroups = 2048;  // (sequence, kv head) groups per launch
+constexpr float kRescaleThreshold = 8.0f;
+
+// Work order.  CTAs are launched in groups, one group per (sequence, kv head):
+// groups of longer sequences first; inside a group the q tiles go heaviest
+// first and the Hq/Hkv query heads that share the kv head are adjacent.  So at
+// any moment only a few heads' K/V are being read and re-reads hit L2, and the
+// block scheduler's greedy fill ends on light tiles.
+struct PrefillParams {
+  CUtensorMap tm_q;   // 3-D {d, Hq, T}, box {64, 1, 128}, 128B swizzle
+  CUtensorMap tm_k;   // 3-D {d, Hkv, T}
+  CUtensorMap tm_v;
+  __nv_bfloat16* out;        // [T, Hq, d]
+  float* lse;                // [T, Hq] or null
+  const int32_t* cu_seqlens; // [B+1]
+  int num_q_heads;
+  int group;                 // Hq / Hkv
+  int causal;
+  float scale_log2;          // scale * log2(e)
+  int num_groups;
+  int group_start[kPrefillMaxGroups + 1];   // first CTA of each group (+ total)
+  uint32_t group_id[kPrefillMaxGroups];     // (sequence << 16) | kv head
+};
+
+constexpr int kPrefillPPThreads = 320;
+
+// Measured on B200 at d=128: any polynomial share slows the kernel (the
+// extra FMA/ALU instructions cost more issue slots than the MUFU time they
+// save), so by default every exponential uses ex2.approx.
+#ifndef FA_PREFILL_POLY_MASK
+#define FA_PREFILL_POLY_MASK 0x0
+#endif
+
+template <int D>
+struct PrefillPPCfg {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
+  static constexpr int NS = (D == 128) ? 5 : 8;           // K/V ring slots
+  static constexpr int Q_OFF = 0;                          // two Q tiles
+  static constexpr int KV_OFF = 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final
+  static constexpr int NUM_BARS = 1 + 2 * NS + 7;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // Bit c set: the exponentials of 32-column chunk c use the FMA-pipe polynomial.
+  static constexpr int POLY_MASK = FA_PREFILL_POLY_MASK;
+};
+
+// 2^x on the FMA/ALU pipes (see the file comment).  Valid for x <= 8; inputs
+// below -125 are clamped (the result is then < 2^-124, negligible next to the
+// row maximum's term 2^0).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = __fadd_rn(x, 12582912.0f);     // 1.5 * 2^23 + round(x)
+  const float n = __fadd_rn(t, -12582912.0f);    // round(x)
+  const float f = __fadd_rn(x, -n);               // in [-1/2, 1/2]
+  float p = fmaf(0.0551716691f, f, 0.242611122f);
+  p = fmaf(p, f, 0.693260985f);
+  p = fmaf(p, f, 0.999928074f);
+  // The low mantissa bits of t are round(x) in two's complement; shifted by 23
+  // they add round(x) to p's exponent (mod 2^32, so negative n works too).
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrefillPPThreads, 1)
+    fa_prefill_pp_kernel(const __grid_constant__ PrefillParams p) {
+  using C = PrefillPPCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- CTA -> (sequence, kv head, two query slots)
+  const int bid = static_cast<int>(blockIdx.x);
+  int lo = 0, hi = p.num_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.group_start[mid] <= bid) lo = mid; else hi = mid - 1;
+  }
+  const int seq = static_cast<int>(p.group_id[lo] >> 16);
+  const int kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
+  const int rank = bid - p.group_start[lo];
+  const int s0 = p.cu_seqlens[seq];
+  const int L = p.cu_seqlens[seq + 1] - s0;
+  const int n_qtiles = (L + C::BM - 1) / C::BM;
+  const int G = p.group;
+  int qtile[2], head[2];
+  if ((G & 1) == 0) {            // two heads of the group, same rows
+    const int half = G >> 1;
+    const int t = n_qtiles - 1 - rank / half;
+    const int hp = rank % half;
+    qtile[0] = qtile[1] = t;
+    head[0] = kv_head * G + 2 * hp;
+    head[1] = head[0] + 1;
+  } else {                        // one head, two consecutive row tiles
+    const int npairs = (n_qtiles + 1) >> 1;
+    const int pr = npairs - 1 - rank / G;
+    qtile[0] = 2 * pr;
+    qtile[1] = 2 * pr + 1;
+    head[0] = head[1] = kv_head * G + rank % G;
+  }
+  int n_kv[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const bool active = qtile[k] >= 0 && qtile[k] < n_qtiles;
+    n_kv[k] = !active ? 0 : (p.causal ? qtile[k] + 1 : n_qtiles);
+  }
+  if (n_kv[0] == 0 && n_kv[1] == 0) return;   // uniform; nothing allocated yet
+  const int n_max = max(n_kv[0], n_kv[1]);
+
+  const uint32_t q_s = base + C::Q_OFF;
+  auto kv_s = [&](int item) { return base + C::KV_OFF + (item % C::NS) * C::TILE_BYTES; };
+  const uint32_t bars = base + C::BAR_OFF;
+  const uint32_t bar_q = bars;
+  auto bar_kv_full = [&](int item) { return bars + 8 * (1 + item % C::NS); };
+  auto bar_kv_empty = [&](int item) { return bars + 8 * (1 + C::NS + item % C::NS); };
+  auto bar_s_full = [&](int k) { return bars + 8 * (1 + 2 * C::NS + k); };
+  auto bar_p_full = [&](int k) { return bars + 8 * (3 + 2 * C::NS + k); };
+  auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * C::NS + k); };
+  const uint32_t bar_final = bars + 8 * (7 + 2 * C::NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(bar_kv_full(i), 1);
+      mbar_init(bar_kv_empty(i), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar_s_full(k), 1);
+      mbar_init(bar_p_full(k), 128);
+      mbar_init(bar_o_done(k), 1);
+    }
+    mbar_init(bar_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      const int nq = (n_kv[0] > 0) + (n_kv[1] > 0);
+      mbar_arrive_expect_tx(bar_q, nq * C::TILE_BYTES);
+      auto load_q = [&](int k, int h, int t) {
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_3d(q_s + k * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tm_q, bar_q, c * 64, h,
+                      s0 + t * C::BM);
+      };
+      if (n_kv[0] > 0) load_q(0, head[0], qtile[0]);
+      if (n_kv[1] > 0) load_q(1, head[1], qtile[1]);
+      int issued = 0;
+      for (int item = 0; item < 2 * n_max; ++item) {
+        if (!mbar_wait(bar_kv_empty(item), ((item / C::NS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar_kv_full(item), C::TILE_BYTES);
+        const CUtensorMap* map = (item & 1) ? &p.tm_v : &p.tm_k;
+        const int row = s0 + (item >> 1) * C::BN;
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_3d(kv_s(item) + c * C::CHUNK_BYTES, map, bar_kv_full(item), c * 64, kv_head, row);
+        ++issued;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i)
+          mbar_wait(bar_kv_full(i), (i / C::NS) & 1, &never);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(C::BM, C::BN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(C::BM, D, true);
+      // k is always a literal below, so per-slot values stay in registers.
+      auto issue_qk = [&](int k, uint32_t kbase) {
+        const uint32_t qb = q_s + k * C::TILE_BYTES;
+        const uint32_t d_tmem = tmem + (k ? 128u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          mma_bf16_ss(d_tmem, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                      idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int k, uint32_t vbase, bool accumulate) {
+        const uint32_t o_tmem = tmem + 256u + (k ? D : 0);
+        const uint32_t p_tmem = tmem + (k ? 128u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_bf16_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 16 * 128, C::CHUNK_BYTES, 1024),
+                      idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+      };
+      const int nkv0 = n_kv[0], nkv1 = n_kv[1];
+      bool ok = mbar_wait(bar_q, 0, abort_flag) && mbar_wait(bar_kv_full(0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after_sync();
+        if (nkv0 > 0) {
+          issue_qk(0, kv_s(0));
+          tc_commit(bar_s_full(0));
+        }
+        if (nkv1 > 0) {
+          issue_qk(1, kv_s(0));
+          tc_commit(bar_s_full(1));
+        }
+        tc_commit(bar_kv_empty(0));
+      }
+      // One slot's step at key tile j: O_k += P_k V_j, then S_k(j+1).
+      // S_k(j+1) overwrites the columns P_k(j) occupies; the PV MMA that reads
+      // them was issued first and MMAs of one thread run in order.
+      auto slot_step = [&](int k, int nk, int j, int v_item, int k_item) -> bool {
+        if (j >= nk) return true;
+        if (!mbar_wait(bar_p_full(k), j & 1, abort_flag)) return false;
+        tc_fence_after_sync();
+        issue_pv(k, kv_s(v_item), j > 0);
+        tc_commit(bar_o_done(k));
+        if (j + 1 < nk) {
+          issue_qk(k, kv_s(k_item));
+          tc_commit(bar_s_full(k));
+        }
+        return true;
+      };
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int v_item = 2 * j + 1, k_item = 2 * j + 2;
+        const bool need_k = (j + 1 < nkv0) || (j + 1 < nkv1);
+        if (!mbar_wait(bar_kv_full(v_item), (v_item / C::NS) & 1, abort_flag)) break;
+        if (need_k && !mbar_wait(bar_kv_full(k_item), (k_item / C::NS) & 1, abort_flag)) break;
+        ok = slot_step(0, nkv0, j, v_item, k_item) && slot_step(1, nkv1, j, v_item, k_item);
+        if (!ok) break;
+        tc_commit(bar_kv_empty(v_item));
+        if (need_k) tc_commit(bar_kv_empty(k_item));
+      }
+      tc_commit(bar_final);
+      volatile int never = 0;
+      mbar_wait(bar_final, 0, &never);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int k = warp >> 2;                       // slot
+    const int r = threadIdx.x & 127;               // row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sc = tmem + lane_base + (k ? 128u : 0u);
+    const uint32_t oc = tmem + lane_base + 256u + (k ? D : 0);
+    const int my_qtile = k ? qtile[1] : qtile[0];
+    const int my_head = k ? head[1] : head[0];
+    const int q_row = my_qtile * C::BM + r;
+    const int nk = k ? n_kv[1] : n_kv[0];
+    float m_ref = 0.0f, l_sum = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(k), j & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after_sync();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_x32(sc + c * 32, s[c]);
+      tmem_ld_wait(s[0]);
+      reg_dep(s[1]);
+      reg_dep(s[2]);
+      reg_dep(s[3]);
+
+      const bool masked = p.causal ? (j == my_qtile) : ((j + 1) * C::BN > L);
+      if (masked) {
+        const int lim = p.causal ? (q_row - j * C::BN) : (L - 1 - j * C::BN);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > lim) s[c][i] = __float_as_uint(-INFINITY);
+      }
+      // row maximum: 8 independent chains, then a tree
+      float mx[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mx[t] = __uint_as_float(s[t >> 1][(t & 1) * 16]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if ((i & 15) == 0) continue;
+          const int t = 2 * c + (i >> 4);
+          mx[t] = fmaxf(mx[t], __uint_as_float(s[c][i]));
+        }
+      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float m_tile = rmax * p.scale_log2;
+      float alpha = 1.0f;
+      bool rescale = false;
+      if (j == 0) {
+        m_ref = (m_tile == -INFINITY) ? 0.0f : m_tile;
+      } else {
+        const bool need = m_tile > m_ref + kRescaleThreshold;
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          alpha = ex2_approx(m_ref - m_tile);
+          m_ref = m_tile;
+        }
+      }
+      const float neg_m = -m_ref;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+        const bool poly = ((C::POLY_MASK >> c) & 1) && !masked;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = fmaf(__uint_as_float(s[c][2 * i]), p.scale_log2, neg_m);
+          const float x1 = fmaf(__uint_as_float(s[c][2 * i + 1]), p.scale_log2, neg_m);
+          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+          ps[(i & 3) * 2] += p0;
+          ps[(i & 3) * 2 + 1] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        // P chunk c (16 packed columns) lands on S columns already in registers.
+        tmem_st_x16(sc + c * 16, pk);
+      }
+      l_sum = l_sum * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+      if (rescale) {
+        // O still holds sum_{i<j} P_i V_i against the old reference maximum:
+        // once PV_{j-1} has landed, scale it by alpha (1 on rows that kept
+        // their maximum).  P_j is already in TMEM; PV_j waits for p_full.
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (j - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld_x32(oc + c * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_x32(oc + c * 32, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(bar_p_full(k));
+    }
+    if (nk > 0 && ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (nk - 1) & 1, abort_flag))) {
+      tc_fence_after_sync();
+      const float inv_l = 1.0f / l_sum;
+      const bool valid = q_row < L;
+      __nv_bfloat16* orow =
+          p.out + (static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_x32(oc + c * 32, o);
+        tmem_ld_wait(o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head] =
+            (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa
