@@ -73,6 +73,10 @@ constexpr int kPrefillPPThreads = 320;
 #ifndef FA_PREFILL_POLY_MASK
 #define FA_PREFILL_POLY_MASK 0x0
 #endif
+// Bit c set: 32-column chunk c uses the packed half-precision MUFU ex2.
+#ifndef FA_PREFILL_F16EX2_MASK
+#define FA_PREFILL_F16EX2_MASK 0x0
+#endif
 
 template <int D>
 struct PrefillPPCfg {
@@ -109,6 +113,27 @@ __device__ __forceinline__ float exp2_poly(float x) {
   // The low mantissa bits of t are round(x) in two's complement; shifted by 23
   // they add round(x) to p's exponent (mod 2^32, so negative n works too).
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two exponentials with one MUFU instruction: the pair is rounded to f16
+// (11-bit significand) and put through ex2.approx.f16x2.  The argument rounding
+// costs a relative error of at most |x| * 2^-11 * ln 2 in 2^x (2.7e-3 at |x|=16,
+// where 2^x < 2^-16 already), comparable to the 2^-9 rounding P gets as bf16.
+__device__ __forceinline__ float2 ex2_pair_f16(float2 x) {
+  uint32_t h, e;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+  float lo, hi;
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi) : "r"(e));
+  return make_float2(lo, hi);
+}
+
+// Three-input maximum (sm_100 max.f32 with three sources).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
@@ -192,7 +217,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s_full(k), 1);
-      mbar_init(bar_p_full(k), 128);
+      mbar_init(bar_p_full(k), 4);
       mbar_init(bar_o_done(k), 1);
     }
     mbar_init(bar_final, 1);
@@ -341,20 +366,17 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i > lim) s[c][i] = __float_as_uint(-INFINITY);
       }
-      // row maximum: 8 independent chains, then a tree
-      float mx[8];
+      // row maximum: one 3-input-max chain per 32-column chunk, then a tree
+      float mx[4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mx[t] = __uint_as_float(s[t >> 1][(t & 1) * 16]);
+      for (int c = 0; c < 4; ++c) {
+        mx[c] = fmax3(__uint_as_float(s[c][0]), __uint_as_float(s[c][1]), __uint_as_float(s[c][2]));
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if ((i & 15) == 0) continue;
-          const int t = 2 * c + (i >> 4);
-          mx[t] = fmaxf(mx[t], __uint_as_float(s[c][i]));
-        }
-      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int i = 3; i < 31; i += 2)
+          mx[c] = fmax3(mx[c], __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
+        mx[c] = fmaxf(mx[c], __uint_as_float(s[c][31]));
+      }
+      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_tile = rmax * p.scale_log2;
       float alpha = 1.0f;
       bool rescale = false;
@@ -368,26 +390,38 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
           m_ref = m_tile;
         }
       }
-      const float neg_m = -m_ref;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // x = s * scale * log2(e) - m on the packed f32x2 FMA pipe
+      const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 neg_m2 = make_float2(-m_ref, -m_ref);
+      float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
         const bool poly = ((C::POLY_MASK >> c) & 1) && !masked;
+        const bool half2 = (FA_PREFILL_F16EX2_MASK >> c) & 1;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float x0 = fmaf(__uint_as_float(s[c][2 * i]), p.scale_log2, neg_m);
-          const float x1 = fmaf(__uint_as_float(s[c][2 * i + 1]), p.scale_log2, neg_m);
-          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-          ps[(i & 3) * 2] += p0;
-          ps[(i & 3) * 2 + 1] += p1;
+          const float2 x = __ffma2_rn(
+              make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), scale2, neg_m2);
+          float p0, p1;
+          if (half2) {
+            const float2 e = ex2_pair_f16(x);
+            p0 = e.x;
+            p1 = e.y;
+          } else {
+            p0 = poly ? exp2_poly(x.x) : ex2_approx(x.x);
+            p1 = poly ? exp2_poly(x.y) : ex2_approx(x.y);
+          }
+          ps[i & 3].x += p0;
+          ps[i & 3].y += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         // P chunk c (16 packed columns) lands on S columns already in registers.
         tmem_st_x16(sc + c * 16, pk);
       }
-      l_sum = l_sum * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+      l_sum = l_sum * alpha + (((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
+                               ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y)));
       if (rescale) {
         // O still holds sum_{i<j} P_i V_i against the old reference maximum:
         // once PV_{j-1} has landed, scale it by alpha (1 on rows that kept
@@ -409,7 +443,8 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(bar_p_full(k));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full(k));   // one arrival per warp
     }
     if (nk > 0 && ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (nk - 1) & 1, abort_flag))) {
       tc_fence_after_sync();
