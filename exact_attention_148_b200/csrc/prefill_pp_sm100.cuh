@@ -272,34 +272,43 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(C::BM, C::BN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(C::BM, D, true);
       // k is always a literal below, so per-slot values stay in registers.
-      auto issue_qk = [&](int k, uint32_t kbase) {
-        const uint32_t qb = q_s + k * C::TILE_BYTES;
+      // This thread's issue rate is on the per-tile critical path (it shares
+      // its SMSP with two softmax warps), so descriptors are built once and
+      // each MMA only adds a compile-time offset (address field in 16-byte
+      // units; no carry leaves the 14-bit field inside shared memory).
+      const uint64_t q_desc = sdesc_sw128(q_s, 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(base + C::KV_OFF, 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(base + C::KV_OFF, C::CHUNK_BYTES, 1024);
+      auto ring_off = [&](int item) { return static_cast<uint64_t>((item % C::NS) * (C::TILE_BYTES >> 4)); };
+      auto issue_qk = [&](int k, int item) {
+        const uint64_t qd = q_desc + (k ? (C::TILE_BYTES >> 4) : 0);
+        const uint64_t kd = k_desc0 + ring_off(item);
         const uint32_t d_tmem = tmem + (k ? 128u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(d_tmem, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                      idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32) >> 4);
+          mma_bf16_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int k, uint32_t vbase, bool accumulate) {
+      auto issue_pv = [&](int k, int item, bool accumulate) {
         const uint32_t o_tmem = tmem + 256u + (k ? D : 0);
         const uint32_t p_tmem = tmem + (k ? 128u : 0u);
+        const uint64_t vd = v_desc0 + ring_off(item);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_bf16_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 16 * 128, C::CHUNK_BYTES, 1024),
-                      idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
+                      (accumulate || kk > 0) ? 1u : 0u);
       };
       const int nkv0 = n_kv[0], nkv1 = n_kv[1];
       bool ok = mbar_wait(bar_q, 0, abort_flag) && mbar_wait(bar_kv_full(0), 0, abort_flag);
       if (ok) {
         tc_fence_after_sync();
         if (nkv0 > 0) {
-          issue_qk(0, kv_s(0));
+          issue_qk(0, 0);
           tc_commit(bar_s_full(0));
         }
         if (nkv1 > 0) {
-          issue_qk(1, kv_s(0));
+          issue_qk(1, 0);
           tc_commit(bar_s_full(1));
         }
         tc_commit(bar_kv_empty(0));
@@ -311,10 +320,10 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
         if (j >= nk) return true;
         if (!mbar_wait(bar_p_full(k), j & 1, abort_flag)) return false;
         tc_fence_after_sync();
-        issue_pv(k, kv_s(v_item), j > 0);
+        issue_pv(k, v_item, j > 0);
         tc_commit(bar_o_done(k));
         if (j + 1 < nk) {
-          issue_qk(k, kv_s(k_item));
+          issue_qk(k, k_item);
           tc_commit(bar_s_full(k));
         }
         return true;
