@@ -269,11 +269,14 @@ def paged_decode_batch() -> DecodeInputs:
     return make_decode(lens, 32, 8, 128, seed=3, name="paged_decode_batch")
 
 
+def paged_decode_batch16_lengths() -> np.ndarray:
+    return np.random.default_rng(3).integers(1024, 32768 + 1, size=16)
+
+
 def paged_decode_batch16() -> DecodeInputs:
     """Profiling-sized variant of the paged batch (16 requests, ~1 GB of KV):
     same length distribution and heads, small enough for multi-pass ncu."""
-    lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=16)
-    return make_decode(lens, 32, 8, 128, seed=13, name="paged_decode_batch16")
+    return make_decode(paged_decode_batch16_lengths(), 32, 8, 128, seed=13, name="paged_decode_batch16")
 
 
 def long_split_decode() -> DecodeInputs:
