@@ -263,23 +263,30 @@ def time_cases(cases, steps, warmup, flush, dist_ctx, e2e=False):
 
 
 class DistCtx:
-    def __init__(self):
+    """One process per GPU (NCCL), or CPU ranks over gloo for tests.  Ranks are
+    independent replicas: the only collectives are the barriers around the
+    timed region and the max over ranks of the measured times."""
+
+    def __init__(self, backend="nccl", timeout_s=300):
         import torch
         import torch.distributed as dist
         from datetime import timedelta
         self.dist = dist
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+        dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s))
         self.rank = dist.get_rank()
         self.world = dist.get_world_size()
         self.local = int(os.environ.get("LOCAL_RANK", 0))
-        torch.cuda.set_device(self.local)
+        self.device = "cpu"
+        if backend == "nccl":
+            torch.cuda.set_device(self.local)
+            self.device = "cuda"
 
     def barrier(self):
         self.dist.barrier()
 
     def max_over_ranks(self, vals):
         import torch
-        t = torch.tensor(vals, dtype=torch.float64, device="cuda")
+        t = torch.tensor(vals, dtype=torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return t.tolist()
 
@@ -391,6 +398,12 @@ def measured_traffic(kind, workload, case=None):
     return None
 
 
+def aggregate_throughput(work_per_replica: float, ms_max: float, n_replicas: int, scale: float) -> float:
+    """Whole-job throughput of N independent replicas: every replica does the
+    same work; the job takes as long as the slowest replica (max over ranks)."""
+    return n_replicas * work_per_replica / (ms_max * 1e-3) / scale
+
+
 def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=None):
     if kind == "tensor":
         achieved = algorithmic / (ms_per_launch * 1e-3) / 1e12
@@ -450,10 +463,10 @@ def run_ours(args):
         e["ms_per_launch"] = round(ms / (c.launches if isinstance(c, PrefillCase) else 1), 4)
         rooflines.append(e)
     if isinstance(main, PrefillCase):
-        value = N * main.flops / (ms_case[0] * 1e-3) / 1e12
+        value = aggregate_throughput(main.flops, ms_case[0], N, 1e12)
         unit = "TFLOP/s"
     else:
-        value = N * main.bytes / (ms_case[0] * 1e-3) / 1e9
+        value = aggregate_throughput(main.bytes, ms_case[0], N, 1e9)
         unit = "GB/s"
     # `roofline` is the kernel with the largest share of the measured step time.
     rl = rooflines[int(np.argmax(ms_case))]

@@ -37,7 +37,7 @@ FA_ERR_BAD_PAGE = -7
 EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
-    "fa_decode_paged_static",
+    "fa_decode_paged_static", "fa_selftest_wait_timeout",
 ]
 
 # Size of the library's static decode scratch (FA_STATIC_SCRATCH_BYTES).
@@ -100,6 +100,8 @@ def library() -> ctypes.CDLL:
     L.fa_version.restype = i32
     L.fa_decode_paged_static.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, f32, vp, vp, vp]
     L.fa_decode_paged_static.restype = i32
+    L.fa_selftest_wait_timeout.argtypes = [i64, vp]
+    L.fa_selftest_wait_timeout.restype = i32
     _lib = L
     return L
 
@@ -329,6 +331,14 @@ def device_status(clear: bool = True, stream=None) -> int:
     _check(library().fa_get_device_status(_stream_ptr(stream), ctypes.byref(v), 1 if clear else 0),
            "fa_get_device_status")
     return v.value
+
+
+def selftest_wait_timeout(limit_us: int = 20000, stream=None) -> int:
+    """Run the bounded-wait self-test kernel and return the device status it
+    leaves (FA_ERR_TIMEOUT when the failure path works); clears the status."""
+    _check(library().fa_selftest_wait_timeout(int(limit_us), _stream_ptr(stream)),
+           "fa_selftest_wait_timeout")
+    return device_status(clear=True, stream=stream)
 
 
 def version() -> int:

@@ -407,6 +407,14 @@ FA_API int fa_get_device_status(void* stream, int* status_host, int clear) {
   return FA_OK;
 }
 
+FA_API int fa_selftest_wait_timeout(int64_t limit_us, void* stream) {
+  const int64_t us = std::min<int64_t>(std::max<int64_t>(limit_us, 1000), 2000000);
+  fa::fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(us) * 1000ull);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}
+
 FA_API int fa_version(void) { return 100; }
 
 // ============================================================================

@@ -1,6 +1,9 @@
 #include "planner.h"
 
 #include <algorithm>
+#include <functional>
+#include <queue>
+#include <vector>
 
 #include "../../include/exact_attention.h"
 
@@ -10,6 +13,67 @@ namespace {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Decode-time model used to choose the split size (measured on B200, 148 SMs):
+// all resident split CTAs share the HBM bandwidth, one CTA alone cannot pull
+// more than ~44 GB/s (its TMA ring depth), each CTA costs ~0.5 us of fill, and a
+// second (merge) launch costs ~5 us.
+constexpr double kHbmBytesPerUs148 = 6.9e6;       // bytes per microsecond, 148 SMs
+constexpr double kCtaBytesPerUs = 4.36e4;
+constexpr double kCtaOverheadUs = 0.5;
+constexpr double kMergeLaunchUs = 5.0;
+
+// Estimated duration (us) of the split kernel (+ merge) for one chunk size:
+// CTAs enter the resident slots in grid order (split fastest, then kv-head
+// group, then request) and every running CTA moves at min(one CTA's limit,
+// HBM bandwidth / running CTAs).  Event simulation over a min-heap of finish
+// points measured in "bytes done by every running CTA" (all running CTAs
+// advance at the same rate, so that scale is shared).
+double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64_t chunk, int slots,
+                          int head_dim, int num_sms) {
+  const double bytes_per_token = 2.0 * head_dim * 2.0;   // K and V rows of one kv head
+  const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
+  const double overhead_bytes = kCtaOverheadUs * kCtaBytesPerUs;
+  std::priority_queue<double, std::vector<double>, std::greater<double>> running;
+  double v = 0.0, t = 0.0;
+  size_t b = 0;
+  int64_t u = 0, sidx = 0;
+  int max_splits = 1;
+  // next CTA in grid order, or a negative value when none is left
+  auto next_cta = [&]() -> double {
+    while (b < lens.size()) {
+      const int64_t L = lens[b];
+      const int64_t n = std::max<int64_t>(1, ceil_div(L, chunk));
+      max_splits = std::max<int>(max_splits, static_cast<int>(n));
+      if (sidx < n) {
+        const int64_t tok = std::max<int64_t>(0, std::min<int64_t>(chunk, L - sidx * chunk));
+        ++sidx;
+        return tok * bytes_per_token + overhead_bytes;
+      }
+      sidx = 0;
+      if (++u == units) {
+        u = 0;
+        ++b;
+      }
+    }
+    return -1.0;
+  };
+  for (int i = 0; i < slots; ++i) {
+    const double c = next_cta();
+    if (c < 0) break;
+    running.push(v + c);
+  }
+  while (!running.empty()) {
+    const double rate = std::min(kCtaBytesPerUs, hbm / static_cast<double>(running.size()));
+    const double nxt = running.top();
+    running.pop();
+    t += (nxt - v) / rate;
+    v = nxt;
+    const double c = next_cta();
+    if (c >= 0) running.push(v + c);
+  }
+  return t + (max_splits > 1 ? kMergeLaunchUs : 0.0);
+}
 }  // namespace
 
 int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
@@ -58,13 +122,29 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
   int64_t chunk;
   if (num_splits_override > 0) {
     chunk = round_up(std::max<int64_t>(1, ceil_div(max_len, num_splits_override)), page_size);
+  } else if (max_len <= kMinChunkTokens) {
+    chunk = round_up(std::max(max_len, 1), page_size);
   } else {
-    // Aim for about kItemsPerSlot items per resident CTA slot so the hardware
-    // scheduler's greedy assignment leaves a short tail, but never split below
-    // kMinChunkTokens keys (each CTA must amortise its pipeline fill).
-    const int64_t slots = static_cast<int64_t>(num_sms) * kDecodeCtasPerSm;
-    const int64_t target = ceil_div(total * units, slots * kItemsPerSlot);
-    chunk = round_up(std::max<int64_t>(target, kMinChunkTokens), page_size);
+    // Try split counts s (chunk = ceil(max_len / s) rounded to a page, at
+    // least kMinChunkTokens keys) plus the many-small-items rule, and keep the
+    // one the decode-time model estimates fastest (ties: fewer splits).
+    const int slots = num_sms * (pl.heads_per_cta == 8 ? 1 : kDecodeCtasPerSm);
+    std::vector<int64_t> cands;
+    for (int s : {1, 2, 3, 4, 5, 6, 8, 10, 12, 16, 20, 24, 32, 48, 64, 96, 128})
+      cands.push_back(round_up(ceil_div(max_len, s), page_size));
+    const int64_t target = ceil_div(total * units, static_cast<int64_t>(slots) * kItemsPerSlot);
+    cands.push_back(round_up(target, page_size));
+    double best_t = 0.0;
+    chunk = 0;
+    for (int64_t c : cands) {
+      c = std::max<int64_t>(c, kMinChunkTokens);
+      if (ceil_div(max_len, c) > kMaxSplits) continue;
+      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, num_sms);
+      if (chunk == 0 || t < best_t * (1.0 - 1e-9) || (t <= best_t * (1.0 + 1e-9) && c > chunk)) {
+        best_t = t;
+        chunk = c;
+      }
+    }
   }
   if (max_len > 0 && ceil_div(max_len, chunk) > kMaxSplits)
     chunk = round_up(ceil_div(max_len, kMaxSplits), page_size);

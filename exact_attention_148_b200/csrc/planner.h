@@ -15,7 +15,7 @@ constexpr uint32_t kPlanMagic = 0xFA148D0Cu;
 constexpr int kMaxSplits = 128;
 constexpr int kMinChunkTokens = 512;
 constexpr int kDecodeCtasPerSm = 2;
-constexpr int kItemsPerSlot = 8;   // target work items per resident CTA slot
+constexpr int kItemsPerSlot = 8;   // the many-small-items candidate: items per resident CTA slot
 
 struct DecodePlan {
   uint32_t magic = kPlanMagic;

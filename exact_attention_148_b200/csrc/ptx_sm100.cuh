@@ -90,6 +90,29 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Failure-detection self-test: wait on a barrier that never completes, bounded
+// by limit_ns; on expiry record FA_ERR_TIMEOUT and return.
+__global__ void fa_selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(b, 0)) {
+      if (global_timer_ns() - t0 > limit_ns) {
+        record_status(FA_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
 // ----------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast.
 // ----------------------------------------------------------------------------

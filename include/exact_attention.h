@@ -212,6 +212,17 @@ int fa_last_cuda_error(void);
  */
 int fa_get_device_status(void* stream, int* status_host, int clear);
 
+/*
+ * fa_selftest_wait_timeout — failure-detection self-test.  Launches one small
+ * kernel that waits on a barrier nothing ever arrives at, with a bound of
+ * limit_us microseconds (clamped to [1000, 2000000]).  When the bound runs out
+ * the kernel records FA_ERR_TIMEOUT in the device status word and returns; it
+ * never traps, so the CUDA context stays usable.  Read the result with
+ * fa_get_device_status().  (The same bounded-wait path guards every wait in
+ * the prefill and decode kernels.)
+ */
+int fa_selftest_wait_timeout(int64_t limit_us, void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int fa_version(void);
 
