@@ -11,6 +11,7 @@ exact/extended arithmetic, and PyTorch's CPU ``scaled_dot_product_attention``
 in float64; none is "parity unpinned".
 """
 from .attention import (  # noqa: F401
+    append_kv_ref,
     attention_probs_ref,
     attention_ref,
     attention_rows_ref,
@@ -19,5 +20,8 @@ from .attention import (  # noqa: F401
     merge_states_ref,
     paged_decode_ref,
     paged_decode_rows_ref,
+    paged_prefill_ref,
+    paged_prefill_rows_ref,
     partial_state_ref,
+    visible_key_count,
 )

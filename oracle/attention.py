@@ -22,7 +22,17 @@ Readings taken where the pages are silent (each also listed in the design doc):
 * LSE: natural log of the sum of exp of the *scaled* scores;
 * an empty key set gives O = 0 and LSE = -inf (only reachable in decode with a
   zero cache length or an empty split);
-* paged decode attends to all ``cache_seqlens[b]`` cached tokens, no mask.
+* paged decode attends to all ``cache_seqlens[b]`` cached tokens, no mask;
+* chunked (paged) prefill: a request's cache holds ``cache_seqlens[b]`` tokens
+  after the new chunk is written, and the chunk's q_len queries are the last
+  q_len positions of that sequence, so under causal masking query i of the
+  chunk (position cache_seqlens[b] - q_len + i) sees keys at positions up to
+  its own (the KV cache of "Flash Attention & Paged Attention", section
+  "FA对Prefill阶段的影响": prefill stores K/V that later steps reuse; the
+  mask keeps the same rule as a full prefill of the whole sequence);
+* KV append: the chunk's n new K/V rows take logical positions
+  cache_seqlens[b] - n ... cache_seqlens[b] - 1 of their request and are
+  written through the page table (same page, section 2).
 
 Split/merge (Flash-Decoding, "Flash Attention & Paged Attention", section
 "FA对decode阶段的影响", steps 3-4): each split yields a partial (O_i, LSE_i)
@@ -47,6 +57,12 @@ def kv_head_of(h: int, num_q_heads: int, num_kv_heads: int) -> int:
 def allowed_key_count(i: int, seqlen: int, causal: bool) -> int:
     """Number of leading keys query i (in-sequence index) may attend to."""
     return i + 1 if causal else seqlen
+
+
+def visible_key_count(i: int, q_len: int, k_len: int, causal: bool) -> int:
+    """Keys visible to query i of a chunk whose q_len queries are the last
+    q_len of a k_len-token sequence (i counted from the chunk's start)."""
+    return k_len - q_len + i + 1 if causal else k_len
 
 
 def _scores(q_rows: np.ndarray, keys: np.ndarray, scale: float) -> np.ndarray:
@@ -272,3 +288,110 @@ def merge_states_ref(o_parts, lse_parts):
         lse = np.where(wsum > 0, M_safe + np.log(np.where(wsum > 0, wsum, 1.0)), NEG_INF)
     o = np.where((wsum > 0)[..., None], o, 0.0)
     return o, lse
+
+
+def append_kv_ref(k_pages, v_pages, k_new, v_new, cu_seqlens_new, block_table, cache_seqlens,
+                  page_size: int = 64, layout: str = "NHD"):
+    """Write each request's new K/V rows into its pages (KV-cache append).
+
+    k_new, v_new: [T_new, Hkv, d] packed by ``cu_seqlens_new``; request b's
+    n_b rows go to logical positions cache_seqlens[b] - n_b + i, each at page
+    block_table[b][pos // page_size], slot pos % page_size.  Returns new
+    (k_pages, v_pages) arrays; every other slot keeps its contents.
+    """
+    kp = np.array(k_pages, copy=True)
+    vp = np.array(v_pages, copy=True)
+    cu = [int(x) for x in cu_seqlens_new]
+    for b in range(len(cu) - 1):
+        n = cu[b + 1] - cu[b]
+        first = int(cache_seqlens[b]) - n
+        if first < 0:
+            raise ValueError("cache length shorter than the appended chunk")
+        for i in range(n):
+            pos = first + i
+            phys = int(block_table[b][pos // page_size])
+            slot = pos % page_size
+            if layout == "NHD":
+                kp[phys, slot] = k_new[cu[b] + i]
+                vp[phys, slot] = v_new[cu[b] + i]
+            else:
+                kp[phys, :, slot] = k_new[cu[b] + i]
+                vp[phys, :, slot] = v_new[cu[b] + i]
+    return kp, vp
+
+
+def _chunk_causal_mask(q_len: int, k_len: int) -> np.ndarray:
+    """True where key j is NOT visible to query i of the chunk."""
+    i = np.arange(q_len)[:, None]
+    j = np.arange(k_len)[None, :]
+    return j > (k_len - q_len + i)
+
+
+def paged_prefill_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens,
+                      causal: bool, scale=None, page_size: int = 64, layout: str = "NHD",
+                      to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+    """Chunked prefill: each request's new queries against its whole paged cache.
+
+    q: [Tq, Hq, d] packed by ``cu_seqlens_q``; request b's cache holds
+    cache_seqlens[b] >= q_len_b tokens (the chunk's own K/V included).
+    Returns (O [Tq, Hq, d], LSE [Tq, Hq]).
+    """
+    q = np.asarray(q)
+    Tq, Hq, d = q.shape
+    Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = np.zeros((Tq, Hq, d))
+    lse = np.full((Tq, Hq), NEG_INF)
+    cu = [int(x) for x in cu_seqlens_q]
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        Lq, Lk = s1 - s0, int(cache_seqlens[b])
+        if Lk < Lq:
+            raise ValueError("cache length shorter than the chunk")
+        for g in range(Hkv):
+            K, V = gather_paged_kv(k_pages, v_pages, block_table[b], Lk, g, page_size, layout)
+            K, V = to_f64(K), to_f64(V)
+            for h in range(Hq):
+                if kv_head_of(h, Hq, Hkv) != g:
+                    continue
+                S = _scores(to_f64(q[s0:s1, h]), K, scale)
+                if causal:
+                    S = np.where(_chunk_causal_mask(Lq, Lk), NEG_INF, S)
+                P, l = _softmax_with_lse(S)
+                out[s0:s1, h] = P @ V
+                lse[s0:s1, h] = l
+    return out, lse
+
+
+def paged_prefill_rows_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens,
+                           causal: bool, scale, rows, page_size: int = 64, layout: str = "NHD",
+                           to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+    """Selected rows (token, q_head) of ``paged_prefill_ref``, each on its own.
+
+    Returns (O [n, d], LSE [n]).
+    """
+    q = np.asarray(q)
+    Tq, Hq, d = q.shape
+    Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    cu = np.asarray(cu_seqlens_q, dtype=np.int64)
+    rows = list(rows)
+    out = np.zeros((len(rows), d))
+    lse = np.zeros(len(rows))
+    cache = {}
+    for n, (t, h) in enumerate(rows):
+        b = int(np.searchsorted(cu, t, side="right") - 1)
+        Lq, Lk = int(cu[b + 1] - cu[b]), int(cache_seqlens[b])
+        i = t - int(cu[b])
+        g = kv_head_of(h, Hq, Hkv)
+        if (b, g) not in cache:
+            K, V = gather_paged_kv(k_pages, v_pages, block_table[b], Lk, g, page_size, layout)
+            cache = {(b, g): (to_f64(K), to_f64(V))}
+        K, V = cache[(b, g)]
+        nk = visible_key_count(i, Lq, Lk, causal)
+        P, l = _softmax_with_lse(_scores(to_f64(q[t, h])[None, :], K[:nk], scale))
+        out[n] = (P @ V[:nk])[0]
+        lse[n] = l[0]
+    return out, lse

@@ -291,3 +291,122 @@ def pin_decode_walk(paged_decode_ref, partial_state_ref, layout="NHD", seed=101)
             ob, lb = partial_state_ref(q[b, h][None], K[:, gh], V[:, gh], 0.6)
             _close(o[b, h], ob[0], 1e-13, f"decode walk O b={b} h={h}")
             _close(l[b, h], lb[0], 1e-13, f"decode walk LSE b={b} h={h}")
+
+
+# --- chunked (paged) prefill and KV append ----------------------------------
+
+def pin_golden_append(append_kv_ref):
+    g = load_golden("chunked_prefill_append.json")
+    kp, vp = append_kv_ref(np.array(g["k_pages_before"]), np.array(g["v_pages_before"]),
+                           np.array(g["k_new"]), np.array(g["v_new"]), g["cu_seqlens_new"],
+                           np.array(g["block_table"]), g["cache_seqlens"], page_size=g["page_size"])
+    _close(kp, g["k_pages_after"], 0.0, "append K pages")
+    _close(vp, g["v_pages_after"], 0.0, "append V pages")
+
+
+def pin_golden_chunked(paged_prefill_ref):
+    g = load_golden("chunked_prefill_append.json")
+    for mode in ("causal", "noncausal"):
+        o, l = paged_prefill_ref(np.array(g["q"]), g["cu_seqlens_q"], np.array(g["k_pages_after"]),
+                                 np.array(g["v_pages_after"]), np.array(g["block_table"]),
+                                 g["cache_seqlens"], mode == "causal", g["scale"],
+                                 page_size=g["page_size"])
+        _close(o, g[mode]["o"], 1e-13, f"chunked {mode} O")
+        _close(l, g[mode]["lse"], 1e-13, f"chunked {mode} LSE")
+
+
+def _scatter_to_pages(seqs, ps, layout, g, spare=2):
+    """Place each request's contiguous K/V ([L, Hkv, d] pairs) into randomly
+    chosen physical pages by hand; returns (k_pages, v_pages, block_table)."""
+    hkv, d = seqs[0][0].shape[1:]
+    npages = [(K.shape[0] + ps - 1) // ps for K, _ in seqs]
+    P = sum(npages) + spare
+    perm = g.permutation(P)
+    shape = (P, ps, hkv, d) if layout == "NHD" else (P, hkv, ps, d)
+    kp = g.standard_normal(shape) * 50.0      # slots nobody owns hold large junk
+    vp = g.standard_normal(shape) * 50.0
+    bt = np.full((len(seqs), max(1, max(npages))), -1)
+    off = 0
+    for b, (K, V) in enumerate(seqs):
+        for t in range(K.shape[0]):
+            phys = perm[off + t // ps]
+            bt[b, t // ps] = phys
+            if layout == "NHD":
+                kp[phys, t % ps] = K[t]
+                vp[phys, t % ps] = V[t]
+            else:
+                kp[phys, :, t % ps] = K[t]
+                vp[phys, :, t % ps] = V[t]
+        off += npages[b]
+    return kp, vp, bt
+
+
+def pin_chunk_matches_full(paged_prefill_ref, attention_ref, layout="NHD", seed=111):
+    """A chunk of the last q_len queries of a sequence must reproduce the same
+    rows of a causal prefill over the whole sequence (the prefix is cached)."""
+    g = np.random.default_rng(seed)
+    hq, hkv, d, ps = 4, 2, 6, 4
+    cases = [(0, 7), (5, 1), (9, 4), (3, 13), (8, 8)]      # (cached prefix, chunk)
+    seqs, qs, full = [], [], []
+    for prefix, n in cases:
+        L = prefix + n
+        q = g.standard_normal((L, hq, d))
+        K = g.standard_normal((L, hkv, d))
+        V = g.standard_normal((L, hkv, d))
+        seqs.append((K, V))
+        qs.append(q[prefix:])
+        full.append(attention_ref(q, K, V, [0, L], True, 0.45))
+    kp, vp, bt = _scatter_to_pages(seqs, ps, layout, g)
+    cu = np.concatenate([[0], np.cumsum([n for _, n in cases])])
+    lens = [p + n for p, n in cases]
+    o, l = paged_prefill_ref(np.concatenate(qs), cu, kp, vp, bt, lens, True, 0.45,
+                             page_size=ps, layout=layout)
+    for b, (prefix, n) in enumerate(cases):
+        of, lf = full[b]
+        _close(o[cu[b]:cu[b + 1]], of[prefix:], 1e-12, f"chunk vs full O case {b}")
+        _close(l[cu[b]:cu[b + 1]], lf[prefix:], 1e-12, f"chunk vs full LSE case {b}")
+
+
+def pin_sdpa_lower_right(paged_prefill_ref, seed=121):
+    """PyTorch CPU scaled_dot_product_attention in float64 with its own
+    lower-right causal bias (torch.nn.attention.bias.causal_lower_right) and
+    enable_gqa, on the gathered contiguous K/V of each request."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention.bias import causal_lower_right
+
+    g = np.random.default_rng(seed)
+    hq, hkv, d, ps = 6, 2, 5, 4
+    cases = [(3, 2), (0, 5), (11, 6), (2, 1)]
+    seqs = [(g.standard_normal((p + n, hkv, d)), g.standard_normal((p + n, hkv, d))) for p, n in cases]
+    kp, vp, bt = _scatter_to_pages(seqs, ps, "NHD", g)
+    cu = np.concatenate([[0], np.cumsum([n for _, n in cases])])
+    q = g.standard_normal((int(cu[-1]), hq, d))
+    lens = [p + n for p, n in cases]
+    for causal in (False, True):
+        o, l = paged_prefill_ref(q, cu, kp, vp, bt, lens, causal, 0.35, page_size=ps)
+        for b, (p, n) in enumerate(cases):
+            K, V = seqs[b]
+            tq = torch.from_numpy(q[cu[b]:cu[b + 1]]).permute(1, 0, 2)[None]
+            tk = torch.from_numpy(K).permute(1, 0, 2)[None]
+            tv = torch.from_numpy(V).permute(1, 0, 2)[None]
+            mask = causal_lower_right(n, p + n) if causal else None
+            ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.35,
+                                                 enable_gqa=True)
+            _close(o[cu[b]:cu[b + 1]], ref[0].permute(1, 0, 2).numpy(), 1e-12,
+                   f"sdpa lower-right case {b} causal={causal}")
+
+
+def pin_chunk_single_query_is_decode(paged_prefill_ref, paged_decode_ref, seed=131):
+    """A one-token chunk under causal masking sees the whole cache: decode."""
+    g = np.random.default_rng(seed)
+    hq, hkv, d, ps = 4, 1, 3, 4
+    lens = [1, 6, 9]
+    seqs = [(g.standard_normal((L, hkv, d)), g.standard_normal((L, hkv, d))) for L in lens]
+    kp, vp, bt = _scatter_to_pages(seqs, ps, "HND", g)
+    q = g.standard_normal((len(lens), hq, d))
+    o, l = paged_prefill_ref(q, np.arange(len(lens) + 1), kp, vp, bt, lens, True, 0.8,
+                             page_size=ps, layout="HND")
+    od, ld = paged_decode_ref(q, kp, vp, bt, lens, 0.8, page_size=ps, layout="HND")
+    _close(o, od, 1e-13, "single-query chunk vs decode O")
+    _close(l, ld, 1e-13, "single-query chunk vs decode LSE")

@@ -114,3 +114,74 @@ def test_paged_walk_mutant_is_caught(monkeypatch):
     pins = [lambda: P.pin_golden_paged(A.paged_decode_ref),
             lambda: P.pin_decode_walk(A.paged_decode_ref, A.partial_state_ref)]
     assert _some_pin_fires(pins)
+
+
+CHUNKED_PINS = [
+    lambda: P.pin_golden_chunked(A.paged_prefill_ref),
+    lambda: P.pin_chunk_matches_full(A.paged_prefill_ref, A.attention_ref),
+    lambda: P.pin_sdpa_lower_right(A.paged_prefill_ref),
+    lambda: P.pin_chunk_single_query_is_decode(A.paged_prefill_ref, A.paged_decode_ref),
+]
+
+CHUNK_MASK_MUTANTS = {
+    # top-left alignment: query i of the chunk sees keys 0..i
+    "top_left": lambda q_len, k_len: np.arange(k_len)[None, :] > np.arange(q_len)[:, None],
+    # off by one: the query's own position masked
+    "excludes_own": lambda q_len, k_len: (np.arange(k_len)[None, :]
+                                          >= (k_len - q_len + np.arange(q_len))[:, None]),
+    # offset in the wrong direction
+    "offset_sign": lambda q_len, k_len: (np.arange(k_len)[None, :]
+                                         > (q_len - k_len + np.arange(q_len))[:, None]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CHUNK_MASK_MUTANTS))
+def test_chunk_mask_mutant_is_caught(name, monkeypatch):
+    monkeypatch.setattr(A, "_chunk_causal_mask", CHUNK_MASK_MUTANTS[name])
+    with np.errstate(all="ignore"):
+        assert _some_pin_fires(CHUNKED_PINS), f"no pin caught mutant {name}"
+
+
+def test_chunked_paged_walk_mutant_is_caught(monkeypatch):
+    """The chunked prefill reading physical pages in order, ignoring the table."""
+    def bad_gather(k_pages, v_pages, row, seqlen, g, ps, layout="NHD"):
+        n = (seqlen + ps - 1) // ps
+        if n == 0:
+            return np.zeros((0, k_pages.shape[-1])), np.zeros((0, k_pages.shape[-1]))
+        if layout == "NHD":
+            return (np.concatenate([k_pages[p, :, g] for p in range(n)])[:seqlen],
+                    np.concatenate([v_pages[p, :, g] for p in range(n)])[:seqlen])
+        return (np.concatenate([k_pages[p, g] for p in range(n)])[:seqlen],
+                np.concatenate([v_pages[p, g] for p in range(n)])[:seqlen])
+    monkeypatch.setattr(A, "gather_paged_kv", bad_gather)
+    assert _some_pin_fires(CHUNKED_PINS)
+
+
+def _append_from_old_length(kp, vp, kn, vn, cu, bt, lens, page_size=64, layout="NHD"):
+    """Mistake: treats cache_seqlens as the length before the append."""
+    n = np.diff(np.asarray(cu))
+    return A.append_kv_ref(kp, vp, kn, vn, cu, bt, np.asarray(lens) + n, page_size, layout)
+
+
+def _append_slot_from_page_index(kp, vp, kn, vn, cu, bt, lens, page_size=64, layout="NHD"):
+    """Mistake: page and slot swapped (pos % page_size picks the page)."""
+    kp = np.array(kp, copy=True)
+    vp = np.array(vp, copy=True)
+    for b in range(len(cu) - 1):
+        n = cu[b + 1] - cu[b]
+        for i in range(n):
+            pos = int(lens[b]) - n + i
+            phys = int(bt[b][pos % page_size])
+            kp[phys, pos // page_size] = kn[cu[b] + i]
+            vp[phys, pos // page_size] = vn[cu[b] + i]
+    return kp, vp
+
+
+@pytest.mark.parametrize("bad", [_append_from_old_length, _append_slot_from_page_index])
+def test_append_mutant_is_caught(bad):
+    with np.errstate(all="ignore"):
+        try:
+            P.pin_golden_append(bad)
+        except (AssertionError, IndexError):
+            return
+    raise AssertionError("append mutant not caught")

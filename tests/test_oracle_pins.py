@@ -132,3 +132,48 @@ def test_tiny_config_rounding_effect_reported():
                                   True, inp.scale)
     assert np.isfinite(o1).all() and np.isfinite(l1).all()
     assert np.max(np.abs(l1 - l2)) > 0.0
+
+
+def test_golden_append():
+    P.pin_golden_append(oracle.append_kv_ref)
+
+
+def test_golden_chunked():
+    P.pin_golden_chunked(oracle.paged_prefill_ref)
+
+
+@pytest.mark.parametrize("layout", ["NHD", "HND"])
+def test_chunk_matches_full(layout):
+    P.pin_chunk_matches_full(oracle.paged_prefill_ref, oracle.attention_ref, layout)
+
+
+def test_sdpa_lower_right():
+    P.pin_sdpa_lower_right(oracle.paged_prefill_ref)
+
+
+def test_chunk_single_query_is_decode():
+    P.pin_chunk_single_query_is_decode(oracle.paged_prefill_ref, oracle.paged_decode_ref)
+
+
+def test_paged_prefill_rows_match_full():
+    g = np.random.default_rng(141)
+    hq, hkv, d, ps = 4, 2, 4, 4
+    cases = [(5, 3), (0, 6)]
+    seqs = [(g.standard_normal((p + n, hkv, d)), g.standard_normal((p + n, hkv, d))) for p, n in cases]
+    kp, vp, bt = P._scatter_to_pages(seqs, ps, "NHD", g)
+    cu = np.array([0, 3, 9])
+    q = g.standard_normal((9, hq, d))
+    lens = [8, 6]
+    for causal in (False, True):
+        o, l = oracle.paged_prefill_ref(q, cu, kp, vp, bt, lens, causal, 0.5, page_size=ps)
+        rows = [(t, h) for t in range(9) for h in range(hq)]
+        orr, lr = oracle.paged_prefill_rows_ref(q, cu, kp, vp, bt, lens, causal, 0.5, rows, page_size=ps)
+        np.testing.assert_allclose(orr, o.reshape(-1, d), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lr, l.reshape(-1), rtol=0, atol=1e-14)
+
+
+def test_visible_key_count_reduces_to_square_causal():
+    for L in (1, 5):
+        for i in range(L):
+            assert oracle.visible_key_count(i, L, L, True) == i + 1
+            assert oracle.visible_key_count(i, L, L, False) == L

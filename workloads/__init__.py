@@ -341,6 +341,175 @@ def poison_unused(inp: DecodeInputs) -> DecodeInputs:
                         inp.cache_seqlens, inp.scale, inp.layout, inp.page_size, dict(inp.extra))
 
 
+# ---------------------------------------------------------------------------
+# Chunked (paged) prefill workloads
+# ---------------------------------------------------------------------------
+
+@dataclass
+class ChunkedPrefillInputs:
+    """A batch of prefill chunks over paged caches that already hold a prefix.
+
+    Request b has ``prefix_lens[b]`` cached tokens in its pages and a new chunk
+    of ``chunk_lens[b]`` tokens: its queries (``q_bits``) and its K/V rows
+    (``k_new_bits``/``v_new_bits``), all packed by ``cu_seqlens_q``.  The pages
+    already reserve room for the chunk (``cache_seqlens`` = prefix + chunk, the
+    length after the append); the chunk's slots hold stale values until the
+    append writes them.
+    """
+    name: str
+    q_bits: np.ndarray            # [Tq, Hq, d]
+    k_new_bits: np.ndarray        # [Tq, Hkv, d]
+    v_new_bits: np.ndarray
+    cu_seqlens_q: np.ndarray      # [B+1] int32
+    k_pages_bits: np.ndarray      # NHD [P, page, Hkv, d] or HND [P, Hkv, page, d]
+    v_pages_bits: np.ndarray
+    block_table: np.ndarray       # [B, max_pages] int32 (unused = -1)
+    cache_seqlens: np.ndarray     # [B] int32, after the append
+    causal: bool
+    scale: float
+    layout: str = "NHD"
+    page_size: int = PAGE_SIZE
+
+    @property
+    def batch(self):
+        return len(self.cache_seqlens)
+
+    @property
+    def num_q_heads(self):
+        return self.q_bits.shape[1]
+
+    @property
+    def num_kv_heads(self):
+        return self.k_new_bits.shape[1]
+
+    @property
+    def head_dim(self):
+        return self.q_bits.shape[2]
+
+    @property
+    def num_pages(self):
+        return self.k_pages_bits.shape[0]
+
+    @property
+    def chunk_lens(self):
+        return np.diff(self.cu_seqlens_q).astype(np.int64)
+
+    @property
+    def prefix_lens(self):
+        return self.cache_seqlens.astype(np.int64) - self.chunk_lens
+
+    def strides(self):
+        """(page_stride, token_stride, head_stride) in elements."""
+        P, a, b, d = self.k_pages_bits.shape
+        if self.layout == "NHD":
+            return a * b * d, b * d, d
+        return a * b * d, d, b * d
+
+    def causal_flops(self) -> float:
+        """Algorithmic FLOPs: 4*d*Hq per (query, visible key) pair."""
+        n = self.chunk_lens
+        k = self.cache_seqlens.astype(np.int64)
+        pairs = (n * (k - n) + n * (n + 1) // 2).sum() if self.causal else (n * k).sum()
+        return 4.0 * self.head_dim * self.num_q_heads * float(pairs)
+
+    def append_bytes(self) -> float:
+        """KV append traffic: the new K and V rows read once and written once."""
+        return 4.0 * self.k_new_bits.size * 2
+
+    def attention_bytes(self) -> float:
+        """Minimum HBM bytes of the attention: Q read, O written, every cached
+        K/V row of each kv head read once."""
+        Tq, Hq, d = self.q_bits.shape
+        kv = 2.0 * float(self.cache_seqlens.astype(np.int64).sum()) * self.num_kv_heads * d * 2
+        return kv + 2.0 * Tq * Hq * d * 2 + Tq * Hq * 4
+
+
+def make_chunked_prefill(prefix_lens, chunk_lens, num_q_heads, num_kv_heads, head_dim, *,
+                         seed=6, causal=True, page_size=PAGE_SIZE, layout="NHD", scale=None,
+                         extra_pages=0, name="chunked_prefill") -> ChunkedPrefillInputs:
+    prefix_lens = np.asarray(prefix_lens, dtype=np.int64)
+    chunk_lens = np.asarray(chunk_lens, dtype=np.int64)
+    assert prefix_lens.shape == chunk_lens.shape and (chunk_lens >= 1).all()
+    total = prefix_lens + chunk_lens
+    B = len(total)
+    npages = (total + page_size - 1) // page_size
+    P = int(npages.sum()) + int(extra_pages)
+    ss = np.random.SeedSequence(seed)
+    s_perm, s_q, s_kn, s_vn, s_k, s_v = ss.spawn(6)
+    perm = np.random.Generator(np.random.PCG64(s_perm)).permutation(P).astype(np.int32)
+    bt = np.full((B, int(max(1, npages.max()))), -1, dtype=np.int32)
+    off = 0
+    for b in range(B):
+        n = int(npages[b])
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    if layout == "NHD":
+        shape = (P, page_size, num_kv_heads, head_dim)
+    elif layout == "HND":
+        shape = (P, num_kv_heads, page_size, head_dim)
+    else:
+        raise ValueError(layout)
+    cu = np.zeros(B + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(chunk_lens)
+    Tq = int(cu[-1])
+    q = _normal_bf16_bits(s_q, (Tq, num_q_heads, head_dim))
+    kn = _normal_bf16_bits(s_kn, (Tq, num_kv_heads, head_dim))
+    vn = _normal_bf16_bits(s_vn, (Tq, num_kv_heads, head_dim))
+    kp = _normal_bf16_bits(s_k, shape)
+    vp = _normal_bf16_bits(s_v, shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    return ChunkedPrefillInputs(name, q, kn, vn, cu, kp, vp, bt, total.astype(np.int32), causal,
+                                float(scale), layout, page_size)
+
+
+def tiny_chunked_prefill(head_dim=128, layout="NHD", causal=True) -> ChunkedPrefillInputs:
+    """Five requests whose (prefix, chunk) pairs cover an empty prefix, a
+    one-token chunk, page-aligned ends and page tails in either half of a
+    128-key tile; 4 q / 2 kv heads."""
+    return make_chunked_prefill([0, 100, 700, 64, 1000], [130, 1, 257, 64, 300], 4, 2, head_dim,
+                                seed=7, causal=causal, layout=layout, extra_pages=3,
+                                name="tiny_chunked_prefill")
+
+
+def chunked_prefill_lengths(seed=6, batch=8):
+    g = np.random.default_rng(seed)
+    prefix = g.integers(1024, 16384 + 1, size=batch)
+    chunk = g.integers(256, 2048 + 1, size=batch)
+    return prefix.astype(np.int64), chunk.astype(np.int64)
+
+
+def chunked_prefill_batch() -> ChunkedPrefillInputs:
+    """8 requests, cached prefix uniform in [1024, 16384], new chunk uniform in
+    [256, 2048], 32 q / 8 kv heads, d=128, causal, shuffled 64-token pages."""
+    prefix, chunk = chunked_prefill_lengths(6)
+    return make_chunked_prefill(prefix, chunk, 32, 8, 128, seed=6, name="chunked_prefill_batch")
+
+
+def poison_chunked(inp: ChunkedPrefillInputs) -> ChunkedPrefillInputs:
+    """NaN in every pool slot outside the cached prefixes: the chunk's own
+    slots (the append must overwrite them), page tails and unused pages."""
+    kp = inp.k_pages_bits.copy()
+    vp = inp.v_pages_bits.copy()
+    ps = inp.page_size
+    valid = np.zeros((inp.num_pages, ps), dtype=bool)
+    for b in range(inp.batch):
+        L = int(inp.prefix_lens[b])
+        for p in range((L + ps - 1) // ps):
+            valid[int(inp.block_table[b, p]), :min(ps, L - p * ps)] = True
+    inv = ~valid
+    if inp.layout == "NHD":
+        kp[inv] = BF16_NAN_BITS
+        vp[inv] = BF16_NAN_BITS
+    else:
+        kp.transpose(0, 2, 1, 3)[inv] = BF16_NAN_BITS
+        vp.transpose(0, 2, 1, 3)[inv] = BF16_NAN_BITS
+    out = ChunkedPrefillInputs(**{**inp.__dict__})
+    out.name = inp.name + "_poison"
+    out.k_pages_bits, out.v_pages_bits = kp, vp
+    return out
+
+
 CONFIGS = {
     "tiny_causal_prefill": tiny_causal_prefill,
     "varlen_causal_prefill": varlen_causal_prefill,
@@ -349,4 +518,6 @@ CONFIGS = {
     "paged_decode_batch16": paged_decode_batch16,
     "long_split_decode": long_split_decode,
     "ragged_split_decode": ragged_split_decode,
+    "tiny_chunked_prefill": tiny_chunked_prefill,
+    "chunked_prefill_batch": chunked_prefill_batch,
 }
