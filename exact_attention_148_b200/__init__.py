@@ -20,6 +20,7 @@ import numpy as np
 __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
     "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
+    "append_kv", "prefill_paged",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +38,7 @@ FA_ERR_BAD_PAGE = -7
 EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
-    "fa_decode_paged_static", "fa_selftest_wait_timeout",
+    "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
 ]
 
 # Size of the library's static decode scratch (FA_STATIC_SCRATCH_BYTES).
@@ -102,6 +103,12 @@ def library() -> ctypes.CDLL:
     L.fa_decode_paged_static.restype = i32
     L.fa_selftest_wait_timeout.argtypes = [i64, vp]
     L.fa_selftest_wait_timeout.restype = i32
+    L.fa_append_kv.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, i64, i64, i64, i64, i32, vp,
+                               i32, vp, vp]
+    L.fa_append_kv.restype = i32
+    L.fa_prefill_paged.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, vp, vp, i32,
+                                   i32, i32, i32, i32, i32, f32, vp, vp, vp]
+    L.fa_prefill_paged.restype = i32
     _lib = L
     return L
 
@@ -303,6 +310,86 @@ def decode_paged_static(q, k_pages, v_pages, block_table, cache_seqlens, plan: D
         _ptr(q), _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(block_table),
         _ptr(cache_seqlens), plan.handle, _scale_arg(scale), _ptr(out), _ptr(lse), _stream_ptr(stream))
     _check(st, "fa_decode_paged_static")
+    return out, lse
+
+
+def _check_pool(k_pages, v_pages, block_table):
+    torch = _torch()
+    if k_pages.dtype != torch.bfloat16 or v_pages.dtype != torch.bfloat16:
+        raise ValueError("k_pages and v_pages must be bfloat16")
+    if not (k_pages.is_contiguous() and v_pages.is_contiguous() and block_table.is_contiguous()):
+        raise ValueError("k_pages, v_pages and block_table must be contiguous")
+    if k_pages.shape != v_pages.shape or k_pages.dim() != 4:
+        raise ValueError("k_pages and v_pages must be 4-D with the same shape")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise ValueError("block_table must be a 2-D int32 tensor")
+
+
+def append_kv(k_new, v_new, cu_seqlens_new, k_pages, v_pages, block_table, cache_seqlens, *,
+              layout: str = "NHD", stream=None):
+    """Write new K/V rows into the paged cache (in place).
+
+    k_new/v_new [T_new, Hkv, d] bf16 packed by cu_seqlens_new [B+1] int32;
+    cache_seqlens [B] int32 are the lengths after the append: request b's new
+    rows go to logical positions cache_seqlens[b] - n_b ... cache_seqlens[b] - 1.
+    """
+    torch = _torch()
+    _require_cuda(k_new, v_new, cu_seqlens_new, k_pages, v_pages, block_table, cache_seqlens)
+    _check_pool(k_pages, v_pages, block_table)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous 3-D bfloat16 tensor")
+    if k_new.shape != v_new.shape:
+        raise ValueError("k_new and v_new must have the same shape")
+    if cu_seqlens_new.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens_new and cache_seqlens must be int32")
+    T, Hkv, d = k_new.shape
+    ps, ts, hs = page_strides(k_pages, layout)
+    page_size = k_pages.shape[1] if layout == "NHD" else k_pages.shape[2]
+    st = library().fa_append_kv(
+        _ptr(k_new), _ptr(v_new), _ptr(cu_seqlens_new), T, cu_seqlens_new.numel() - 1, Hkv, d,
+        _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, page_size, _ptr(block_table),
+        block_table.shape[1], _ptr(cache_seqlens), _stream_ptr(stream))
+    _check(st, "fa_append_kv")
+
+
+def prefill_paged(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens, *,
+                  causal: bool = True, scale: float | None = None, layout: str = "NHD",
+                  out=None, lse=None, cu_seqlens_q_host=None, cache_seqlens_host=None,
+                  return_lse: bool = True, stream=None):
+    """Chunked prefill: new queries [Tq, Hq, d] (packed by cu_seqlens_q) against
+    each request's whole paged cache of cache_seqlens[b] keys; causal queries
+    are the last q_len positions of their sequence.  Returns (out, lse)."""
+    torch = _torch()
+    _require_cuda(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens, out, lse)
+    _check_pool(k_pages, v_pages, block_table)
+    if q.dtype != torch.bfloat16 or not q.is_contiguous() or q.dim() != 3:
+        raise ValueError("q must be a contiguous 3-D bfloat16 tensor")
+    if cu_seqlens_q.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens_q and cache_seqlens must be int32")
+    T, Hq, d = q.shape
+    Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
+    page_size = k_pages.shape[1] if layout == "NHD" else k_pages.shape[2]
+    if cu_seqlens_q_host is None:
+        cu_seqlens_q_host = cu_seqlens_q.cpu().numpy()
+    if cache_seqlens_host is None:
+        cache_seqlens_host = cache_seqlens.cpu().numpy()
+    cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_q_host, dtype=np.int32))
+    len_h = np.ascontiguousarray(np.asarray(cache_seqlens_host, dtype=np.int32))
+    batch = len(cu_h) - 1
+    if len(len_h) != batch:
+        raise ValueError("cache_seqlens must have one entry per request")
+    ps, ts, hs = page_strides(k_pages, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    st = library().fa_prefill_paged(
+        _ptr(q), _ptr(cu_seqlens_q), cu_h.ctypes.data_as(ctypes.c_void_p), _ptr(k_pages),
+        _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(block_table), block_table.shape[1],
+        _ptr(cache_seqlens), len_h.ctypes.data_as(ctypes.c_void_p), batch, Hq, Hkv, d, page_size,
+        1 if causal else 0, _scale_arg(scale), _ptr(out), _ptr(lse), _stream_ptr(stream))
+    _check(st, "fa_prefill_paged")
     return out, lse
 
 

@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "../../include/exact_attention.h"
+#include "append_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "planner.h"
 #include "prefill_pp_sm100.cuh"
@@ -89,12 +90,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------- prefill
 // groups: (sequence << 16 | kv head, number of CTAs) in launch order.
-template <int D>
+template <int D, bool PAGED>
 int launch_prefill(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t, int>>& groups,
                    cudaStream_t stream) {
   constexpr int kSmem = fa::PrefillPPCfg<D>::SMEM_BYTES;
   constexpr int kThreads = fa::kPrefillPPThreads;
-  auto kernel = fa::fa_prefill_pp_kernel<D>;
+  auto kernel = fa::fa_prefill_pp_kernel<D, PAGED>;
   int st = ensure_smem(reinterpret_cast<const void*>(kernel), kSmem);
   if (st != FA_OK) return st;
   for (size_t off = 0; off < groups.size(); off += fa::kPrefillMaxGroups) {
@@ -112,6 +113,71 @@ int launch_prefill(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t,
     FA_CUDA_CHECK(cudaGetLastError());
   }
   return FA_OK;
+}
+
+// Launch order of the prefill CTAs: sequences heaviest first (most query-key
+// pairs; their groups carry the most work), one group of CTAs per (sequence,
+// kv head).  A CTA takes two heads of the group at one q tile when the group
+// is even, else two consecutive q tiles of one head, so a group has
+// ceil(Lq/128) * G/2 or ceil(ceil(Lq/128)/2) * G CTAs.
+// q_lens[b] >= 1 queries, k_lens[b] >= q_lens[b] keys (equal when unpaged).
+int build_prefill_groups(const std::vector<int64_t>& q_lens, const std::vector<int64_t>& k_lens,
+                         int num_q_heads, int num_kv_heads, bool causal,
+                         std::vector<std::pair<uint32_t, int>>* groups) {
+  const int batch = static_cast<int>(q_lens.size());
+  std::vector<std::pair<double, int>> by_work;   // (query-key pairs, sequence)
+  for (int b = 0; b < batch; ++b) {
+    const double lq = static_cast<double>(q_lens[b]), lk = static_cast<double>(k_lens[b]);
+    by_work.emplace_back(causal ? lq * (lk - lq) + 0.5 * lq * (lq + 1.0) : lq * lk, b);
+  }
+  std::stable_sort(by_work.begin(), by_work.end(),
+                   [](const auto& a, const auto& b) { return a.first > b.first; });
+  const int group = num_q_heads / num_kv_heads;
+  groups->clear();
+  groups->reserve(static_cast<size_t>(batch) * num_kv_heads);
+  for (const auto& e : by_work) {
+    const int ntiles = static_cast<int>((q_lens[e.second] + 127) / 128);
+    const int ctas = (group % 2 == 0) ? ntiles * (group / 2) : ((ntiles + 1) / 2) * group;
+    for (int g = 0; g < num_kv_heads; ++g)
+      groups->emplace_back((static_cast<uint32_t>(e.second) << 16) | static_cast<uint32_t>(g), ctas);
+  }
+  return FA_OK;
+}
+
+// 4-D tensor map over a K or V page pool: dim 0 = the d contiguous columns,
+// dims 1..3 = token slot, kv head and page ordered by increasing stride.  The
+// box is `box_cols` columns x a whole page of tokens x 1 head x 1 page.
+// Reports which dimension holds the kv head and which the page.
+int encode_page_pool_map(CUtensorMap* map, const void* pool, int64_t num_pages, int64_t page_stride,
+                         int64_t token_stride, int64_t head_stride, int page_size, int num_kv_heads,
+                         int head_dim, int box_cols, CUtensorMapSwizzle swz, int* head_coord,
+                         int* page_coord) {
+  struct Dim { int64_t stride; int64_t extent; int role; };   // role 0 token, 1 head, 2 page
+  Dim dd[3] = {{token_stride, page_size, 0}, {head_stride, num_kv_heads, 1},
+               {page_stride, num_pages, 2}};
+  std::sort(dd, dd + 3, [](const Dim& a, const Dim& b) { return a.stride < b.stride; });
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), 0, 0, 0};
+  cuuint64_t strides[3];
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), 1, 1, 1};
+  for (int i = 0; i < 3; ++i) {
+    dims[i + 1] = static_cast<cuuint64_t>(dd[i].extent);
+    strides[i] = static_cast<cuuint64_t>(dd[i].stride) * 2;
+    if (dd[i].role == 0) box[i + 1] = static_cast<cuuint32_t>(page_size);
+    if (dd[i].role == 1) *head_coord = i + 1;
+    if (dd[i].role == 2) *page_coord = i + 1;
+  }
+  return encode_map(map, pool, 4, dims, strides, box, swz);
+}
+
+// Shared checks of a page pool's description (element strides).
+bool valid_pool(const void* k_pages, const void* v_pages, int64_t num_pages, int64_t page_stride,
+                int64_t token_stride, int64_t head_stride) {
+  if (!k_pages || !v_pages || !aligned(k_pages, 16) || !aligned(v_pages, 16)) return false;
+  if (num_pages < 1 || num_pages > INT32_MAX) return false;
+  if (page_stride <= 0 || token_stride <= 0 || head_stride <= 0 || page_stride % 8 ||
+      token_stride % 8 || head_stride % 8)
+    return false;
+  return true;
 }
 
 // ---------------------------------------------------------------------------- decode
@@ -167,30 +233,18 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
   if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
   if (cu_seqlens_host[0] != 0) return FA_ERR_INVALID_ARG;
   if (num_kv_heads > 65535) return FA_ERR_UNSUPPORTED;
-  // Sequences longest first (their groups carry the most work); each sequence
-  // contributes one group of ceil(L/128) * (Hq/Hkv) CTAs per kv head.
-  std::vector<std::pair<int64_t, int>> by_len;   // (length, sequence)
+  std::vector<int64_t> lens;
   for (int b = 0; b < batch; ++b) {
     const int64_t L = static_cast<int64_t>(cu_seqlens_host[b + 1]) - cu_seqlens_host[b];
     if (L < 1) return FA_ERR_INVALID_ARG;
     if ((L + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;
-    by_len.emplace_back(L, b);
+    lens.push_back(L);
   }
   const int64_t T = cu_seqlens_host[batch];
   if (T * num_q_heads * head_dim >= (int64_t{1} << 40)) return FA_ERR_UNSUPPORTED;
-  std::stable_sort(by_len.begin(), by_len.end(),
-                   [](const auto& a, const auto& b) { return a.first > b.first; });
   const int group = num_q_heads / num_kv_heads;
   std::vector<std::pair<uint32_t, int>> groups;
-  groups.reserve(static_cast<size_t>(batch) * num_kv_heads);
-  for (const auto& e : by_len) {
-    const int ntiles = static_cast<int>((e.first + 127) / 128);
-    // A CTA takes two heads of the group at one q tile when the group is
-    // even, else two consecutive q tiles of one head.
-    const int ctas = (group % 2 == 0) ? ntiles * (group / 2) : ((ntiles + 1) / 2) * group;
-    for (int g = 0; g < num_kv_heads; ++g)
-      groups.emplace_back((static_cast<uint32_t>(e.second) << 16) | static_cast<uint32_t>(g), ctas);
-  }
+  build_prefill_groups(lens, lens, num_q_heads, num_kv_heads, causal != 0, &groups);
 
   static thread_local fa::PrefillParams prm;   // ~17 KB; kept off the stack
   std::memset(&prm, 0, sizeof(prm));
@@ -221,7 +275,136 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return head_dim == 128 ? launch_prefill<128>(prm, groups, s) : launch_prefill<64>(prm, groups, s);
+  return head_dim == 128 ? launch_prefill<128, false>(prm, groups, s)
+                         : launch_prefill<64, false>(prm, groups, s);
+}
+
+FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
+                            const int32_t* cu_seqlens_q_host, const void* k_pages,
+                            const void* v_pages, int64_t num_pages, int64_t page_stride,
+                            int64_t token_stride, int64_t head_stride, const int32_t* block_table,
+                            int max_pages_per_seq, const int32_t* cache_seqlens_dev,
+                            const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                            int num_kv_heads, int head_dim, int page_size, int causal, float scale,
+                            void* out, float* lse, void* stream) {
+  if (!q || !cu_seqlens_q_dev || !cu_seqlens_q_host || !block_table || !cache_seqlens_dev ||
+      !cache_seqlens_host || !out)
+    return FA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || num_q_heads < 1 || num_kv_heads < 1 ||
+      num_q_heads > 65535 || num_q_heads % num_kv_heads != 0 || max_pages_per_seq < 1)
+    return FA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (page_size != fa::kPrefillPage) return FA_ERR_UNSUPPORTED;
+  if (num_kv_heads > 65535) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(cu_seqlens_q_dev, 4) ||
+      !aligned(block_table, 4) || !aligned(cache_seqlens_dev, 4))
+    return FA_ERR_INVALID_ARG;
+  if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride))
+    return FA_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, head_dim);
+  if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
+  if (cu_seqlens_q_host[0] != 0) return FA_ERR_INVALID_ARG;
+  const int64_t capacity = static_cast<int64_t>(max_pages_per_seq) * page_size;
+  if (capacity > INT32_MAX) return FA_ERR_INVALID_ARG;
+  std::vector<int64_t> q_lens, k_lens;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t lq = static_cast<int64_t>(cu_seqlens_q_host[b + 1]) - cu_seqlens_q_host[b];
+    const int64_t lk = cache_seqlens_host[b];
+    if (lq < 1 || lk < lq || lk > capacity) return FA_ERR_INVALID_ARG;
+    if ((lq + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;
+    q_lens.push_back(lq);
+    k_lens.push_back(lk);
+  }
+  const int64_t T = cu_seqlens_q_host[batch];
+  if (T * num_q_heads * head_dim >= (int64_t{1} << 40)) return FA_ERR_UNSUPPORTED;
+  std::vector<std::pair<uint32_t, int>> groups;
+  build_prefill_groups(q_lens, k_lens, num_q_heads, num_kv_heads, causal != 0, &groups);
+
+  static thread_local fa::PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  {
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                                static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                   static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+    int st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
+  int st = encode_page_pool_map(&prm.tm_k, k_pages, num_pages, page_stride, token_stride, head_stride,
+                                page_size, num_kv_heads, head_dim, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                                &prm.head_coord, &prm.page_coord);
+  if (st != FA_OK) return st;
+  st = encode_page_pool_map(&prm.tm_v, v_pages, num_pages, page_stride, token_stride, head_stride,
+                            page_size, num_kv_heads, head_dim, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                            &prm.head_coord, &prm.page_coord);
+  if (st != FA_OK) return st;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.cu_seqlens = cu_seqlens_q_dev;
+  prm.block_table = block_table;
+  prm.cache_seqlens = cache_seqlens_dev;
+  prm.max_pages = max_pages_per_seq;
+  prm.num_pages = static_cast<int>(num_pages);
+  prm.num_q_heads = num_q_heads;
+  prm.group = num_q_heads / num_kv_heads;
+  prm.causal = causal ? 1 : 0;
+  prm.scale_log2 = scale * kLog2e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return head_dim == 128 ? launch_prefill<128, true>(prm, groups, s)
+                         : launch_prefill<64, true>(prm, groups, s);
+}
+
+FA_API int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_seqlens_new_dev,
+                        int total_new, int batch, int num_kv_heads, int head_dim, void* k_pages,
+                        void* v_pages, int64_t num_pages, int64_t page_stride,
+                        int64_t token_stride, int64_t head_stride, int page_size,
+                        const int32_t* block_table, int max_pages_per_seq,
+                        const int32_t* cache_seqlens_dev, void* stream) {
+  if (!k_new || !v_new || !cu_seqlens_new_dev || !block_table || !cache_seqlens_dev)
+    return FA_ERR_INVALID_ARG;
+  if (total_new < 0 || batch < 1 || num_kv_heads < 1 || max_pages_per_seq < 1)
+    return FA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (page_size != fa::kAppendPage) return FA_ERR_UNSUPPORTED;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(cu_seqlens_new_dev, 4) ||
+      !aligned(block_table, 4) || !aligned(cache_seqlens_dev, 4))
+    return FA_ERR_INVALID_ARG;
+  if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride))
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_pages_per_seq) * page_size > INT32_MAX) return FA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(total_new) * num_kv_heads * head_dim >= (int64_t{1} << 40))
+    return FA_ERR_UNSUPPORTED;
+  if (total_new == 0) return FA_OK;
+  fa::AppendParams ap;
+  ap.k_new = static_cast<const uint4*>(k_new);
+  ap.v_new = static_cast<const uint4*>(v_new);
+  ap.cu_seqlens = cu_seqlens_new_dev;
+  ap.cache_seqlens = cache_seqlens_dev;
+  ap.block_table = block_table;
+  ap.k_pages = static_cast<__nv_bfloat16*>(k_pages);
+  ap.v_pages = static_cast<__nv_bfloat16*>(v_pages);
+  ap.page_stride = page_stride;
+  ap.token_stride = token_stride;
+  ap.head_stride = head_stride;
+  ap.total_new = total_new;
+  ap.batch = batch;
+  ap.num_kv_heads = num_kv_heads;
+  ap.max_pages = max_pages_per_seq;
+  ap.num_pages = static_cast<int>(num_pages);
+  // One warp per token; at most 16 resident blocks per SM's worth of grid.
+  int dev = 0, sms = 148;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  FA_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int64_t want = (static_cast<int64_t>(total_new) + 7) / 8;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128)
+    fa::fa_append_kv_kernel<128><<<grid, fa::kAppendThreads, 0, s>>>(ap);
+  else
+    fa::fa_append_kv_kernel<64><<<grid, fa::kAppendThreads, 0, s>>>(ap);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
 }
 
 FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
@@ -279,9 +462,7 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
   if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
       !aligned(lse, 4) || !aligned(block_table, 4) || !aligned(cache_seqlens_dev, 4))
     return FA_ERR_INVALID_ARG;
-  if (num_pages < 1 || num_pages > INT32_MAX) return FA_ERR_INVALID_ARG;
-  if (page_stride <= 0 || token_stride <= 0 || head_stride <= 0 || page_stride % 8 ||
-      token_stride % 8 || head_stride % 8)
+  if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride))
     return FA_ERR_INVALID_ARG;
   if (pl.workspace_bytes > 0) {
     if (workspace == nullptr || !aligned(workspace, 256)) return FA_ERR_INVALID_ARG;
@@ -292,25 +473,14 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
 
   static thread_local fa::DecodeParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  // 4-D map over the pool: dim 0 = d (contiguous); dims 1..3 = token slot,
-  // kv head, page, ordered by increasing stride.
-  struct Dim { int64_t stride; int64_t extent; int role; };   // role 0 token, 1 head, 2 page
-  Dim dd[3] = {{token_stride, pl.page_size, 0}, {head_stride, pl.num_kv_heads, 1},
-               {page_stride, num_pages, 2}};
-  std::sort(dd, dd + 3, [](const Dim& a, const Dim& b) { return a.stride < b.stride; });
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(pl.head_dim), 0, 0, 0};
-  cuuint64_t strides[3];
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(pl.head_dim), 1, 1, 1};
-  for (int i = 0; i < 3; ++i) {
-    dims[i + 1] = static_cast<cuuint64_t>(dd[i].extent);
-    strides[i] = static_cast<cuuint64_t>(dd[i].stride) * 2;
-    if (dd[i].role == 0) box[i + 1] = fa::kDecodePage;
-    if (dd[i].role == 1) prm.head_coord = i + 1;
-    if (dd[i].role == 2) prm.page_coord = i + 1;
-  }
-  int st = encode_map(&prm.tm_k, k_pages, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  // whole rows (d columns) of one 64-token page per box, no swizzle
+  int st = encode_page_pool_map(&prm.tm_k, k_pages, num_pages, page_stride, token_stride, head_stride,
+                                pl.page_size, pl.num_kv_heads, pl.head_dim, pl.head_dim,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord);
   if (st != FA_OK) return st;
-  st = encode_map(&prm.tm_v, v_pages, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  st = encode_page_pool_map(&prm.tm_v, v_pages, num_pages, page_stride, token_stride, head_stride,
+                            pl.page_size, pl.num_kv_heads, pl.head_dim, pl.head_dim,
+                            CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord);
   if (st != FA_OK) return st;
 
   prm.q = static_cast<const __nv_bfloat16*>(q);

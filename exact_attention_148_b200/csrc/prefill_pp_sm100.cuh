@@ -49,13 +49,24 @@ constexpr float kRescaleThreshold = 8.0f;
 // first and the Hq/Hkv query heads that share the kv head are adjacent.  So at
 // any moment only a few heads' K/V are being read and re-reads hit L2, and the
 // block scheduler's greedy fill ends on light tiles.
+//
+// Paged form (chunked prefill): K/V come from a page pool through block_table
+// instead of being packed like Q.  Request b's cache holds cache_seqlens[b]
+// keys, its q_len queries are the last q_len of them, and a causal query i
+// sees keys up to position cache_seqlens[b] - q_len + i.
 struct PrefillParams {
   CUtensorMap tm_q;   // 3-D {d, Hq, T}, box {64, 1, 128}, 128B swizzle
-  CUtensorMap tm_k;   // 3-D {d, Hkv, T}
-  CUtensorMap tm_v;
+  CUtensorMap tm_k;   // packed: 3-D {d, Hkv, T}; paged: 4-D over the pool, box of
+  CUtensorMap tm_v;   //   64 columns x one 64-token page, 128B swizzle
   __nv_bfloat16* out;        // [T, Hq, d]
   float* lse;                // [T, Hq] or null
-  const int32_t* cu_seqlens; // [B+1]
+  const int32_t* cu_seqlens; // [B+1] query offsets
+  const int32_t* block_table;    // paged: [B, max_pages]
+  const int32_t* cache_seqlens;  // paged: [B] keys per request
+  int max_pages;
+  int num_pages;
+  int head_coord;            // paged: tensor-map dimension (1..3) of the kv head
+  int page_coord;            // paged: tensor-map dimension (1..3) of the page id
   int num_q_heads;
   int group;                 // Hq / Hkv
   int causal;
@@ -90,8 +101,8 @@ struct PrefillPPCfg {
   static constexpr int Q_OFF = 0;                          // two Q tiles
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final
-  static constexpr int NUM_BARS = 1 + 2 * NS + 7;
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final, v_tail
+  static constexpr int NUM_BARS = 1 + 2 * NS + 8;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -146,7 +157,9 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-template <int D>
+constexpr int kPrefillPage = 64;
+
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     fa_prefill_pp_kernel(const __grid_constant__ PrefillParams p) {
   using C = PrefillPPCfg<D>;
@@ -169,8 +182,19 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   const int kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
   const int rank = bid - p.group_start[lo];
   const int s0 = p.cu_seqlens[seq];
-  const int L = p.cu_seqlens[seq + 1] - s0;
+  const int L = p.cu_seqlens[seq + 1] - s0;     // queries
   const int n_qtiles = (L + C::BM - 1) / C::BM;
+  int Lk = L;                                   // keys
+  if constexpr (PAGED) {
+    Lk = p.cache_seqlens[seq];
+    const int cap = p.max_pages * kPrefillPage;
+    if (Lk < L || Lk > cap) {
+      if (rank == 0 && threadIdx.x == 0) record_status(FA_ERR_PLAN_MISMATCH);
+      Lk = min(max(Lk, L), cap);
+    }
+  }
+  const int off = p.causal ? Lk - L : 0;        // query i sits at key position i + off
+  const int n_ktiles = (Lk + C::BN - 1) / C::BN;
   const int G = p.group;
   int qtile[2], head[2];
   if ((G & 1) == 0) {            // two heads of the group, same rows
@@ -191,7 +215,9 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const bool active = qtile[k] >= 0 && qtile[k] < n_qtiles;
-    n_kv[k] = !active ? 0 : (p.causal ? qtile[k] + 1 : n_qtiles);
+    n_kv[k] = !active ? 0
+                      : (p.causal ? min(n_ktiles, (qtile[k] * C::BM + C::BM - 1 + off) / C::BN + 1)
+                                  : n_ktiles);
   }
   if (n_kv[0] == 0 && n_kv[1] == 0) return;   // uniform; nothing allocated yet
   const int n_max = max(n_kv[0], n_kv[1]);
@@ -206,6 +232,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   auto bar_p_full = [&](int k) { return bars + 8 * (3 + 2 * C::NS + k); };
   auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * C::NS + k); };
   const uint32_t bar_final = bars + 8 * (7 + 2 * C::NS);
+  const uint32_t bar_vtail = bars + 8 * (8 + 2 * C::NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -221,6 +248,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       mbar_init(bar_o_done(k), 1);
     }
     mbar_init(bar_final, 1);
+    mbar_init(bar_vtail, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -233,7 +261,109 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-  if (warp == 8) {
+  if (PAGED && warp == 8) {
+    // ------------------------------------------------- TMA producer, paged K/V
+    // Key tile jt is logical pages 2jt and 2jt+1; their physical ids are read
+    // 32 at a time by the whole warp.  A page past the cache end (or an id
+    // outside the pool, which is also recorded) is loaded from page index
+    // num_pages, i.e. out of the tensor map's bounds, which TMA fills with
+    // zeros without touching memory.  The cache's last page may end inside
+    // the page: its slots past the end hold whatever the pool had, so the V
+    // tile holding it lands on its own barrier, the warp zeroes those rows
+    // (0 * NaN would otherwise reach O through P V), and only then marks the
+    // tile full.  That tile is always the last one loaded.
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      const int nq = (n_kv[0] > 0) + (n_kv[1] > 0);
+      mbar_arrive_expect_tx(bar_q, nq * C::TILE_BYTES);
+      auto load_q = [&](int k, int h, int t) {
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_3d(q_s + k * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tm_q, bar_q, c * 64, h,
+                      s0 + t * C::BM);
+      };
+      if (n_kv[0] > 0) load_q(0, head[0], qtile[0]);
+      if (n_kv[1] > 0) load_q(1, head[1], qtile[1]);
+    }
+    const int32_t* bt_row = p.block_table + static_cast<size_t>(seq) * p.max_pages;
+    const int tail_tile = (Lk % kPrefillPage != 0) ? (Lk - 1) / C::BN : -1;
+    int pg_base = -1, pg_mine = 0, issued = 0, tail_item = -1;
+    bool ok = true;
+    for (int item = 0; item < 2 * n_max; ++item) {
+      const int jt = item >> 1;
+      const int lp0 = 2 * jt;
+      if ((lp0 & ~31) != pg_base) {
+        pg_base = lp0 & ~31;
+        const int lp = pg_base + lane;
+        int id = p.num_pages;
+        if (lp * kPrefillPage < Lk) {
+          id = bt_row[lp];
+          if (id < 0 || id >= p.num_pages) {
+            record_status(FA_ERR_BAD_PAGE);
+            id = p.num_pages;
+          }
+        }
+        pg_mine = id;
+      }
+      const int ph0 = __shfl_sync(0xffffffffu, pg_mine, lp0 & 31);
+      const int ph1 = __shfl_sync(0xffffffffu, pg_mine, (lp0 + 1) & 31);
+      if (lane == 0) {
+        if (mbar_wait(bar_kv_empty(item), ((item / C::NS) & 1) ^ 1, abort_flag)) {
+          const bool vtail = (item & 1) && jt == tail_tile;
+          const uint32_t bar = vtail ? bar_vtail : bar_kv_full(item);
+          mbar_arrive_expect_tx(bar, C::TILE_BYTES);
+          const CUtensorMap* map = (item & 1) ? &p.tm_v : &p.tm_k;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int phys = h ? ph1 : ph0;
+            const int c1 = (p.head_coord == 1) ? kv_head : (p.page_coord == 1 ? phys : 0);
+            const int c2 = (p.head_coord == 2) ? kv_head : (p.page_coord == 2 ? phys : 0);
+            const int c3 = (p.head_coord == 3) ? kv_head : (p.page_coord == 3 ? phys : 0);
+#pragma unroll
+            for (int c = 0; c < C::CHUNKS; ++c)
+              tma_load_4d(kv_s(item) + c * C::CHUNK_BYTES + h * (C::CHUNK_BYTES / 2), map, bar,
+                          c * 64, c1, c2, c3);
+          }
+          ++issued;
+          if (vtail) tail_item = item;
+        } else {
+          ok = false;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    }
+    tail_item = __shfl_sync(0xffffffffu, tail_item, 0);
+    bool tail_landed = true;
+    if (tail_item >= 0) {
+      tail_landed = __all_sync(0xffffffffu, mbar_wait(bar_vtail, 0, abort_flag));
+      if (tail_landed) {
+        // rows [Lk, end of its page) of the tile, in every 64-column chunk
+        const int r0 = Lk - (tail_item >> 1) * C::BN;
+        const int r1 = ((Lk + kPrefillPage - 1) / kPrefillPage) * kPrefillPage - (tail_item >> 1) * C::BN;
+        uint4* tile = reinterpret_cast<uint4*>(smem + C::KV_OFF + (tail_item % C::NS) * C::TILE_BYTES);
+        const int per_chunk = (r1 - r0) * 8;          // 16-byte stores per chunk
+        for (int e = lane; e < C::CHUNKS * per_chunk; e += 32) {
+          const int c = e / per_chunk, w = e % per_chunk;
+          tile[(c * C::CHUNK_BYTES + r0 * 128) / 16 + w] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_kv_full(tail_item));
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int never = 0;
+      for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i) {
+        if (i == tail_item) {
+          if (!tail_landed) mbar_wait(bar_vtail, 0, &never);
+        } else {
+          mbar_wait(bar_kv_full(i), (i / C::NS) & 1, &never);
+        }
+      }
+    }
+  } else if (warp == 8) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -353,6 +483,10 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     const int my_head = k ? head[1] : head[0];
     const int q_row = my_qtile * C::BM + r;
     const int nk = k ? n_kv[1] : n_kv[0];
+    // Last visible key of this row, and the smallest such bound in the tile:
+    // key tiles reaching past the latter need the mask.
+    const int row_last = p.causal ? min(q_row + off, Lk - 1) : Lk - 1;
+    const int tile_last = p.causal ? min(my_qtile * C::BM + off, Lk - 1) : Lk - 1;
     float m_ref = 0.0f, l_sum = 0.0f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
@@ -366,9 +500,9 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       reg_dep(s[2]);
       reg_dep(s[3]);
 
-      const bool masked = p.causal ? (j == my_qtile) : ((j + 1) * C::BN > L);
+      const bool masked = j * C::BN + C::BN - 1 > tile_last;
       if (masked) {
-        const int lim = p.causal ? (q_row - j * C::BN) : (L - 1 - j * C::BN);
+        const int lim = row_last - j * C::BN;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll

@@ -93,6 +93,66 @@ int fa_prefill(const void* q, const void* k, const void* v,
                void* out, float* lse, void* stream);
 
 /*
+ * fa_append_kv — write new K/V rows into a paged KV cache (the cache that
+ * prefill fills for later steps: niuteng5618.github.io "Flash Attention &
+ * Paged Attention", section "FA对Prefill阶段的影响"; fixed-size pages behind a
+ * logical-to-physical page table: same page, section 2).
+ *
+ *   k_new, v_new [total_new, Hkv, d] bf16, packed by cu_seqlens_new_dev
+ *       ([batch+1] int32 device; cu_seqlens_new_dev[batch] == total_new).
+ *   k_pages, v_pages, num_pages, page/token/head strides: the page pool, as
+ *       for fa_decode_paged (written here).
+ *   block_table [batch, max_pages_per_seq] int32 device.
+ *   cache_seqlens_dev [batch] int32: each request's length AFTER the append.
+ *       Request b's n_b new rows take logical positions
+ *       cache_seqlens[b] - n_b ... cache_seqlens[b] - 1, i.e. token t goes to
+ *       page block_table[b][t / page_size], slot t % page_size.
+ *   page_size: 64.
+ * Only the slots of the new rows are written.  A row whose request has
+ * n_b > cache_seqlens[b], or a length past max_pages_per_seq * page_size, is
+ * skipped and FA_ERR_PLAN_MISMATCH recorded in the device status word; a page
+ * id outside [0, num_pages) is skipped and FA_ERR_BAD_PAGE recorded.
+ * total_new == 0 enqueues nothing.
+ */
+int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_seqlens_new_dev,
+                 int total_new, int batch, int num_kv_heads, int head_dim, void* k_pages,
+                 void* v_pages, int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                 int64_t head_stride, int page_size, const int32_t* block_table,
+                 int max_pages_per_seq, const int32_t* cache_seqlens_dev, void* stream);
+
+/*
+ * fa_prefill_paged — chunked prefill: each request's new queries attend to its
+ * whole paged KV cache (the cached prefix plus the chunk's own K/V, already
+ * written with fa_append_kv).  Same tiled tcgen05 kernel as fa_prefill, with
+ * K/V tiles fetched page by page through block_table.
+ *
+ *   q [Tq, Hq, d] bf16 packed by cu_seqlens_q_dev / cu_seqlens_q_host
+ *       ([batch+1] int32; q_len_b = cu[b+1] - cu[b] >= 1).
+ *   k_pages, v_pages, num_pages, strides, block_table, max_pages_per_seq:
+ *       the page pool and table, as for fa_decode_paged.
+ *   cache_seqlens_dev / cache_seqlens_host [batch] int32: keys per request,
+ *       k_len_b >= q_len_b, k_len_b <= max_pages_per_seq * page_size.
+ *   causal != 0: the chunk's queries are the last q_len_b positions of the
+ *       request's sequence, so query i sees keys 0 .. k_len_b - q_len_b + i
+ *       (with k_len_b == q_len_b this is fa_prefill's causal mask).
+ *       causal == 0: every query sees all k_len_b keys.
+ *   page_size: 64.  scale: NaN means 1/sqrt(d).
+ *   out [Tq, Hq, d] bf16; lse [Tq, Hq] fp32 or NULL.
+ * Cache slots past k_len_b in a request's last page may hold anything (NaN
+ * included): they are never used.  A block_table entry outside the pool reads
+ * as zeros and records FA_ERR_BAD_PAGE; device lengths that disagree with the
+ * host copies record FA_ERR_PLAN_MISMATCH.  The host and device copies of
+ * cu_seqlens_q and cache_seqlens must hold the same values.
+ */
+int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
+                     const int32_t* cu_seqlens_q_host, const void* k_pages, const void* v_pages,
+                     int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                     int64_t head_stride, const int32_t* block_table, int max_pages_per_seq,
+                     const int32_t* cache_seqlens_dev, const int32_t* cache_seqlens_host,
+                     int batch, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
+                     int causal, float scale, void* out, float* lse, void* stream);
+
+/*
  * fa_decode_plan — host-only split and load-balance planning for paged
  * decode (the "plan" stage: wsisp.com "FIA / FlashAttention", section 二;
  * Flash-Decoding's split along the context: niuteng5618.github.io, section

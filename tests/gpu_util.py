@@ -76,3 +76,33 @@ def decode_device_inputs(inp: W.DecodeInputs):
     return dict(q=to_dev_bf16(inp.q_bits), k=to_dev_bf16(inp.k_pages_bits),
                 v=to_dev_bf16(inp.v_pages_bits), bt=to_dev_i32(inp.block_table),
                 lens=to_dev_i32(inp.cache_seqlens))
+
+
+def chunked_device_inputs(inp: W.ChunkedPrefillInputs):
+    return dict(q=to_dev_bf16(inp.q_bits), k_new=to_dev_bf16(inp.k_new_bits),
+                v_new=to_dev_bf16(inp.v_new_bits), cu=to_dev_i32(inp.cu_seqlens_q),
+                k=to_dev_bf16(inp.k_pages_bits), v=to_dev_bf16(inp.v_pages_bits),
+                bt=to_dev_i32(inp.block_table), lens=to_dev_i32(inp.cache_seqlens))
+
+
+def chunked_on_gpu(inp: W.ChunkedPrefillInputs, dev=None, append=True, **kw):
+    """KV append (optional) then chunked prefill over the paged cache."""
+    import exact_attention_148_b200 as fa
+    if dev is None:
+        dev = chunked_device_inputs(inp)
+    if append:
+        fa.append_kv(dev["k_new"], dev["v_new"], dev["cu"], dev["k"], dev["v"], dev["bt"],
+                     dev["lens"], layout=inp.layout)
+    out, lse = fa.prefill_paged(dev["q"], dev["cu"], dev["k"], dev["v"], dev["bt"], dev["lens"],
+                                causal=inp.causal, scale=inp.scale, layout=inp.layout,
+                                cu_seqlens_q_host=inp.cu_seqlens_q,
+                                cache_seqlens_host=inp.cache_seqlens, **kw)
+    return out, lse, dev
+
+
+def oracle_pool_after_append(inp: W.ChunkedPrefillInputs):
+    """Page pool bits after the oracle's append (bit patterns, no arithmetic)."""
+    import oracle
+    return oracle.append_kv_ref(inp.k_pages_bits, inp.v_pages_bits, inp.k_new_bits, inp.v_new_bits,
+                                inp.cu_seqlens_q, inp.block_table, inp.cache_seqlens,
+                                inp.page_size, inp.layout)

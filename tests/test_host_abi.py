@@ -208,3 +208,48 @@ def test_python_binding_refuses_cpu_tensors(lib):
     cu = torch.tensor([0, 128], dtype=torch.int32)
     with pytest.raises(ValueError, match="CUDA"):
         fa.prefill(q, q, q, cu)
+
+
+def test_prefill_paged_validation_before_any_cuda_call(lib):
+    cu = np.array([0, 100, 300], dtype=np.int32)
+    lens = np.array([150, 200], dtype=np.int32)
+    A = 0x10000
+    strides = (64 * 2 * 128, 2 * 128, 128)
+
+    def call(q=A, cu=cu, lens=lens, hq=4, hkv=2, d=128, ps=64, max_pages=4, npages=10,
+             strides=strides, scale=float("nan"), bt=A):
+        return lib.fa_prefill_paged(
+            _fake(q), _fake(A), cu.ctypes.data_as(ctypes.c_void_p), _fake(A), _fake(A), npages,
+            *strides, _fake(bt), max_pages, _fake(A), lens.ctypes.data_as(ctypes.c_void_p),
+            len(cu) - 1, hq, hkv, d, ps, 1, scale, _fake(A), None, None)
+    assert call(q=0) == fa.FA_ERR_INVALID_ARG
+    assert call(bt=0) == fa.FA_ERR_INVALID_ARG
+    assert call(q=A + 2) == fa.FA_ERR_INVALID_ARG
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(ps=16) == fa.FA_ERR_UNSUPPORTED
+    assert call(hq=6, hkv=4) == fa.FA_ERR_INVALID_ARG
+    assert call(npages=0) == fa.FA_ERR_INVALID_ARG
+    assert call(strides=(64 * 2 * 128, 2 * 128, 100)) == fa.FA_ERR_INVALID_ARG
+    assert call(scale=-2.0) == fa.FA_ERR_INVALID_ARG
+    # cache shorter than the chunk, and a cache past the table's capacity
+    assert call(lens=np.array([99, 200], dtype=np.int32)) == fa.FA_ERR_INVALID_ARG
+    assert call(max_pages=3) == fa.FA_ERR_INVALID_ARG               # 200 > 3 * 64
+    assert call(cu=np.array([0, 0, 300], dtype=np.int32)) == fa.FA_ERR_INVALID_ARG
+
+
+def test_append_validation_before_any_cuda_call(lib):
+    A = 0x10000
+    strides = (64 * 2 * 128, 2 * 128, 128)
+
+    def call(k=A, total=10, d=128, ps=64, npages=10, strides=strides, bt=A, kp=A):
+        return lib.fa_append_kv(_fake(k), _fake(A), _fake(A), total, 2, 2, d, _fake(kp), _fake(A),
+                                npages, *strides, ps, _fake(bt), 4, _fake(A), None)
+    assert call(k=0) == fa.FA_ERR_INVALID_ARG
+    assert call(kp=0) == fa.FA_ERR_INVALID_ARG
+    assert call(k=A + 8) == fa.FA_ERR_INVALID_ARG
+    assert call(total=-1) == fa.FA_ERR_INVALID_ARG
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(ps=32) == fa.FA_ERR_UNSUPPORTED
+    assert call(npages=0) == fa.FA_ERR_INVALID_ARG
+    assert call(strides=(64 * 2 * 128, 2 * 128, 12)) == fa.FA_ERR_INVALID_ARG
+    assert call(total=0) == fa.FA_OK                                 # nothing to enqueue
