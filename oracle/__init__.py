@@ -25,3 +25,4 @@ from .attention import (  # noqa: F401
     partial_state_ref,
     visible_key_count,
 )
+from .fp8 import dequantize_e4m3, e4m3_to_f64  # noqa: F401

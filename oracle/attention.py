@@ -212,13 +212,18 @@ def gather_paged_kv(k_pages, v_pages, block_table_row, seqlen: int, kv_head: int
 
 def paged_decode_rows_ref(q, k_pages, v_pages, block_table, cache_seqlens, scale,
                           rows, page_size: int = 64, layout: str = "NHD",
-                          to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+                          to_f64=lambda a: np.asarray(a, dtype=np.float64),
+                          k_to_f64=None, v_to_f64=None):
     """Decode output for selected (request, q_head) rows.
 
-    ``to_f64`` widens gathered cache slices (e.g. bf16 bit patterns); by default
-    the cache is taken to already hold float values.
+    ``to_f64`` widens the query and gathered cache slices (e.g. bf16 bit
+    patterns); ``k_to_f64`` / ``v_to_f64``, when given, replace it for the K
+    and V slices (e.g. dequantising an FP8 cache).  By default everything is
+    taken to already hold float values.
     Returns (O [n, d], LSE [n]).
     """
+    k_conv = k_to_f64 if k_to_f64 is not None else to_f64
+    v_conv = v_to_f64 if v_to_f64 is not None else to_f64
     B, Hq, d = q.shape
     Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
     if scale is None:
@@ -232,7 +237,7 @@ def paged_decode_rows_ref(q, k_pages, v_pages, block_table, cache_seqlens, scale
         if key not in cache:
             K, V = gather_paged_kv(k_pages, v_pages, block_table[b], int(cache_seqlens[b]), g,
                                    page_size, layout)
-            cache = {key: (to_f64(K), to_f64(V))}
+            cache = {key: (k_conv(K), v_conv(V))}
         K, V = cache[key]
         qi = to_f64(q[b, h])[None, :]
         P, l = _softmax_with_lse(_scores(qi, K, scale))
@@ -243,7 +248,8 @@ def paged_decode_rows_ref(q, k_pages, v_pages, block_table, cache_seqlens, scale
 
 def paged_decode_ref(q, k_pages, v_pages, block_table, cache_seqlens, scale=None,
                      page_size: int = 64, layout: str = "NHD",
-                     to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+                     to_f64=lambda a: np.asarray(a, dtype=np.float64),
+                     k_to_f64=None, v_to_f64=None):
     """One query row per request against its whole paged KV cache.
 
     q: [B, Hq, d]. Returns (O [B, Hq, d], LSE [B, Hq]).
@@ -251,7 +257,7 @@ def paged_decode_ref(q, k_pages, v_pages, block_table, cache_seqlens, scale=None
     B, Hq, d = q.shape
     rows = [(b, h) for b in range(B) for h in range(Hq)]
     o, l = paged_decode_rows_ref(q, k_pages, v_pages, block_table, cache_seqlens, scale, rows,
-                                 page_size, layout, to_f64)
+                                 page_size, layout, to_f64, k_to_f64, v_to_f64)
     return o.reshape(B, Hq, d), l.reshape(B, Hq)
 
 

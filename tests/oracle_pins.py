@@ -410,3 +410,33 @@ def pin_chunk_single_query_is_decode(paged_prefill_ref, paged_decode_ref, seed=1
     od, ld = paged_decode_ref(q, kp, vp, bt, lens, 0.8, page_size=ps, layout="HND")
     _close(o, od, 1e-13, "single-query chunk vs decode O")
     _close(l, ld, 1e-13, "single-query chunk vs decode LSE")
+
+
+# --- FP8 (E4M3) KV cache ------------------------------------------------------
+
+def pin_e4m3_codes(e4m3_to_f64):
+    """Hand-decoded codes, then all 256 codes against PyTorch's float8_e4m3fn."""
+    import torch
+    g = load_golden("fp8_decode.json")
+    for code, val in g["codes"].items():
+        got = float(e4m3_to_f64(np.array([int(code, 16)], dtype=np.uint8))[0])
+        assert got == val and math.copysign(1.0, got) == math.copysign(1.0, val), \
+            f"E4M3 {code}: {got} != {val}"
+    allb = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(allb).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = e4m3_to_f64(allb)
+    assert np.array_equal(np.isnan(got), np.isnan(ref)), "E4M3 NaN codes"
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok]), "E4M3 values vs torch float8_e4m3fn"
+
+
+def pin_golden_fp8_decode(paged_decode_ref, dequantize_e4m3):
+    g = load_golden("fp8_decode.json")
+    kp = np.array(g["k_pages"], dtype=np.uint8)
+    vp = np.array(g["v_pages"], dtype=np.uint8)
+    o, l = paged_decode_ref(np.array(g["q"]), kp, vp, np.array(g["block_table"]),
+                            np.array(g["cache_seqlens"]), g["scale"], page_size=g["page_size"],
+                            k_to_f64=lambda a: dequantize_e4m3(a, g["k_scale"]),
+                            v_to_f64=lambda a: dequantize_e4m3(a, g["v_scale"]))
+    _close(o, g["o"], 1e-13, "fp8 decode O")
+    _close(l, g["lse"], 1e-13, "fp8 decode LSE")

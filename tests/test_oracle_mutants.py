@@ -185,3 +185,37 @@ def test_append_mutant_is_caught(bad):
         except (AssertionError, IndexError):
             return
     raise AssertionError("append mutant not caught")
+
+
+E4M3_MUTANTS = {
+    # exponent bias 8 instead of 7
+    "bias8": lambda b: np.where(((np.asarray(b, np.int64) >> 3) & 15) == 0,
+                                np.ldexp((np.asarray(b, np.int64) & 7) / 8.0, -6),
+                                np.ldexp(1.0 + (np.asarray(b, np.int64) & 7) / 8.0,
+                                         ((np.asarray(b, np.int64) >> 3) & 15) - 8))
+    * np.where(np.asarray(b, np.int64) >> 7, -1.0, 1.0),
+    # subnormals decoded with an implicit leading one
+    "no_subnormal": lambda b: np.ldexp(1.0 + (np.asarray(b, np.int64) & 7) / 8.0,
+                                       ((np.asarray(b, np.int64) >> 3) & 15) - 7)
+    * np.where(np.asarray(b, np.int64) >> 7, -1.0, 1.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(E4M3_MUTANTS))
+def test_e4m3_mutant_is_caught(name):
+    with np.errstate(all="ignore"):
+        try:
+            P.pin_e4m3_codes(E4M3_MUTANTS[name])
+        except AssertionError:
+            return
+    raise AssertionError(f"E4M3 mutant {name} not caught")
+
+
+def test_fp8_scales_swapped_is_caught():
+    from oracle import fp8
+    swapped = lambda bits, scale: fp8.dequantize_e4m3(bits, 0.5 if scale != 0.5 else math.log(3.0))
+    try:
+        P.pin_golden_fp8_decode(A.paged_decode_ref, swapped)
+    except AssertionError:
+        return
+    raise AssertionError("swapped K/V scales not caught")

@@ -177,3 +177,11 @@ def test_visible_key_count_reduces_to_square_causal():
         for i in range(L):
             assert oracle.visible_key_count(i, L, L, True) == i + 1
             assert oracle.visible_key_count(i, L, L, False) == L
+
+
+def test_e4m3_codes():
+    P.pin_e4m3_codes(oracle.e4m3_to_f64)
+
+
+def test_golden_fp8_decode():
+    P.pin_golden_fp8_decode(oracle.paged_decode_ref, oracle.dequantize_e4m3)

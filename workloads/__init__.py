@@ -212,9 +212,15 @@ class DecodeInputs:
             return a * b * d, b * d, d
         return a * b * d, d, b * d
 
+    @property
+    def kv_elem_bytes(self):
+        """2 for a bf16 cache, 1 for an FP8 (E4M3) cache."""
+        return self.k_pages_bits.dtype.itemsize
+
     def kv_bytes(self) -> float:
         """Bytes of K and V the decode must read: every cached token once."""
-        return 2.0 * float(self.cache_seqlens.astype(np.int64).sum()) * self.num_kv_heads * self.head_dim * 2
+        return (2.0 * float(self.cache_seqlens.astype(np.int64).sum()) * self.num_kv_heads *
+                self.head_dim * self.kv_elem_bytes)
 
     def algorithmic_bytes(self) -> float:
         """KV read once + q read + out/lse written + block_table entries used."""
@@ -289,6 +295,35 @@ def ragged_split_decode() -> DecodeInputs:
     return make_decode([131072] + [2048] * 63, 32, 32, 128, seed=5, name="ragged_split_decode")
 
 
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
+    """Quantise x / scale to FP8 E4M3 codes (uint8): round to nearest even,
+    saturating at +-448 (PyTorch's float8_e4m3fn cast after clipping)."""
+    import torch
+    y = np.clip(np.asarray(x, dtype=np.float32) / np.float32(scale), -E4M3_MAX, E4M3_MAX)
+    return torch.from_numpy(np.ascontiguousarray(y)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def to_fp8_cache(inp: DecodeInputs, amax: float = 4.0) -> DecodeInputs:
+    """The same cache quantised to E4M3 with one scale per tensor:
+    scale = amax / 448, so +-amax (4 standard deviations of the N(0,1) draws)
+    spans the format's range.  Scales go in ``extra['k_scale'/'v_scale']``."""
+    k_scale = v_scale = amax / E4M3_MAX
+    kp = quantize_e4m3(bf16_bits_to_f32(inp.k_pages_bits), k_scale)
+    vp = quantize_e4m3(bf16_bits_to_f32(inp.v_pages_bits), v_scale)
+    extra = dict(inp.extra, k_scale=float(k_scale), v_scale=float(v_scale))
+    return DecodeInputs(inp.name + "_fp8", inp.q_bits, kp, vp, inp.block_table, inp.cache_seqlens,
+                        inp.scale, inp.layout, inp.page_size, extra)
+
+
+def paged_decode_batch_fp8() -> DecodeInputs:
+    """paged_decode_batch (64 requests, U[1024, 32768], 32 q / 8 kv heads,
+    d=128) with its KV cache in FP8 E4M3, per-tensor scales."""
+    return to_fp8_cache(paged_decode_batch())
+
+
 def relayout(inp: DecodeInputs, layout: str) -> DecodeInputs:
     """Same cache contents in the other page layout (NHD <-> HND)."""
     if layout == inp.layout:
@@ -315,6 +350,7 @@ def permute_pages(inp: DecodeInputs, seed: int) -> DecodeInputs:
 
 
 BF16_NAN_BITS = 0x7FC0
+E4M3_NAN_BITS = 0x7F
 
 
 def poison_unused(inp: DecodeInputs) -> DecodeInputs:
@@ -331,12 +367,13 @@ def poison_unused(inp: DecodeInputs) -> DecodeInputs:
             n = min(ps, L - p * ps)
             valid[phys, :n] = True
     inv = ~valid
+    nan = E4M3_NAN_BITS if kp.dtype == np.uint8 else BF16_NAN_BITS
     if inp.layout == "NHD":
-        kp[inv] = BF16_NAN_BITS
-        vp[inv] = BF16_NAN_BITS
+        kp[inv] = nan
+        vp[inv] = nan
     else:
-        kp.transpose(0, 2, 1, 3)[inv] = BF16_NAN_BITS
-        vp.transpose(0, 2, 1, 3)[inv] = BF16_NAN_BITS
+        kp.transpose(0, 2, 1, 3)[inv] = nan
+        vp.transpose(0, 2, 1, 3)[inv] = nan
     return DecodeInputs(inp.name + "_poison", inp.q_bits, kp, vp, inp.block_table,
                         inp.cache_seqlens, inp.scale, inp.layout, inp.page_size, dict(inp.extra))
 
@@ -518,6 +555,7 @@ CONFIGS = {
     "paged_decode_batch16": paged_decode_batch16,
     "long_split_decode": long_split_decode,
     "ragged_split_decode": ragged_split_decode,
+    "paged_decode_batch_fp8": paged_decode_batch_fp8,
     "tiny_chunked_prefill": tiny_chunked_prefill,
     "chunked_prefill_batch": chunked_prefill_batch,
 }
