@@ -71,7 +71,12 @@ def _scores(q_rows: np.ndarray, keys: np.ndarray, scale: float) -> np.ndarray:
 
 
 def _softmax_with_lse(s: np.ndarray):
-    """Row softmax of a (possibly -inf masked) score block, plus its LSE."""
+    """Row softmax of a (possibly -inf masked) score block, plus its LSE.
+
+    Rows with no allowed key (all -inf, or no columns at all) get zero
+    weights and LSE = -inf."""
+    if s.shape[-1] == 0:
+        return np.zeros(s.shape), np.full(s.shape[:-1], NEG_INF)
     m = np.max(s, axis=-1, keepdims=True)
     finite = np.isfinite(m)
     m_safe = np.where(finite, m, 0.0)

@@ -185,3 +185,20 @@ def test_e4m3_codes():
 
 def test_golden_fp8_decode():
     P.pin_golden_fp8_decode(oracle.paged_decode_ref, oracle.dequantize_e4m3)
+
+
+def test_empty_cache_decodes_to_zero():
+    """A request with no cached token: O = 0 and LSE = -inf (the empty-key
+    reading), next to a normal request that must be unaffected."""
+    g = np.random.default_rng(151)
+    kp = g.standard_normal((3, 4, 1, 2))
+    vp = g.standard_normal((3, 4, 1, 2))
+    bt = np.array([[0, 1], [-1, -1]])
+    q = g.standard_normal((2, 1, 2))
+    o, l = oracle.paged_decode_ref(q, kp, vp, bt, [5, 0], 0.5, page_size=4)
+    assert np.array_equal(o[1], np.zeros((1, 2))) and np.isneginf(l[1, 0])
+    K = np.concatenate([kp[0, :, 0], kp[1, :1, 0]])
+    V = np.concatenate([vp[0, :, 0], vp[1, :1, 0]])
+    ob, lb = oracle.partial_state_ref(q[0], K, V, 0.5)
+    np.testing.assert_allclose(o[0], ob, atol=1e-14)
+    np.testing.assert_allclose(l[0], lb, atol=1e-14)
