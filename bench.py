@@ -9,7 +9,9 @@ One step = one pass of the whole hot path over one batch of synthetic input:
      plan and fa_decode_paged (split kernel + merge kernel).
 The line's ``value`` is the prefill throughput in TFLOP/s (causal algorithmic
 FLOPs); the decode half reports HBM GB/s under ``decode``.  ``--workload``
-selects a single configuration instead (one line for that configuration).
+selects a single configuration instead (one line for that configuration);
+``chunked_prefill_batch`` times a chunked-prefill step (fa_append_kv of the
+chunk's K/V into the paged cache, then fa_prefill_paged over the whole cache).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 launch under torch.distributed.run; every rank runs an independent
@@ -41,7 +43,8 @@ SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill"}
 DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode",
-                    "paged_decode_batch16"}
+                    "paged_decode_batch16", "paged_decode_batch_fp8"}
+CHUNKED_WORKLOADS = {"chunked_prefill_batch", "tiny_chunked_prefill"}
 
 
 def load_peaks():
@@ -171,9 +174,14 @@ class DecodeCase:
         import torch
         import exact_attention_148_b200 as fa
         self.inp = inp
+        self.fp8 = inp.kv_elem_bytes == 1
         self.q = _dev_bf16(inp.q_bits, device)
-        self.kp = _dev_bf16(inp.k_pages_bits, device)
-        self.vp = _dev_bf16(inp.v_pages_bits, device)
+        if self.fp8:
+            self.kp = torch.from_numpy(inp.k_pages_bits).to(device)
+            self.vp = torch.from_numpy(inp.v_pages_bits).to(device)
+        else:
+            self.kp = _dev_bf16(inp.k_pages_bits, device)
+            self.vp = _dev_bf16(inp.v_pages_bits, device)
         self.bt = _dev_i32(inp.block_table, device)
         self.lens = _dev_i32(inp.cache_seqlens, device)
         t0 = time.perf_counter()
@@ -188,8 +196,9 @@ class DecodeCase:
         self.bytes = inp.algorithmic_bytes()
         self.launches = 1 + (1 if self.plan.info.max_splits > 1 else 0)
         self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
-        self.h_k = torch.from_numpy(inp.k_pages_bits.view(np.int16)).pin_memory()
-        self.h_v = torch.from_numpy(inp.v_pages_bits.view(np.int16)).pin_memory()
+        kv_view = np.uint8 if self.fp8 else np.int16
+        self.h_k = torch.from_numpy(inp.k_pages_bits.view(kv_view)).pin_memory()
+        self.h_v = torch.from_numpy(inp.v_pages_bits.view(kv_view)).pin_memory()
         self.h_bt = torch.from_numpy(inp.block_table).pin_memory()
         self.h_lens = torch.from_numpy(inp.cache_seqlens).pin_memory()
         self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
@@ -197,14 +206,20 @@ class DecodeCase:
 
     def run(self):
         import exact_attention_148_b200 as fa
+        if self.fp8:
+            fa.decode_paged_fp8(self.q, self.kp, self.vp, self.bt, self.lens, self.plan,
+                                k_scale=self.inp.extra["k_scale"], v_scale=self.inp.extra["v_scale"],
+                                layout=self.inp.layout, scale=self.inp.scale, out=self.out,
+                                lse=self.lse, workspace=self.ws)
+            return
         fa.decode_paged(self.q, self.kp, self.vp, self.bt, self.lens, self.plan, layout=self.inp.layout,
                         scale=self.inp.scale, out=self.out, lse=self.lse, workspace=self.ws)
 
     def run_e2e(self):
         import torch
         self.q.view(torch.int16).copy_(self.h_q, non_blocking=True)
-        self.kp.view(torch.int16).copy_(self.h_k, non_blocking=True)
-        self.vp.view(torch.int16).copy_(self.h_v, non_blocking=True)
+        self.kp.view(self.h_k.dtype).copy_(self.h_k, non_blocking=True)
+        self.vp.view(self.h_v.dtype).copy_(self.h_v, non_blocking=True)
         self.bt.copy_(self.h_bt, non_blocking=True)
         self.lens.copy_(self.h_lens, non_blocking=True)
         self.run()
@@ -213,7 +228,7 @@ class DecodeCase:
 
     def h2d_bytes(self):
         i = self.inp
-        return 2 * (i.q_bits.size + i.k_pages_bits.size + i.v_pages_bits.size) + \
+        return 2 * i.q_bits.size + i.k_pages_bits.nbytes + i.v_pages_bits.nbytes + \
             4 * (i.block_table.size + i.cache_seqlens.size)
 
     def d2h_bytes(self):
@@ -224,9 +239,116 @@ class DecodeCase:
         info = self.plan.info
         return {"workload": i.name, "batch": i.batch, "cache_tokens_total": int(i.cache_seqlens.sum()),
                 "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads, "head_dim": i.head_dim,
-                "page_size": i.page_size, "layout": i.layout, "chunk_tokens": info.chunk_tokens,
+                "page_size": i.page_size, "layout": i.layout,
+                "kv_dtype": "e4m3 (per-tensor scales)" if self.fp8 else "bf16",
+                "chunk_tokens": info.chunk_tokens,
                 "max_splits": info.max_splits, "work_items": info.num_work_items,
                 "plan_ms": round(self.plan_ms, 3), "algorithmic_gb": round(self.bytes / 1e9, 4)}
+
+
+class ChunkedState:
+    """Device buffers of one chunked-prefill step: the chunk's q / k / v, the
+    paged cache (prefix resident across steps) and the outputs."""
+
+    def __init__(self, inp: W.ChunkedPrefillInputs, device):
+        import torch
+        self.inp = inp
+        self.q = _dev_bf16(inp.q_bits, device)
+        self.k_new = _dev_bf16(inp.k_new_bits, device)
+        self.v_new = _dev_bf16(inp.v_new_bits, device)
+        self.cu = _dev_i32(inp.cu_seqlens_q, device)
+        self.kp = _dev_bf16(inp.k_pages_bits, device)
+        self.vp = _dev_bf16(inp.v_pages_bits, device)
+        self.bt = _dev_i32(inp.block_table, device)
+        self.lens = _dev_i32(inp.cache_seqlens, device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=device)
+        self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
+        self.h_k = torch.from_numpy(inp.k_new_bits.view(np.int16)).pin_memory()
+        self.h_v = torch.from_numpy(inp.v_new_bits.view(np.int16)).pin_memory()
+        self.h_cu = torch.from_numpy(inp.cu_seqlens_q).pin_memory()
+        self.h_lens = torch.from_numpy(inp.cache_seqlens).pin_memory()
+        self.h_bt = torch.from_numpy(inp.block_table).pin_memory()
+        self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+
+class AppendCase:
+    """fa_append_kv of the chunk's K/V rows into the paged cache."""
+
+    def __init__(self, st: ChunkedState):
+        self.st = st
+        self.inp = st.inp
+        self.bytes = st.inp.append_bytes()
+        self.launches = 1
+
+    def run(self):
+        import exact_attention_148_b200 as fa
+        s = self.st
+        fa.append_kv(s.k_new, s.v_new, s.cu, s.kp, s.vp, s.bt, s.lens, layout=s.inp.layout)
+
+    def run_e2e(self):
+        """The step's inputs (chunk q/k/v and its table rows) come from pinned
+        host memory; the cached prefix is resident state."""
+        import torch
+        s = self.st
+        s.q.view(torch.int16).copy_(s.h_q, non_blocking=True)
+        s.k_new.view(torch.int16).copy_(s.h_k, non_blocking=True)
+        s.v_new.view(torch.int16).copy_(s.h_v, non_blocking=True)
+        s.cu.copy_(s.h_cu, non_blocking=True)
+        s.lens.copy_(s.h_lens, non_blocking=True)
+        s.bt.copy_(s.h_bt, non_blocking=True)
+        self.run()
+
+    def h2d_bytes(self):
+        i = self.inp
+        return 2 * (i.q_bits.size + i.k_new_bits.size + i.v_new_bits.size) + \
+            4 * (i.cu_seqlens_q.size + i.cache_seqlens.size + i.block_table.size)
+
+    def d2h_bytes(self):
+        return 0
+
+    def describe(self):
+        return {"kernel": "fa_append_kv_kernel", "new_tokens": int(self.inp.cu_seqlens_q[-1]),
+                "algorithmic_gb": round(self.bytes / 1e9, 4)}
+
+
+class ChunkedAttnCase:
+    """fa_prefill_paged: the chunk's queries against each whole paged cache."""
+
+    def __init__(self, st: ChunkedState):
+        self.st = st
+        self.inp = st.inp
+        self.flops = st.inp.causal_flops()
+        self.launches = -(-sum(-(-int(L) // 128) for L in st.inp.chunk_lens) // 2048)
+
+    def run(self):
+        import exact_attention_148_b200 as fa
+        s = self.st
+        fa.prefill_paged(s.q, s.cu, s.kp, s.vp, s.bt, s.lens, causal=s.inp.causal, scale=s.inp.scale,
+                         layout=s.inp.layout, out=s.out, lse=s.lse,
+                         cu_seqlens_q_host=s.inp.cu_seqlens_q, cache_seqlens_host=s.inp.cache_seqlens)
+
+    def run_e2e(self):
+        import torch
+        s = self.st
+        self.run()
+        s.h_out.copy_(s.out.view(torch.int16), non_blocking=True)
+        s.h_lse.copy_(s.lse, non_blocking=True)
+
+    def h2d_bytes(self):
+        return 0
+
+    def d2h_bytes(self):
+        return 2 * self.inp.q_bits.size + 4 * self.st.lse.numel()
+
+    def describe(self):
+        i = self.inp
+        return {"workload": i.name, "batch": i.batch, "chunk_tokens_total": int(i.chunk_lens.sum()),
+                "prefix_tokens_total": int(i.prefix_lens.sum()), "num_q_heads": i.num_q_heads,
+                "num_kv_heads": i.num_kv_heads, "head_dim": i.head_dim, "page_size": i.page_size,
+                "layout": i.layout, "causal": bool(i.causal),
+                "algorithmic_tflop": round(self.flops / 1e12, 4)}
 
 
 # ----------------------------------------------------------------------------- timing
@@ -336,18 +458,52 @@ def oracle_decode_sample(inp: W.DecodeInputs, budget_s: float):
     import oracle
     flops_bytes, secs, rows = 0.0, 0.0, []
     G = inp.num_q_heads // inp.num_kv_heads
+    conv = {}
+    if inp.kv_elem_bytes == 1:
+        ks, vs = inp.extra["k_scale"], inp.extra["v_scale"]
+        conv = dict(k_to_f64=lambda a: oracle.dequantize_e4m3(a, ks),
+                    v_to_f64=lambda a: oracle.dequantize_e4m3(a, vs))
     for b in range(inp.batch):
         rws = [(b, h) for h in range(0, inp.num_q_heads, G)][:2]   # two kv heads' first q head
         t0 = time.perf_counter()
         oracle.paged_decode_rows_ref(inp.q_bits, inp.k_pages_bits, inp.v_pages_bits, inp.block_table,
                                      inp.cache_seqlens, inp.scale, rws, inp.page_size, inp.layout,
-                                     to_f64=W.as_f64)
+                                     to_f64=W.as_f64, **conv)
         secs += time.perf_counter() - t0
-        flops_bytes += len(rws) * 2.0 * int(inp.cache_seqlens[b]) * inp.head_dim * 2
+        flops_bytes += len(rws) * 2.0 * int(inp.cache_seqlens[b]) * inp.head_dim * inp.kv_elem_bytes
         rows.append(b)
         if secs >= budget_s:
             break
     return flops_bytes, secs, f"oracle paged_decode_rows_ref, 2 kv heads of requests {rows}"
+
+
+def oracle_chunked_sample(inp: W.ChunkedPrefillInputs, budget_s: float):
+    """The oracle's chunked prefill on one (request, query head) at a time,
+    shortest requests first, until about budget_s has passed."""
+    import oracle
+    kp_all, vp_all = oracle.append_kv_ref(inp.k_pages_bits, inp.v_pages_bits, inp.k_new_bits,
+                                          inp.v_new_bits, inp.cu_seqlens_q, inp.block_table,
+                                          inp.cache_seqlens, inp.page_size, inp.layout)
+    head_axis = 2 if inp.layout == "NHD" else 1
+    kp = np.take(kp_all, [0], axis=head_axis)
+    vp = np.take(vp_all, [0], axis=head_axis)
+    flops, secs, done = 0.0, 0.0, []
+    cu = inp.cu_seqlens_q
+    for b in np.argsort(inp.cache_seqlens):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        n, k = s1 - s0, int(inp.cache_seqlens[b])
+        t0 = time.perf_counter()
+        oracle.paged_prefill_ref(inp.q_bits[s0:s1, 0:1], [0, n], kp, vp, inp.block_table[b:b + 1],
+                                 inp.cache_seqlens[b:b + 1], inp.causal, inp.scale, inp.page_size,
+                                 inp.layout, to_f64=W.as_f64)
+        secs += time.perf_counter() - t0
+        pairs = n * (k - n) + n * (n + 1) // 2 if inp.causal else n * k
+        flops += 4.0 * inp.head_dim * pairs
+        done.append((k - n, n))
+        if secs >= budget_s:
+            break
+    return flops, secs, (f"oracle paged_prefill_ref on query head 0 of requests with "
+                         f"(prefix, chunk) = {done}")
 
 
 # ----------------------------------------------------------------------------- main
@@ -359,12 +515,17 @@ def build_cases(workload, device, num_splits):
         return [PrefillCase(W.CONFIGS[workload](), device)]
     if workload in DECODE_WORKLOADS:
         return [DecodeCase(W.CONFIGS[workload](), device, num_splits)]
+    if workload in CHUNKED_WORKLOADS:
+        st = ChunkedState(W.CONFIGS[workload](), device)
+        return [AppendCase(st), ChunkedAttnCase(st)]
     raise SystemExit(f"unknown workload {workload}")
 
 
 def kernel_source_hash(kind):
     import hashlib
-    files = ["ptx_sm100.cuh", "prefill_pp_sm100.cuh" if kind == "prefill" else "decode_sm100.cuh"]
+    files = {"prefill": ["ptx_sm100.cuh", "prefill_pp_sm100.cuh"],
+             "decode": ["ptx_sm100.cuh", "decode_sm100.cuh"],
+             "append": ["ptx_sm100.cuh", "append_sm100.cuh"]}[kind]
     m = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "exact_attention_148_b200", "csrc", f), "rb") as fh:
@@ -385,7 +546,7 @@ def measured_traffic(kind, workload, case=None):
     rows = {}
     for ln in lines:
         parts = [x.strip() for x in ln.strip().strip("|").split("|")]
-        if len(parts) >= 5 and parts[0] in ("prefill", "decode") and parts[3].isdigit():
+        if len(parts) >= 5 and parts[0] in ("prefill", "decode", "append") and parts[3].isdigit():
             rows[(parts[0], parts[1])] = (parts[2], int(parts[3]) + int(parts[4]))
     sha = kernel_source_hash(kind)
     if (kind, workload) in rows and rows[(kind, workload)][0] == sha:
@@ -455,14 +616,28 @@ def run_ours(args):
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
                                measured_traffic("prefill", c.inp.name))
             e["kernel"] = "fa_prefill_pp_kernel<%d>" % c.inp.head_dim
+        elif isinstance(c, ChunkedAttnCase):
+            e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
+                               measured_traffic("prefill", c.inp.name))
+            e["kernel"] = "fa_prefill_pp_kernel<%d, paged>" % c.inp.head_dim
+        elif isinstance(c, AppendCase):
+            e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
+                               measured_traffic("append", c.inp.name))
+            e["kernel"] = "fa_append_kv_kernel<%d>" % c.inp.head_dim
         else:
             e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
                                measured_traffic("decode", c.inp.name, c))
-            e["kernel"] = "fa_decode_split_kernel + fa_merge_kernel (one decode call)"
+            e["kernel"] = ("fa_decode_split_kernel<e4m3>" if c.fp8 else "fa_decode_split_kernel") + \
+                " + fa_merge_kernel (one decode call)"
         e["workload"] = c.inp.name
-        e["ms_per_launch"] = round(ms / (c.launches if isinstance(c, PrefillCase) else 1), 4)
+        e["ms_per_launch"] = round(ms / c.launches, 4)
         rooflines.append(e)
-    if isinstance(main, PrefillCase):
+    chunked = isinstance(main, AppendCase)
+    if chunked:
+        # the whole chunked step (append + attention) against the attention FLOPs
+        value = aggregate_throughput(cases[1].flops, ms_step, N, 1e12)
+        unit = "TFLOP/s"
+    elif isinstance(main, PrefillCase):
         value = aggregate_throughput(main.flops, ms_case[0], N, 1e12)
         unit = "TFLOP/s"
     else:
@@ -474,15 +649,23 @@ def run_ours(args):
                  "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
                  "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                  "data": "synthetic (seeded N(0,1) rounded to bf16; see workloads/)"})
-    cfg = {"workload": " + ".join(c.inp.name for c in cases),
+    cfg = {"workload": cases[1].inp.name + " (append + chunked prefill)" if chunked else
+           " + ".join(c.inp.name for c in cases),
            "l2": "flushed before every step (256 MiB write), outside the timed events; "
                  "inputs also exceed L2",
            "parallelism": f"replicas x{N}" if N > 1 else "single GPU"}
     for i, c in enumerate(cases):
-        cfg["prefill" if isinstance(c, PrefillCase) else "decode"] = c.describe()
+        key = {PrefillCase: "prefill", DecodeCase: "decode", AppendCase: "append",
+               ChunkedAttnCase: "chunked_prefill"}[type(c)]
+        cfg[key] = c.describe()
     line["config"] = cfg
     line["roofline"] = rl
-    if len(cases) > 1:
+    if chunked:
+        line["append"] = {"value": round(N * main.bytes / (ms_case[0] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                          "ms": round(ms_case[0], 4), "roofline": rooflines[0]}
+        line["chunked_prefill_ms"] = round(ms_case[1], 4)
+        line["chunked_prefill_tflops"] = round(N * cases[1].flops / (ms_case[1] * 1e-3) / 1e12, 2)
+    elif len(cases) > 1:
         dc = cases[1]
         line["decode"] = {"value": round(N * dc.bytes / (ms_case[1] * 1e-3) / 1e9, 1), "unit": "GB/s",
                           "ms": round(ms_case[1], 4), "roofline": rooflines[1],
@@ -490,7 +673,9 @@ def run_ours(args):
         line["prefill_ms"] = round(ms_case[0], 4)
         line["prefill_roofline"] = rooflines[0]
     if e2e_case is not None:
-        if isinstance(main, PrefillCase):
+        if chunked:
+            e2e_v = N * cases[1].flops / (sum(e2e_case) * 1e-3) / 1e12
+        elif isinstance(main, PrefillCase):
             e2e_v = N * main.flops / (e2e_case[0] * 1e-3) / 1e12
         else:
             e2e_v = N * main.bytes / (e2e_case[0] * 1e-3) / 1e9
@@ -498,12 +683,13 @@ def run_ours(args):
                        "h2d_bytes_per_step": int(sum(c.h2d_bytes() for c in cases)),
                        "d2h_bytes_per_step": int(sum(c.d2h_bytes() for c in cases)),
                        "ms_per_step": round(sum(e2e_case), 3),
-                       "path": "pinned host -> device copies, C-ABI calls, device -> pinned host copies"}
+                       "path": "pinned host -> device copies, C-ABI calls, device -> pinned host copies"
+                               + ("; the paged cache's prefix stays resident" if chunked else "")}
     line["gpu_launches"] = int(launches)
     line["clocks"] = clocks
     line["device_status"] = status
     if rank == 0 and N == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(main, args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(cases[1] if chunked else main, args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_ctx is not None:
@@ -514,6 +700,9 @@ def cpu_baseline(case, budget):
     threads = blas_threads()
     if isinstance(case, PrefillCase):
         work, secs, desc = oracle_prefill_sample(case.inp, budget)
+        val, unit = work / secs / 1e12, "TFLOP/s"
+    elif isinstance(case, ChunkedAttnCase):
+        work, secs, desc = oracle_chunked_sample(case.inp, budget)
         val, unit = work / secs / 1e12, "TFLOP/s"
     else:
         work, secs, desc = oracle_decode_sample(case.inp, budget)
@@ -532,7 +721,7 @@ def run_reference(args):
     if main == "default":
         inp = W.varlen_causal_prefill()
         is_prefill = True
-    elif main in PREFILL_WORKLOADS:
+    elif main in PREFILL_WORKLOADS or main in CHUNKED_WORKLOADS:
         inp = W.CONFIGS[main]()
         is_prefill = True
     else:
@@ -540,6 +729,8 @@ def run_reference(args):
         is_prefill = False
     per_step = max(1.0, args.cpu_budget / max(1, args.steps))
     fn = oracle_prefill_sample if is_prefill else oracle_decode_sample
+    if main in CHUNKED_WORKLOADS:
+        fn = oracle_chunked_sample
     for _ in range(args.warmup and 1):
         fn(inp, 0.0)
     work, secs = 0.0, 0.0
@@ -571,7 +762,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
-                    help="default | " + " | ".join(sorted(PREFILL_WORKLOADS | DECODE_WORKLOADS)))
+                    help="default | " + " | ".join(sorted(PREFILL_WORKLOADS | DECODE_WORKLOADS |
+                                                          CHUNKED_WORKLOADS)))
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
     "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
-    "append_kv", "prefill_paged",
+    "append_kv", "prefill_paged", "decode_paged_fp8",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -39,6 +39,7 @@ EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
+    "fa_decode_paged_fp8",
 ]
 
 # Size of the library's static decode scratch (FA_STATIC_SCRATCH_BYTES).
@@ -109,6 +110,9 @@ def library() -> ctypes.CDLL:
     L.fa_prefill_paged.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, vp, vp, i32,
                                    i32, i32, i32, i32, i32, f32, vp, vp, vp]
     L.fa_prefill_paged.restype = i32
+    L.fa_decode_paged_fp8.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, f32, f32, f32, vp,
+                                      vp, vp, ctypes.c_size_t, vp]
+    L.fa_decode_paged_fp8.restype = i32
     _lib = L
     return L
 
@@ -287,6 +291,41 @@ def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePl
         _ptr(cache_seqlens), plan.handle, _scale_arg(scale), _ptr(out), _ptr(lse), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(st, "fa_decode_paged")
+    return out, lse
+
+
+def decode_paged_fp8(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePlan, *,
+                     k_scale: float, v_scale: float, layout: str = "NHD",
+                     scale: float | None = None, out=None, lse=None, workspace=None,
+                     return_lse: bool = True, stream=None):
+    """``decode_paged`` over an FP8 E4M3 cache: k_pages / v_pages are uint8
+    (or float8_e4m3fn) tensors of E4M3 codes, dequantised as k_scale * k8 and
+    v_scale * v8.  Returns (out bf16, lse fp32)."""
+    torch = _torch()
+    _require_cuda(q, k_pages, v_pages, block_table, cache_seqlens, out, lse, workspace)
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bfloat16")
+    if k_pages.element_size() != 1 or v_pages.element_size() != 1:
+        raise ValueError("k_pages and v_pages must hold one-byte E4M3 codes")
+    if not (k_pages.is_contiguous() and v_pages.is_contiguous() and q.is_contiguous()
+            and block_table.is_contiguous()):
+        raise ValueError("tensors must be contiguous")
+    if k_pages.shape != v_pages.shape:
+        raise ValueError("k_pages and v_pages must have the same shape")
+    B, Hq, d = q.shape
+    ps, ts, hs = page_strides(k_pages, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None and plan.workspace_bytes > 0:
+        workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
+    st = library().fa_decode_paged_fp8(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(block_table),
+        _ptr(cache_seqlens), plan.handle, _scale_arg(scale), float(k_scale), float(v_scale),
+        _ptr(out), _ptr(lse), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(st, "fa_decode_paged_fp8")
     return out, lse
 
 

@@ -67,13 +67,28 @@ __global__ void __launch_bounds__(kAppendThreads) fa_append_kv_kernel(const Appe
     const int64_t dst_row = static_cast<int64_t>(phys) * p.page_stride +
                             static_cast<int64_t>(pos % kAppendPage) * p.token_stride;
     const size_t src_row = static_cast<size_t>(t) * p.num_kv_heads * VEC;
-    for (int e = lane; e < p.num_kv_heads * VEC; e += 32) {
-      const int h = e / VEC, w = e % VEC;
-      const int64_t dst = dst_row + h * p.head_stride + w * 8;   // elements
-      const uint4 kv = p.k_new[src_row + e];
-      const uint4 vv = p.v_new[src_row + e];
-      *reinterpret_cast<uint4*>(p.k_pages + dst) = kv;
-      *reinterpret_cast<uint4*>(p.v_pages + dst) = vv;
+    const int pieces = p.num_kv_heads * VEC;
+    // Up to four 16-byte pieces of K and of V per lane in flight before the
+    // stores (the sources are read-only for the whole kernel).
+    for (int e0 = lane; e0 < pieces; e0 += 4 * 32) {
+      uint4 kv[4], vv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + 32 * u;
+        if (e < pieces) {
+          kv[u] = __ldg(p.k_new + src_row + e);
+          vv[u] = __ldg(p.v_new + src_row + e);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + 32 * u;
+        if (e < pieces) {
+          const int64_t dst = dst_row + (e / VEC) * p.head_stride + (e % VEC) * 8;   // elements
+          *reinterpret_cast<uint4*>(p.k_pages + dst) = kv[u];
+          *reinterpret_cast<uint4*>(p.v_pages + dst) = vv[u];
+        }
+      }
     }
   }
 }

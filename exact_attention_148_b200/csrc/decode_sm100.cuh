@@ -26,6 +26,16 @@
 //
 // Accumulation order depends only on logical token positions, never on the
 // physical page ids, so permuting the page pool gives bit-identical output.
+//
+// FP8 cache (KV8): K/V pages hold E4M3 bytes with one scale per tensor.  A byte
+// s.eeee.mmm is widened with integer operations only: placed in a float's
+// bits 31 and 26..20 it reads as its E4M3 value times 2^-120 exactly (the
+// E4M3 exponent field lands in the float's biased exponent, so subnormals map
+// to float subnormals with the same ratio).  Scores are multiplied back by
+// 2^120 after the dot-product reduction (k_scale is folded into the query's
+// pre-scale); probabilities are taken as p * 2^60 so the P V accumulation
+// (~2^-60 p v) stays in the normal float range, and the final division
+// removes both factors and applies v_scale.
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -55,16 +65,23 @@ struct DecodeParams {
   int max_splits;
   int head_coord;                // tensor-map dimension (1..3) indexed by kv head
   int page_coord;                // tensor-map dimension (1..3) indexed by page id
-  float scale_log2;
+  float scale_log2;              // scale * log2(e) (* k_scale for an FP8 cache)
+  float v_scale;                 // FP8 cache: V dequantisation scale
 };
 
-template <int D, int GC>
+constexpr float kTwo60 = 1152921504606846976.0f;                           // 2^60
+constexpr float kTwo120 = 1329227995784915872903807060280344576.0f;       // 2^120
+
+template <int D, int GC, bool KV8>
 struct DecodeCfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(GC == 1 || GC == 2 || GC == 4 || GC == 8, "1, 2, 4 or 8 heads per CTA");
-  static constexpr int STAGES = 3;
+  static constexpr int ELEM = KV8 ? 1 : 2;             // bytes per cached element
+  // An FP8 page is half the bytes: twice the stages keeps as many bytes in flight.
+  static constexpr int STAGES = KV8 ? 6 : 3;
   static constexpr int COLS = D / 16;                  // columns per lane
-  static constexpr int TILE_BYTES = kDecodePage * D * 2;
+  static constexpr int ROW_BYTES = D * ELEM;
+  static constexpr int TILE_BYTES = kDecodePage * ROW_BYTES;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = STAGES * TILE_BYTES;
   static constexpr int SC_OFF = 2 * STAGES * TILE_BYTES;        // 4 warps x 16 x GC floats
@@ -133,12 +150,43 @@ __device__ __forceinline__ void load_bf16_row(const uint8_t* src, float2 (&f)[CO
   }
 }
 
+// E4M3 byte i (0..3, compile-time) of w as a float equal to its value times
+// 2^-120: the byte goes to bits 31..24, an arithmetic shift by 4 puts
+// s.eeee.mmm at bits 27..20 with the sign copied above, and the mask keeps the
+// sign at bit 31 and eeee.mmm at bits 26..20.
+template <int I>
+__device__ __forceinline__ float e4m3_scaled(uint32_t w) {
+  const int32_t t = static_cast<int32_t>(w << (24 - 8 * I));
+  return __int_as_float((t >> 4) & static_cast<int32_t>(0x87F00000u));
+}
+
+template <int COLS>
+__device__ __forceinline__ void load_e4m3_row(const uint8_t* src, float2 (&f)[COLS / 2]) {
+  if constexpr (COLS == 8) {
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    f[0] = make_float2(e4m3_scaled<0>(u.x), e4m3_scaled<1>(u.x));
+    f[1] = make_float2(e4m3_scaled<2>(u.x), e4m3_scaled<3>(u.x));
+    f[2] = make_float2(e4m3_scaled<0>(u.y), e4m3_scaled<1>(u.y));
+    f[3] = make_float2(e4m3_scaled<2>(u.y), e4m3_scaled<3>(u.y));
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+    f[0] = make_float2(e4m3_scaled<0>(u), e4m3_scaled<1>(u));
+    f[1] = make_float2(e4m3_scaled<2>(u), e4m3_scaled<3>(u));
+  }
+}
+
+template <bool KV8, int COLS>
+__device__ __forceinline__ void load_kv_row(const uint8_t* src, float2 (&f)[COLS / 2]) {
+  if constexpr (KV8) load_e4m3_row<COLS>(src, f);
+  else load_bf16_row<COLS>(src, f);
+}
+
 // Two CTAs per SM (their rings overlap each other's pipeline fill), except
 // with 8 packed heads, whose accumulators need the larger register budget.
-template <int D, int GC>
+template <int D, int GC, bool KV8>
 __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
     fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
-  using C = DecodeCfg<D, GC>;
+  using C = DecodeCfg<D, GC, KV8>;
   constexpr int COLS = C::COLS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -270,7 +318,7 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
       for (int ii = 0; ii < 8; ++ii) {
         const int tt = warp * 16 + 2 * ii + half;
         float2 kf[COLS / 2];
-        load_bf16_row<COLS>(Ks + tt * (D * 2) + c0 * 2, kf);
+        load_kv_row<KV8, COLS>(Ks + tt * C::ROW_BYTES + c0 * C::ELEM, kf);
 #pragma unroll
         for (int gi = 0; gi < GC; ++gi) {
           float2 a = make_float2(0.f, 0.f);
@@ -285,7 +333,7 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
         const int idx = xbase + k;
         const int ii = idx / GC, gi = idx % GC;
         const int tok = 2 * ii + half;
-        const float val = (tok0 + tok < t_end) ? part[k] : -INFINITY;
+        const float val = (tok0 + tok < t_end) ? (KV8 ? part[k] * kTwo120 : part[k]) : -INFINITY;
         if (writer) sc[tok * GC + gi] = val;
       }
       __syncwarp();
@@ -309,7 +357,8 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
 #pragma unroll
       for (int k = 0; k < PER; ++k) {
         const int idx = lane + 32 * k;
-        const float pv = ex2_approx(sv[k] - m_use);
+        // FP8: p * 2^60 keeps the P V products of E4M3 values (x 2^-120) normal
+        const float pv = ex2_approx(KV8 ? (sv[k] - m_use) + 60.0f : sv[k] - m_use);
         if (idx < E) sc[idx] = pv;
         ps += pv;
       }
@@ -333,7 +382,7 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
       for (int ii = 0; ii < 8; ++ii) {
         const int tok = 2 * ii + half;
         float2 vf[COLS / 2];
-        load_bf16_row<COLS>(Vs + (warp * 16 + tok) * (D * 2) + c0 * 2, vf);
+        load_kv_row<KV8, COLS>(Vs + (warp * 16 + tok) * C::ROW_BYTES + c0 * C::ELEM, vf);
         if (tok0 + tok >= t_end) {   // page tail past the cache end: never read its values
 #pragma unroll
           for (int c = 0; c < COLS / 2; ++c) vf[c] = make_float2(0.f, 0.f);
@@ -390,9 +439,13 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
           lsum += cmb_l[w * GC + gi] * f;
           o += cmb_o[(w * GC + gi) * D + c] * f;
         }
-        o = o / lsum;
+        if constexpr (KV8)   // o ~ 2^-60 sum p v, lsum = 2^60 sum p
+          o = (o * kTwo60) * (kTwo60 * p.v_scale / lsum);
+        else
+          o = o / lsum;
       }
-      const float lse_v = (M == -INFINITY) ? -INFINITY : (M + log2f(lsum)) * 0.69314718055994530942f;
+      const float lse_v = (M == -INFINITY) ? -INFINITY
+                                           : (M + log2f(lsum) - (KV8 ? 60.0f : 0.0f)) * 0.69314718055994530942f;
       const size_t row = static_cast<size_t>(b) * p.num_q_heads + qh0 + gi;
       if (direct) {
         p.out[row * D + c] = __float2bfloat16_rn(o);

@@ -57,11 +57,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-               const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz) {
+               const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
   const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+  CUresult r = fn(map, dtype, rank, const_cast<void*>(base), dims,
                   strides_bytes, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(static_cast<int>(r) + 10000);
@@ -151,7 +152,7 @@ int build_prefill_groups(const std::vector<int64_t>& q_lens, const std::vector<i
 int encode_page_pool_map(CUtensorMap* map, const void* pool, int64_t num_pages, int64_t page_stride,
                          int64_t token_stride, int64_t head_stride, int page_size, int num_kv_heads,
                          int head_dim, int box_cols, CUtensorMapSwizzle swz, int* head_coord,
-                         int* page_coord) {
+                         int* page_coord, int elem_bytes = 2) {
   struct Dim { int64_t stride; int64_t extent; int role; };   // role 0 token, 1 head, 2 page
   Dim dd[3] = {{token_stride, page_size, 0}, {head_stride, num_kv_heads, 1},
                {page_stride, num_pages, 2}};
@@ -161,30 +162,33 @@ int encode_page_pool_map(CUtensorMap* map, const void* pool, int64_t num_pages, 
   cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), 1, 1, 1};
   for (int i = 0; i < 3; ++i) {
     dims[i + 1] = static_cast<cuuint64_t>(dd[i].extent);
-    strides[i] = static_cast<cuuint64_t>(dd[i].stride) * 2;
+    strides[i] = static_cast<cuuint64_t>(dd[i].stride) * elem_bytes;
     if (dd[i].role == 0) box[i + 1] = static_cast<cuuint32_t>(page_size);
     if (dd[i].role == 1) *head_coord = i + 1;
     if (dd[i].role == 2) *page_coord = i + 1;
   }
-  return encode_map(map, pool, 4, dims, strides, box, swz);
+  return encode_map(map, pool, 4, dims, strides, box, swz,
+                    elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
-// Shared checks of a page pool's description (element strides).
+// Shared checks of a page pool's description (element strides; every stride
+// must be a multiple of 16 bytes).
 bool valid_pool(const void* k_pages, const void* v_pages, int64_t num_pages, int64_t page_stride,
-                int64_t token_stride, int64_t head_stride) {
+                int64_t token_stride, int64_t head_stride, int elem_bytes = 2) {
   if (!k_pages || !v_pages || !aligned(k_pages, 16) || !aligned(v_pages, 16)) return false;
   if (num_pages < 1 || num_pages > INT32_MAX) return false;
-  if (page_stride <= 0 || token_stride <= 0 || head_stride <= 0 || page_stride % 8 ||
-      token_stride % 8 || head_stride % 8)
+  const int64_t m = 16 / elem_bytes;
+  if (page_stride <= 0 || token_stride <= 0 || head_stride <= 0 || page_stride % m ||
+      token_stride % m || head_stride % m)
     return false;
   return true;
 }
 
 // ---------------------------------------------------------------------------- decode
-template <int D, int GC>
+template <int D, int GC, bool KV8>
 int launch_decode_split(const fa::DecodeParams& prm, dim3 grid, cudaStream_t stream) {
-  using C = fa::DecodeCfg<D, GC>;
-  auto kernel = fa::fa_decode_split_kernel<D, GC>;
+  using C = fa::DecodeCfg<D, GC, KV8>;
+  auto kernel = fa::fa_decode_split_kernel<D, GC, KV8>;
   int st = ensure_smem(reinterpret_cast<const void*>(kernel), C::SMEM_BYTES);
   if (st != FA_OK) return st;
   kernel<<<grid, fa::kDecodeThreads, C::SMEM_BYTES, stream>>>(prm);
@@ -192,13 +196,13 @@ int launch_decode_split(const fa::DecodeParams& prm, dim3 grid, cudaStream_t str
   return FA_OK;
 }
 
-template <int D>
+template <int D, bool KV8>
 int dispatch_decode_gc(int gc, const fa::DecodeParams& prm, dim3 grid, cudaStream_t stream) {
   switch (gc) {
-    case 1: return launch_decode_split<D, 1>(prm, grid, stream);
-    case 2: return launch_decode_split<D, 2>(prm, grid, stream);
-    case 4: return launch_decode_split<D, 4>(prm, grid, stream);
-    case 8: return launch_decode_split<D, 8>(prm, grid, stream);
+    case 1: return launch_decode_split<D, 1, KV8>(prm, grid, stream);
+    case 2: return launch_decode_split<D, 2, KV8>(prm, grid, stream);
+    case 4: return launch_decode_split<D, 4, KV8>(prm, grid, stream);
+    case 8: return launch_decode_split<D, 8, KV8>(prm, grid, stream);
   }
   return FA_ERR_UNSUPPORTED;
 }
@@ -450,11 +454,15 @@ FA_API void fa_plan_free(fa_plan* plan) {
   }
 }
 
-FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
-                           int64_t page_stride, int64_t token_stride, int64_t head_stride,
-                           const int32_t* block_table, const int32_t* cache_seqlens_dev,
-                           const fa_plan* plan, float scale, void* out, float* lse, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+namespace {
+
+// fa_decode_paged and fa_decode_paged_fp8: kv8 selects E4M3 pages with
+// per-tensor scales (k_scale, v_scale); both are 1 for a bf16 cache.
+int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                      int64_t page_stride, int64_t token_stride, int64_t head_stride,
+                      const int32_t* block_table, const int32_t* cache_seqlens_dev,
+                      const fa_plan* plan, float scale, bool kv8, float k_scale, float v_scale,
+                      void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   if (plan == nullptr || plan->p.magic != fa::kPlanMagic) return FA_ERR_INVALID_ARG;
   const fa::DecodePlan& pl = plan->p;
   if (!q || !k_pages || !v_pages || !block_table || !cache_seqlens_dev || !out)
@@ -462,7 +470,10 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
   if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
       !aligned(lse, 4) || !aligned(block_table, 4) || !aligned(cache_seqlens_dev, 4))
     return FA_ERR_INVALID_ARG;
-  if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride))
+  const int elem_bytes = kv8 ? 1 : 2;
+  if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride, elem_bytes))
+    return FA_ERR_INVALID_ARG;
+  if (!(k_scale > 0.0f) || std::isinf(k_scale) || !(v_scale > 0.0f) || std::isinf(v_scale))
     return FA_ERR_INVALID_ARG;
   if (pl.workspace_bytes > 0) {
     if (workspace == nullptr || !aligned(workspace, 256)) return FA_ERR_INVALID_ARG;
@@ -476,11 +487,13 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
   // whole rows (d columns) of one 64-token page per box, no swizzle
   int st = encode_page_pool_map(&prm.tm_k, k_pages, num_pages, page_stride, token_stride, head_stride,
                                 pl.page_size, pl.num_kv_heads, pl.head_dim, pl.head_dim,
-                                CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord);
+                                CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord,
+                                elem_bytes);
   if (st != FA_OK) return st;
   st = encode_page_pool_map(&prm.tm_v, v_pages, num_pages, page_stride, token_stride, head_stride,
                             pl.page_size, pl.num_kv_heads, pl.head_dim, pl.head_dim,
-                            CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord);
+                            CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord,
+                            elem_bytes);
   if (st != FA_OK) return st;
 
   prm.q = static_cast<const __nv_bfloat16*>(q);
@@ -501,12 +514,17 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
   prm.num_pages = static_cast<int>(num_pages);
   prm.chunk_tokens = pl.chunk_tokens;
   prm.max_splits = pl.max_splits;
-  prm.scale_log2 = scale * kLog2e;
+  prm.scale_log2 = scale * kLog2e * k_scale;
+  prm.v_scale = v_scale;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(pl.max_splits, pl.num_kv_heads * pl.subgroups, pl.batch);
-  st = pl.head_dim == 128 ? dispatch_decode_gc<128>(pl.heads_per_cta, prm, grid, s)
-                          : dispatch_decode_gc<64>(pl.heads_per_cta, prm, grid, s);
+  if (kv8)
+    st = pl.head_dim == 128 ? dispatch_decode_gc<128, true>(pl.heads_per_cta, prm, grid, s)
+                            : dispatch_decode_gc<64, true>(pl.heads_per_cta, prm, grid, s);
+  else
+    st = pl.head_dim == 128 ? dispatch_decode_gc<128, false>(pl.heads_per_cta, prm, grid, s)
+                            : dispatch_decode_gc<64, false>(pl.heads_per_cta, prm, grid, s);
   if (st != FA_OK) return st;
   if (pl.max_splits > 1) {
     fa::MergeParams mp;
@@ -523,6 +541,29 @@ FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pag
     st = launch_merge(mp, pl.head_dim, s);
   }
   return st;
+}
+
+}  // namespace
+
+FA_API int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                           int64_t page_stride, int64_t token_stride, int64_t head_stride,
+                           const int32_t* block_table, const int32_t* cache_seqlens_dev,
+                           const fa_plan* plan, float scale, void* out, float* lse, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return decode_paged_impl(q, k_pages, v_pages, num_pages, page_stride, token_stride, head_stride,
+                           block_table, cache_seqlens_dev, plan, scale, false, 1.0f, 1.0f, out, lse,
+                           workspace, workspace_bytes, stream);
+}
+
+FA_API int fa_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages,
+                               int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                               int64_t head_stride, const int32_t* block_table,
+                               const int32_t* cache_seqlens_dev, const fa_plan* plan, float scale,
+                               float k_scale, float v_scale, void* out, float* lse, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return decode_paged_impl(q, k_pages, v_pages, num_pages, page_stride, token_stride, head_stride,
+                           block_table, cache_seqlens_dev, plan, scale, true, k_scale, v_scale, out,
+                           lse, workspace, workspace_bytes, stream);
 }
 
 FA_API int fa_merge_states(const float* o_parts, const float* lse_parts, int num_states, int rows,

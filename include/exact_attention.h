@@ -211,6 +211,28 @@ int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, int
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_decode_paged_fp8 — fa_decode_paged over an FP8 KV cache (FP8 inference
+ * kernels: wsisp.com "FIA / FlashAttention", section 三, FP8 row).
+ *
+ * Same arguments, plan and workspace as fa_decode_paged, except:
+ *   k_pages, v_pages: E4M3 bytes (OCP FP8 E4M3: bias 7, subnormals, max 448),
+ *       same page layouts; strides are in elements (= bytes) and must be
+ *       multiples of 16.
+ *   k_scale, v_scale: per-tensor dequantisation scales (> 0, finite): the
+ *       cached key is k_scale * E4M3(k8), the value v_scale * E4M3(v8).
+ * q stays bf16; scores, softmax and P V accumulate in fp32; out is bf16.
+ * The code S.1111.111 (NaN in E4M3) is read as a finite +-480; a quantiser
+ * that saturates never writes it.  Slots past a request's cache length may
+ * hold any byte.
+ */
+int fa_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages,
+                        int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                        int64_t head_stride, const int32_t* block_table,
+                        const int32_t* cache_seqlens_dev, const fa_plan* plan, float scale,
+                        float k_scale, float v_scale, void* out, float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
  * fa_decode_paged_static — fa_decode_paged for callers that cannot allocate.
  *
  * The pages have no counterpart to this entry point; it exists for callers

@@ -43,7 +43,8 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
         lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
         lse_ref = np.asarray(lse_ref, dtype=np.float64)
         both_inf = np.isneginf(lse_gpu) & np.isneginf(lse_ref)
-        d = np.where(both_inf, 0.0, np.abs(lse_gpu - lse_ref))
+        with np.errstate(invalid="ignore"):
+            d = np.where(both_inf, 0.0, np.abs(lse_gpu - lse_ref))
         lerr = float(np.nanmax(d)) if d.size else 0.0
         assert not np.isnan(d).any(), f"{what}: NaN LSE"
         assert lerr <= LSE_ABS, f"{what}: LSE abs {lerr:.3e} > {LSE_ABS}"

@@ -27,7 +27,7 @@ def lib():
 def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_expected_api():
@@ -253,3 +253,19 @@ def test_append_validation_before_any_cuda_call(lib):
     assert call(npages=0) == fa.FA_ERR_INVALID_ARG
     assert call(strides=(64 * 2 * 128, 2 * 128, 12)) == fa.FA_ERR_INVALID_ARG
     assert call(total=0) == fa.FA_OK                                 # nothing to enqueue
+
+
+def test_decode_fp8_validation_before_any_cuda_call(lib):
+    p = _plan([1000, 3000], hq=8, hkv=2, splits=4)
+    A = 0x10000
+
+    def call(strides=(64 * 2 * 128, 2 * 128, 128), ks=0.5, vs=0.5):
+        return lib.fa_decode_paged_fp8(_fake(A), _fake(A), _fake(A), 100, *strides, _fake(A),
+                                       _fake(A), p.handle, float("nan"), ks, vs, _fake(A), None,
+                                       _fake(A), p.workspace_bytes, None)
+    assert call(ks=0.0) == fa.FA_ERR_INVALID_ARG
+    assert call(vs=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert call(ks=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert call(vs=float("nan")) == fa.FA_ERR_INVALID_ARG
+    # byte strides must be multiples of 16 (8 is fine for bf16 elements, not for bytes)
+    assert call(strides=(64 * 2 * 128, 2 * 128, 8)) == fa.FA_ERR_INVALID_ARG
