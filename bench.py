@@ -170,7 +170,7 @@ class PrefillCase:
 
 
 class DecodeCase:
-    def __init__(self, inp: W.DecodeInputs, device, num_splits=0):
+    def __init__(self, inp: W.DecodeInputs, device, num_splits=0, kernel="auto"):
         import torch
         import exact_attention_148_b200 as fa
         self.inp = inp
@@ -188,7 +188,8 @@ class DecodeCase:
         self.plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=inp.num_q_heads,
                                    num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
                                    page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
-                                   num_splits=num_splits)
+                                   num_splits=num_splits, kv_dtype="e4m3" if self.fp8 else "bf16",
+                                   kernel=kernel)
         self.plan_ms = (time.perf_counter() - t0) * 1e3
         self.ws = torch.empty(max(self.plan.workspace_bytes, 256), dtype=torch.uint8, device=device)
         self.out = torch.empty_like(self.q)
@@ -243,6 +244,7 @@ class DecodeCase:
                 "kv_dtype": "e4m3 (per-tensor scales)" if self.fp8 else "bf16",
                 "chunk_tokens": info.chunk_tokens,
                 "max_splits": info.max_splits, "work_items": info.num_work_items,
+                "split_kernel": "tensor cores (tcgen05)" if info.tensor_cores else "CUDA cores",
                 "plan_ms": round(self.plan_ms, 3), "algorithmic_gb": round(self.bytes / 1e9, 4)}
 
 
@@ -508,13 +510,14 @@ def oracle_chunked_sample(inp: W.ChunkedPrefillInputs, budget_s: float):
 
 # ----------------------------------------------------------------------------- main
 
-def build_cases(workload, device, num_splits):
+def build_cases(workload, device, num_splits, kernel="auto"):
     if workload == "default":
-        return [PrefillCase(W.varlen_causal_prefill(), device), DecodeCase(W.paged_decode_batch(), device)]
+        return [PrefillCase(W.varlen_causal_prefill(), device),
+                DecodeCase(W.paged_decode_batch(), device, 0, kernel)]
     if workload in PREFILL_WORKLOADS:
         return [PrefillCase(W.CONFIGS[workload](), device)]
     if workload in DECODE_WORKLOADS:
-        return [DecodeCase(W.CONFIGS[workload](), device, num_splits)]
+        return [DecodeCase(W.CONFIGS[workload](), device, num_splits, kernel)]
     if workload in CHUNKED_WORKLOADS:
         st = ChunkedState(W.CONFIGS[workload](), device)
         return [AppendCase(st), ChunkedAttnCase(st)]
@@ -589,7 +592,7 @@ def run_ours(args):
     device = torch.device("cuda", dist_ctx.local if dist_ctx else 0)
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
-    cases = build_cases(args.workload, device, args.num_splits)
+    cases = build_cases(args.workload, device, args.num_splits, args.decode_kernel)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -627,8 +630,8 @@ def run_ours(args):
         else:
             e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
                                measured_traffic("decode", c.inp.name, c))
-            e["kernel"] = ("fa_decode_split_kernel<e4m3>" if c.fp8 else "fa_decode_split_kernel") + \
-                " + fa_merge_kernel (one decode call)"
+            e["kernel"] = ("fa_decode_tc_kernel" if c.plan.info.tensor_cores else "fa_decode_split_kernel") + \
+                ("<e4m3>" if c.fp8 else "") + " + fa_merge_kernel (one decode call)"
         e["workload"] = c.inp.name
         e["ms_per_launch"] = round(ms / c.launches, 4)
         rooflines.append(e)
@@ -765,6 +768,7 @@ def main():
                     help="default | " + " | ".join(sorted(PREFILL_WORKLOADS | DECODE_WORKLOADS |
                                                           CHUNKED_WORKLOADS)))
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")

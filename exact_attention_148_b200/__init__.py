@@ -39,8 +39,14 @@ EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
-    "fa_decode_paged_fp8",
+    "fa_decode_paged_fp8", "fa_decode_plan_kv",
 ]
+
+FA_KV_BF16, FA_KV_E4M3 = 0, 1
+FA_DECODE_AUTO, FA_DECODE_CUDA_CORES, FA_DECODE_TENSOR_CORES = 0, 1, 2
+_KV_DTYPES = {"bf16": FA_KV_BF16, "e4m3": FA_KV_E4M3}
+_KERNELS = {"auto": FA_DECODE_AUTO, "cuda_cores": FA_DECODE_CUDA_CORES,
+            "tensor_cores": FA_DECODE_TENSOR_CORES}
 
 # Size of the library's static decode scratch (FA_STATIC_SCRATCH_BYTES).
 STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -61,7 +67,8 @@ class _PlanInfo(ctypes.Structure):
         ("head_dim", ctypes.c_int), ("page_size", ctypes.c_int), ("max_pages_per_seq", ctypes.c_int),
         ("chunk_tokens", ctypes.c_int), ("max_splits", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
         ("num_work_items", ctypes.c_int), ("max_seqlen", ctypes.c_int),
-        ("workspace_bytes", ctypes.c_size_t),
+        ("workspace_bytes", ctypes.c_size_t), ("kv_dtype", ctypes.c_int),
+        ("tensor_cores", ctypes.c_int),
     ]
 
 
@@ -83,6 +90,9 @@ def library() -> ctypes.CDLL:
     L.fa_decode_plan.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                  ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t)]
     L.fa_decode_plan.restype = i32
+    L.fa_decode_plan_kv.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, i32,
+                                    ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t)]
+    L.fa_decode_plan_kv.restype = i32
     L.fa_plan_get_info.argtypes = [vp, ctypes.POINTER(_PlanInfo)]
     L.fa_plan_get_info.restype = i32
     L.fa_plan_free.argtypes = [vp]
@@ -204,6 +214,8 @@ class PlanInfo:
     num_work_items: int
     max_seqlen: int
     workspace_bytes: int
+    kv_dtype: int
+    tensor_cores: int
 
 
 class DecodePlan:
@@ -234,19 +246,22 @@ class DecodePlan:
 
 def decode_plan(cache_seqlens_host, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
                 page_size: int = 64, max_pages_per_seq: int, num_sms: int | None = None,
-                num_splits: int = 0) -> DecodePlan:
+                num_splits: int = 0, kv_dtype: str = "bf16", kernel: str = "auto") -> DecodePlan:
     """Plan the split of every request's cached context (host only, no GPU needed
-    when ``num_sms`` is given)."""
+    when ``num_sms`` is given).  ``kv_dtype``: "bf16" (for decode_paged) or
+    "e4m3" (for decode_paged_fp8); ``kernel``: "auto", "cuda_cores" or
+    "tensor_cores"."""
     lens = np.ascontiguousarray(np.asarray(cache_seqlens_host, dtype=np.int32))
     if num_sms is None:
         torch = _torch()
         num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     h = ctypes.c_void_p()
     ws = ctypes.c_size_t()
-    st = library().fa_decode_plan(lens.ctypes.data_as(ctypes.c_void_p), len(lens), num_q_heads,
-                                  num_kv_heads, head_dim, page_size, max_pages_per_seq, num_sms,
-                                  num_splits, ctypes.byref(h), ctypes.byref(ws))
-    _check(st, "fa_decode_plan")
+    st = library().fa_decode_plan_kv(lens.ctypes.data_as(ctypes.c_void_p), len(lens), num_q_heads,
+                                     num_kv_heads, head_dim, page_size, max_pages_per_seq, num_sms,
+                                     num_splits, _KV_DTYPES[kv_dtype], _KERNELS[kernel],
+                                     ctypes.byref(h), ctypes.byref(ws))
+    _check(st, "fa_decode_plan_kv")
     return DecodePlan(h, ws.value)
 
 

@@ -48,6 +48,7 @@ constexpr int kDecodeThreads = 160;
 struct DecodeParams {
   CUtensorMap tm_k;   // 4-D over the page pool, dims sorted by stride: {d, ., ., .}
   CUtensorMap tm_v;
+  CUtensorMap tm_q;   // tensor-core kernel, bf16: 3-D {d, Hq, B}, box {64, NPAD, 1}
   const __nv_bfloat16* q;        // [B, Hq, d]
   const int32_t* block_table;    // [B, max_pages]
   const int32_t* cache_seqlens;  // [B]

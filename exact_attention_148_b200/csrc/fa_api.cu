@@ -16,6 +16,7 @@
 #include "../../include/exact_attention.h"
 #include "append_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "decode_tc_sm100.cuh"
 #include "planner.h"
 #include "prefill_pp_sm100.cuh"
 
@@ -205,6 +206,17 @@ int dispatch_decode_gc(int gc, const fa::DecodeParams& prm, dim3 grid, cudaStrea
     case 8: return launch_decode_split<D, 8, KV8>(prm, grid, stream);
   }
   return FA_ERR_UNSUPPORTED;
+}
+
+template <bool KV8, int NPAD>
+int launch_decode_tc(const fa::DecodeParams& prm, dim3 grid, cudaStream_t stream) {
+  using C = fa::DecodeTcCfg<KV8, NPAD>;
+  auto kernel = fa::fa_decode_tc_kernel<KV8, NPAD>;
+  int st = ensure_smem(reinterpret_cast<const void*>(kernel), C::SMEM_BYTES);
+  if (st != FA_OK) return st;
+  kernel<<<grid, fa::kDecodeTcThreads, C::SMEM_BYTES, stream>>>(prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
 }
 
 int launch_merge(const fa::MergeParams& mp, int head_dim, cudaStream_t stream) {
@@ -411,15 +423,17 @@ FA_API int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_
   return FA_OK;
 }
 
-FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
-                          int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
-                          int num_sms, int num_splits_override, fa_plan** plan_out,
-                          size_t* workspace_bytes) {
+FA_API int fa_decode_plan_kv(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                             int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                             int num_sms, int num_splits_override, int kv_dtype, int kernel,
+                             fa_plan** plan_out, size_t* workspace_bytes) {
   if (plan_out == nullptr) return FA_ERR_INVALID_ARG;
   *plan_out = nullptr;
+  if (kv_dtype != FA_KV_BF16 && kv_dtype != FA_KV_E4M3) return FA_ERR_INVALID_ARG;
   fa::DecodePlan p;
   int st = fa::make_decode_plan(cache_seqlens_host, batch, num_q_heads, num_kv_heads, head_dim,
-                                page_size, max_pages_per_seq, num_sms, num_splits_override, &p);
+                                page_size, max_pages_per_seq, num_sms, num_splits_override,
+                                kv_dtype == FA_KV_E4M3 ? 1 : 2, kernel, &p);
   if (st != FA_OK) return st;
   fa_plan* plan = new (std::nothrow) fa_plan;
   if (plan == nullptr) return FA_ERR_INVALID_ARG;
@@ -427,6 +441,15 @@ FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_
   *plan_out = plan;
   if (workspace_bytes) *workspace_bytes = plan->p.workspace_bytes;
   return FA_OK;
+}
+
+FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                          int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                          int num_sms, int num_splits_override, fa_plan** plan_out,
+                          size_t* workspace_bytes) {
+  return fa_decode_plan_kv(cache_seqlens_host, batch, num_q_heads, num_kv_heads, head_dim, page_size,
+                           max_pages_per_seq, num_sms, num_splits_override, FA_KV_BF16,
+                           FA_DECODE_AUTO, plan_out, workspace_bytes);
 }
 
 FA_API int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info) {
@@ -444,6 +467,8 @@ FA_API int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info) {
   info->num_work_items = p.num_work_items;
   info->max_seqlen = p.max_seqlen;
   info->workspace_bytes = p.workspace_bytes;
+  info->kv_dtype = p.kv_elem_bytes == 1 ? FA_KV_E4M3 : FA_KV_BF16;
+  info->tensor_cores = p.tensor_cores ? 1 : 0;
   return FA_OK;
 }
 
@@ -471,6 +496,7 @@ int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, i
       !aligned(lse, 4) || !aligned(block_table, 4) || !aligned(cache_seqlens_dev, 4))
     return FA_ERR_INVALID_ARG;
   const int elem_bytes = kv8 ? 1 : 2;
+  if (pl.kv_elem_bytes != elem_bytes) return FA_ERR_PLAN_MISMATCH;
   if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride, elem_bytes))
     return FA_ERR_INVALID_ARG;
   if (!(k_scale > 0.0f) || std::isinf(k_scale) || !(v_scale > 0.0f) || std::isinf(v_scale))
@@ -484,17 +510,29 @@ int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, i
 
   static thread_local fa::DecodeParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  // whole rows (d columns) of one 64-token page per box, no swizzle
+  // CUDA-core kernel: whole rows (d columns) of one 64-token page per box, no
+  // swizzle.  Tensor-core kernel: 128-byte column chunks with the 128-byte
+  // swizzle the MMA operand descriptors expect.
+  const int box_cols = pl.tensor_cores ? 128 / elem_bytes : pl.head_dim;
+  const CUtensorMapSwizzle swz = pl.tensor_cores ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   int st = encode_page_pool_map(&prm.tm_k, k_pages, num_pages, page_stride, token_stride, head_stride,
-                                pl.page_size, pl.num_kv_heads, pl.head_dim, pl.head_dim,
-                                CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord,
-                                elem_bytes);
+                                pl.page_size, pl.num_kv_heads, pl.head_dim, box_cols, swz,
+                                &prm.head_coord, &prm.page_coord, elem_bytes);
   if (st != FA_OK) return st;
   st = encode_page_pool_map(&prm.tm_v, v_pages, num_pages, page_stride, token_stride, head_stride,
-                            pl.page_size, pl.num_kv_heads, pl.head_dim, pl.head_dim,
-                            CU_TENSOR_MAP_SWIZZLE_NONE, &prm.head_coord, &prm.page_coord,
-                            elem_bytes);
+                            pl.page_size, pl.num_kv_heads, pl.head_dim, box_cols, swz,
+                            &prm.head_coord, &prm.page_coord, elem_bytes);
   if (st != FA_OK) return st;
+  const int npad = pl.group <= 8 ? 8 : 16;
+  if (pl.tensor_cores && !kv8) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(pl.head_dim),
+                                static_cast<cuuint64_t>(pl.num_q_heads), static_cast<cuuint64_t>(pl.batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pl.head_dim) * 2,
+                                   static_cast<cuuint64_t>(pl.num_q_heads) * pl.head_dim * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(npad), 1};
+    st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
 
   prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.block_table = block_table;
@@ -519,7 +557,12 @@ int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, i
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(pl.max_splits, pl.num_kv_heads * pl.subgroups, pl.batch);
-  if (kv8)
+  if (pl.tensor_cores) {
+    if (kv8)
+      st = npad == 8 ? launch_decode_tc<true, 8>(prm, grid, s) : launch_decode_tc<true, 16>(prm, grid, s);
+    else
+      st = npad == 8 ? launch_decode_tc<false, 8>(prm, grid, s) : launch_decode_tc<false, 16>(prm, grid, s);
+  } else if (kv8)
     st = pl.head_dim == 128 ? dispatch_decode_gc<128, true>(pl.heads_per_cta, prm, grid, s)
                             : dispatch_decode_gc<64, true>(pl.heads_per_cta, prm, grid, s);
   else

@@ -16,12 +16,24 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Decode-time model used to choose the split size (measured on B200, 148 SMs):
 // all resident split CTAs share the HBM bandwidth, one CTA alone cannot pull
-// more than ~44 GB/s (its TMA ring depth), each CTA costs ~0.5 us of fill, and a
-// second (merge) launch costs ~5 us.
+// more than its ring depth allows (~44 GB/s for the CUDA-core kernel's three
+// 32 KB stages; the tensor-core kernel keeps 192 KB (bf16) or 96 KB (E4M3) in
+// flight), each CTA costs ~0.5 us of fill, and a second (merge) launch costs
+// ~5 us.
 constexpr double kHbmBytesPerUs148 = 6.9e6;       // bytes per microsecond, 148 SMs
-constexpr double kCtaBytesPerUs = 4.36e4;
 constexpr double kCtaOverheadUs = 0.5;
 constexpr double kMergeLaunchUs = 5.0;
+
+struct CtaModel {
+  double bytes_per_us;   // one CTA's ceiling
+  int ctas_per_sm;
+};
+
+CtaModel cta_model(bool tensor_cores, int kv_elem_bytes, int heads_per_cta) {
+  // (the CUDA-core kernel's E4M3 ring holds as many bytes as its bf16 one)
+  if (tensor_cores) return {kv_elem_bytes == 1 ? 7.0e4 : 1.4e5, kv_elem_bytes == 1 ? 2 : 1};
+  return {4.36e4, heads_per_cta == 8 ? 1 : 2};
+}
 
 // Estimated duration (us) of the split kernel (+ merge) for one chunk size:
 // CTAs enter the resident slots in grid order (split fastest, then kv-head
@@ -30,10 +42,10 @@ constexpr double kMergeLaunchUs = 5.0;
 // points measured in "bytes done by every running CTA" (all running CTAs
 // advance at the same rate, so that scale is shared).
 double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64_t chunk, int slots,
-                          int head_dim, int num_sms) {
-  const double bytes_per_token = 2.0 * head_dim * 2.0;   // K and V rows of one kv head
+                          int head_dim, int kv_elem_bytes, double cta_bytes_per_us, int num_sms) {
+  const double bytes_per_token = 2.0 * head_dim * kv_elem_bytes;   // K and V rows of one kv head
   const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
-  const double overhead_bytes = kCtaOverheadUs * kCtaBytesPerUs;
+  const double overhead_bytes = kCtaOverheadUs * cta_bytes_per_us;
   std::priority_queue<double, std::vector<double>, std::greater<double>> running;
   double v = 0.0, t = 0.0;
   size_t b = 0;
@@ -64,7 +76,7 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
     running.push(v + c);
   }
   while (!running.empty()) {
-    const double rate = std::min(kCtaBytesPerUs, hbm / static_cast<double>(running.size()));
+    const double rate = std::min(cta_bytes_per_us, hbm / static_cast<double>(running.size()));
     const double nxt = running.top();
     running.pop();
     t += (nxt - v) / rate;
@@ -78,8 +90,11 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
 
 int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
                      int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
-                     int num_sms, int num_splits_override, DecodePlan* plan) {
+                     int num_sms, int num_splits_override, int kv_elem_bytes, int kernel,
+                     DecodePlan* plan) {
   if (plan == nullptr || cache_seqlens_host == nullptr) return FA_ERR_INVALID_ARG;
+  if (kv_elem_bytes != 1 && kv_elem_bytes != 2) return FA_ERR_INVALID_ARG;
+  if (kernel < kDecodeKernelAuto || kernel > kDecodeKernelTensorCores) return FA_ERR_INVALID_ARG;
   if (batch < 1 || batch > 65535 || num_q_heads < 1 || num_kv_heads < 1 ||
       max_pages_per_seq < 1 || num_sms < 1 || num_splits_override < 0)
     return FA_ERR_INVALID_ARG;
@@ -98,11 +113,22 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
   pl.max_pages_per_seq = max_pages_per_seq;
   pl.num_sms = num_sms;
   pl.group = num_q_heads / num_kv_heads;
-  for (int gc : {8, 4, 2, 1})
-    if (pl.group % gc == 0) {
-      pl.heads_per_cta = gc;
-      break;
-    }
+  pl.kv_elem_bytes = kv_elem_bytes;
+  const bool tc_ok = head_dim == 128 && pl.group <= kTensorCoreMaxGroup;
+  if (kernel == kDecodeKernelTensorCores && !tc_ok) return FA_ERR_UNSUPPORTED;
+  // Tensor cores by default for an E4M3 cache (the CUDA-core loop spends an
+  // integer widening and G FMAs on every byte) and for groups of 8 or more.
+  pl.tensor_cores = kernel == kDecodeKernelTensorCores ||
+                    (kernel == kDecodeKernelAuto && tc_ok && (kv_elem_bytes == 1 || pl.group >= 8));
+  if (pl.tensor_cores) {
+    pl.heads_per_cta = pl.group;
+  } else {
+    for (int gc : {8, 4, 2, 1})
+      if (pl.group % gc == 0) {
+        pl.heads_per_cta = gc;
+        break;
+      }
+  }
   pl.subgroups = pl.group / pl.heads_per_cta;
   if (static_cast<int64_t>(num_kv_heads) * pl.subgroups > 65535) return FA_ERR_UNSUPPORTED;
 
@@ -128,7 +154,8 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     // Try split counts s (chunk = ceil(max_len / s) rounded to a page, at
     // least kMinChunkTokens keys) plus the many-small-items rule, and keep the
     // one the decode-time model estimates fastest (ties: fewer splits).
-    const int slots = num_sms * (pl.heads_per_cta == 8 ? 1 : kDecodeCtasPerSm);
+    const CtaModel cm = cta_model(pl.tensor_cores, kv_elem_bytes, pl.heads_per_cta);
+    const int slots = num_sms * cm.ctas_per_sm;
     std::vector<int64_t> cands;
     for (int s : {1, 2, 3, 4, 5, 6, 8, 10, 12, 16, 20, 24, 32, 48, 64, 96, 128})
       cands.push_back(round_up(ceil_div(max_len, s), page_size));
@@ -139,7 +166,8 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     for (int64_t c : cands) {
       c = std::max<int64_t>(c, kMinChunkTokens);
       if (ceil_div(max_len, c) > kMaxSplits) continue;
-      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, num_sms);
+      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes,
+                                          cm.bytes_per_us, num_sms);
       if (chunk == 0 || t < best_t * (1.0 - 1e-9) || (t <= best_t * (1.0 + 1e-9) && c > chunk)) {
         best_t = t;
         chunk = c;

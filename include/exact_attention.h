@@ -55,6 +55,16 @@ typedef enum {
 /* Opaque host-side decode plan, created by fa_decode_plan, freed by fa_plan_free. */
 typedef struct fa_plan fa_plan;
 
+/* Element type of a paged KV cache. */
+typedef enum { FA_KV_BF16 = 0, FA_KV_E4M3 = 1 } fa_kv_dtype;
+
+/* Decode split kernel a plan targets. */
+typedef enum {
+  FA_DECODE_AUTO = 0,          /* the planner chooses */
+  FA_DECODE_CUDA_CORES = 1,    /* fp32 FMAs per element, up to 8 heads per CTA */
+  FA_DECODE_TENSOR_CORES = 2   /* tcgen05 MMAs, all G <= 16 heads of a kv head per CTA; d = 128 */
+} fa_decode_kernel;
+
 /* Read-only view of a plan (for tests and tools). */
 typedef struct {
   int batch;
@@ -69,6 +79,8 @@ typedef struct {
   int num_work_items;    /* non-empty (request, kv-head group, split) items */
   int max_seqlen;        /* longest planned cache length */
   size_t workspace_bytes;
+  int kv_dtype;          /* fa_kv_dtype the plan was made for */
+  int tensor_cores;      /* 1 if the plan runs the tensor-core split kernel */
 } fa_plan_info;
 
 /*
@@ -176,6 +188,21 @@ int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads
                    int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
                    int num_sms, int num_splits_override, fa_plan** plan_out,
                    size_t* workspace_bytes);
+
+/*
+ * fa_decode_plan_kv — fa_decode_plan for a given cache element type and split
+ * kernel.  kv_dtype: FA_KV_BF16 (plans for fa_decode_paged) or FA_KV_E4M3
+ * (plans for fa_decode_paged_fp8; a plan is only accepted by the entry point
+ * of its type, else FA_ERR_PLAN_MISMATCH).  kernel: FA_DECODE_AUTO picks the
+ * tensor-core kernel for an E4M3 cache or a group of 8 or more heads when
+ * d = 128 and Hq/Hkv <= 16; FA_DECODE_TENSOR_CORES outside that range is
+ * FA_ERR_UNSUPPORTED.  fa_decode_plan(...) is
+ * fa_decode_plan_kv(..., FA_KV_BF16, FA_DECODE_AUTO, ...).
+ */
+int fa_decode_plan_kv(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                      int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                      int num_sms, int num_splits_override, int kv_dtype, int kernel,
+                      fa_plan** plan_out, size_t* workspace_bytes);
 
 int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info);
 void fa_plan_free(fa_plan* plan);

@@ -59,7 +59,7 @@ def prefill_on_gpu(inp: W.PrefillInputs, **kw):
                       cu_seqlens_host=inp.cu_seqlens, **kw)
 
 
-def decode_on_gpu(inp: W.DecodeInputs, num_splits=0, plan=None, dev=None, **kw):
+def decode_on_gpu(inp: W.DecodeInputs, num_splits=0, plan=None, dev=None, kernel="auto", **kw):
     import exact_attention_148_b200 as fa
     if dev is None:
         dev = decode_device_inputs(inp)
@@ -67,7 +67,7 @@ def decode_on_gpu(inp: W.DecodeInputs, num_splits=0, plan=None, dev=None, **kw):
         plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=inp.num_q_heads,
                               num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
                               page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
-                              num_splits=num_splits)
+                              num_splits=num_splits, kernel=kernel)
     out, lse = fa.decode_paged(dev["q"], dev["k"], dev["v"], dev["bt"], dev["lens"], plan,
                                layout=inp.layout, scale=inp.scale, **kw)
     return out, lse, plan

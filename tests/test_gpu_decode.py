@@ -15,8 +15,8 @@ def oracle_rows(inp, rows):
                                         inp.page_size, inp.layout, to_f64=W.as_f64)
 
 
-def check_all_rows(inp, num_splits=0, what=""):
-    out, lse, plan = decode_on_gpu(inp, num_splits)
+def check_all_rows(inp, num_splits=0, what="", kernel="auto"):
+    out, lse, plan = decode_on_gpu(inp, num_splits, kernel=kernel)
     rows = [(b, h) for b in range(inp.batch) for h in range(inp.num_q_heads)]
     o_ref, l_ref = oracle_rows(inp, rows)
     compare(bf16_to_f64(out).reshape(-1, inp.head_dim), lse.cpu().numpy().reshape(-1), o_ref, l_ref,
@@ -169,3 +169,22 @@ def test_ragged_split_decode_config_sampled():
     inp = W.ragged_split_decode()
     rows = [(0, h) for h in (0, 7, 31)] + _sample(inp, 24, 5)
     check_sampled(inp, sorted(set(rows)), 0, "ragged split decode")
+
+
+@pytest.mark.parametrize("kernel", ["tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (8, 2), (16, 2), (6, 2), (12, 1), (8, 1)])
+def test_group_sizes_both_kernels(hq, hkv, kernel):
+    inp = W.make_decode([70, 1500, 129, 0, 4097], hq, hkv, 128, seed=900 + hq * 7 + hkv)
+    check_all_rows(inp, 0, f"decode {kernel} hq={hq} hkv={hkv}", kernel)
+    check_all_rows(inp, 5, f"decode {kernel} hq={hq} hkv={hkv} 5 splits", kernel)
+
+
+def test_tensor_core_poisoned_and_permuted():
+    import torch
+    inp = W.poison_unused(W.make_decode(SMALL_LENS, 16, 2, 128, seed=950, extra_pages=4))
+    check_all_rows(inp, 3, "tc poisoned", "tensor_cores")
+    a = decode_on_gpu(inp, 3, kernel="tensor_cores")
+    b = decode_on_gpu(W.permute_pages(inp, 7), 3, kernel="tensor_cores")
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    c = decode_on_gpu(W.relayout(inp, "HND"), 3, kernel="tensor_cores")
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])

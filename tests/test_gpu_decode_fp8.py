@@ -20,13 +20,13 @@ def fp8_device_inputs(inp):
                 bt=to_dev_i32(inp.block_table), lens=to_dev_i32(inp.cache_seqlens))
 
 
-def run_fp8(inp, num_splits=0, dev=None):
+def run_fp8(inp, num_splits=0, dev=None, kernel="auto"):
     import exact_attention_148_b200 as fa
     dev = dev or fp8_device_inputs(inp)
     plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=inp.num_q_heads,
                           num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
                           page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
-                          num_splits=num_splits)
+                          num_splits=num_splits, kv_dtype="e4m3", kernel=kernel)
     out, lse = fa.decode_paged_fp8(dev["q"], dev["k"], dev["v"], dev["bt"], dev["lens"], plan,
                                    k_scale=inp.extra["k_scale"], v_scale=inp.extra["v_scale"],
                                    layout=inp.layout, scale=inp.scale)
@@ -42,10 +42,10 @@ def oracle_rows(inp, rows):
                                         v_to_f64=lambda a: oracle.dequantize_e4m3(a, vs))
 
 
-def check_all_rows(inp, num_splits=0, what=""):
+def check_all_rows(inp, num_splits=0, what="", kernel="auto"):
     import exact_attention_148_b200 as fa
     assert fa.device_status(clear=True) == 0
-    out, lse = run_fp8(inp, num_splits)
+    out, lse = run_fp8(inp, num_splits, kernel=kernel)
     rows = [(b, h) for b in range(inp.batch) for h in range(inp.num_q_heads)]
     o_ref, l_ref = oracle_rows(inp, rows)
     compare(bf16_to_f64(out).reshape(-1, inp.head_dim), lse.cpu().numpy().reshape(-1), o_ref, l_ref,
@@ -57,18 +57,29 @@ def check_all_rows(inp, num_splits=0, what=""):
 SMALL_LENS = [1, 63, 64, 65, 1000, 4097, 0]
 
 
+KERNELS = ["tensor_cores", "cuda_cores"]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("num_splits", [0, 1, 3, 16])
-def test_small_batch_all_rows(num_splits):
+def test_small_batch_all_rows(num_splits, kernel):
     inp = W.to_fp8_cache(W.make_decode(SMALL_LENS, 8, 2, 128, seed=800))
-    check_all_rows(inp, num_splits, f"fp8 decode splits={num_splits}")
+    check_all_rows(inp, num_splits, f"fp8 decode splits={num_splits} {kernel}", kernel)
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2), (16, 2), (6, 2), (8, 1)])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2), (16, 2), (6, 2), (8, 1), (32, 2), (12, 1)])
 def test_group_sizes(d, hq, hkv):
+    """Automatic kernel choice: tensor cores at d = 128 for groups up to 16."""
     inp = W.to_fp8_cache(W.make_decode([70, 1500, 129], hq, hkv, d, seed=810 + d + hq + hkv))
     check_all_rows(inp, 0, f"fp8 d={d} hq={hq} hkv={hkv}")
     check_all_rows(inp, 4, f"fp8 d={d} hq={hq} hkv={hkv} 4 splits")
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2), (16, 2), (6, 2)])
+def test_group_sizes_cuda_cores(hq, hkv):
+    inp = W.to_fp8_cache(W.make_decode([70, 1500, 129], hq, hkv, 128, seed=815 + hq + hkv))
+    check_all_rows(inp, 3, f"fp8 cuda cores hq={hq} hkv={hkv}", "cuda_cores")
 
 
 def test_hnd_layout_is_bit_identical():
@@ -87,24 +98,28 @@ def test_page_permutation_is_bit_identical():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_unused_slots_hold_nan_codes():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_unused_slots_hold_nan_codes(kernel):
     inp = W.poison_unused(W.to_fp8_cache(W.make_decode(SMALL_LENS, 8, 2, 128, seed=840,
                                                        extra_pages=3)))
-    check_all_rows(inp, 2, "fp8 poisoned")
+    check_all_rows(inp, 2, f"fp8 poisoned {kernel}", kernel)
 
 
-def test_subnormal_heavy_cache():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_subnormal_heavy_cache(kernel):
     """Scales 1024x too large: many codes land in the E4M3 subnormal range."""
     inp = W.to_fp8_cache(W.make_decode([500, 2000], 8, 2, 128, seed=850), amax=4.0 * 1024)
     codes = inp.k_pages_bits & 0x7F
     assert np.mean((codes >> 3) == 0) > 0.05
-    check_all_rows(inp, 0, "fp8 subnormal-heavy")
+    check_all_rows(inp, 0, f"fp8 subnormal-heavy {kernel}", kernel)
 
 
-def test_every_code_decodes_exactly():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_every_code_decodes_exactly(kernel):
     """One cached token per request: O is that token's V row and LSE its score,
     so every E4M3 code (NaN codes excepted) is checked on its own, through
-    both the V and the K path."""
+    both the V and the K path.  (On tensor cores P = 1 is exact in E4M3 and
+    the one-hot query splits exactly, so this stays exact there too.)"""
     import exact_attention_148_b200 as fa
     B, Hq, Hkv, d = 32, 8, 1, 128
     base = W.make_decode([1] * B, Hq, Hkv, d, seed=860)
@@ -123,7 +138,7 @@ def test_every_code_decodes_exactly():
             q[b, h, c] = 1.0
     inp = W.DecodeInputs("every_code", W.f32_to_bf16_bits(q), kp, vp, base.block_table,
                          base.cache_seqlens, 1.0, extra={"k_scale": 1.0 / 64, "v_scale": 1.0})
-    out, lse = run_fp8(inp)
+    out, lse = run_fp8(inp, kernel=kernel)
     assert fa.device_status(clear=True) == 0
     want_v = oracle.e4m3_to_f64(vp[base.block_table[:, 0], 0, 0, :])        # [B, d]
     got = bf16_to_f64(out)                                                   # [B, Hq, d]
@@ -134,9 +149,10 @@ def test_every_code_decodes_exactly():
     np.testing.assert_allclose(lse.cpu().numpy(), want_s, rtol=2e-6, atol=2e-6)
 
 
-def test_full_size_sampled_rows():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_full_size_sampled_rows(kernel):
     inp = W.paged_decode_batch_fp8()
-    out, lse = run_fp8(inp)
+    out, lse = run_fp8(inp, kernel=kernel)
     g = np.random.default_rng(11)
     rows = [(int(b), int(h)) for b, h in zip(g.integers(0, inp.batch, 48),
                                              g.integers(0, inp.num_q_heads, 48))]

@@ -58,12 +58,14 @@ def test_version_and_strerror(lib):
     assert fa.strerror(12345) == "unknown status"
 
 
-def _plan(lens, hq=32, hkv=8, d=128, max_pages=None, num_sms=148, splits=0):
+def _plan(lens, hq=32, hkv=8, d=128, max_pages=None, num_sms=148, splits=0, kv_dtype="bf16",
+          kernel="auto"):
     lens = np.asarray(lens, dtype=np.int32)
     if max_pages is None:
         max_pages = max(1, int(np.max((lens + 63) // 64)))
     return fa.decode_plan(lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
-                          max_pages_per_seq=max_pages, num_sms=num_sms, num_splits=splits)
+                          max_pages_per_seq=max_pages, num_sms=num_sms, num_splits=splits,
+                          kv_dtype=kv_dtype, kernel=kernel)
 
 
 def _splits(L, chunk):
@@ -121,11 +123,43 @@ def test_plan_is_deterministic(lib):
 
 
 def test_plan_heads_per_cta(lib):
+    cc = dict(kernel="cuda_cores")
     assert _plan([100], hq=32, hkv=8).info.heads_per_cta == 4
     assert _plan([100], hq=32, hkv=32).info.heads_per_cta == 1
-    assert _plan([100], hq=32, hkv=2).info.heads_per_cta == 8     # 16 per kv head -> 2 CTAs
+    assert _plan([100], hq=32, hkv=2, **cc).info.heads_per_cta == 8     # 16 per kv head -> 2 CTAs
     assert _plan([100], hq=12, hkv=4).info.heads_per_cta == 1     # group 3
     assert _plan([100], hq=12, hkv=2).info.heads_per_cta == 2     # group 6
+
+
+def test_plan_kernel_choice(lib):
+    """Tensor cores for an E4M3 cache or a group of 8..16 heads at d = 128."""
+    p = _plan([100], hq=32, hkv=8)
+    assert p.info.tensor_cores == 0 and p.info.kv_dtype == fa.FA_KV_BF16
+    p = _plan([100], hq=32, hkv=8, kv_dtype="e4m3")
+    assert p.info.tensor_cores == 1 and p.info.kv_dtype == fa.FA_KV_E4M3 and p.info.heads_per_cta == 4
+    p = _plan([100], hq=32, hkv=2)
+    assert p.info.tensor_cores == 1 and p.info.heads_per_cta == 16
+    assert _plan([100], hq=64, hkv=2).info.tensor_cores == 0                 # group 32
+    assert _plan([100], hq=16, hkv=2, d=64).info.tensor_cores == 0           # d = 64
+    assert _plan([100], hq=32, hkv=8, kernel="tensor_cores").info.tensor_cores == 1
+    assert _plan([100], hq=32, hkv=8, kv_dtype="e4m3", kernel="cuda_cores").info.tensor_cores == 0
+    with pytest.raises(fa.FAError) as e:
+        _plan([100], hq=64, hkv=2, kernel="tensor_cores")
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+def test_plan_dtype_must_match_entry_point(lib):
+    A = 0x10000
+    p = _plan([1000, 3000], hq=8, hkv=2, kv_dtype="bf16")
+    st = lib.fa_decode_paged_fp8(_fake(A), _fake(A), _fake(A), 100, 64 * 2 * 128, 2 * 128, 128,
+                                 _fake(A), _fake(A), p.handle, float("nan"), 1.0, 1.0, _fake(A), None,
+                                 _fake(A), p.workspace_bytes, None)
+    assert st == fa.FA_ERR_PLAN_MISMATCH
+    p8 = _plan([1000, 3000], hq=8, hkv=2, kv_dtype="e4m3")
+    st = lib.fa_decode_paged(_fake(A), _fake(A), _fake(A), 100, 64 * 2 * 128, 2 * 128, 128,
+                             _fake(A), _fake(A), p8.handle, float("nan"), _fake(A), None,
+                             _fake(A), p8.workspace_bytes, None)
+    assert st == fa.FA_ERR_PLAN_MISMATCH
 
 
 def test_plan_rejects_cache_overflow(lib):
@@ -256,7 +290,7 @@ def test_append_validation_before_any_cuda_call(lib):
 
 
 def test_decode_fp8_validation_before_any_cuda_call(lib):
-    p = _plan([1000, 3000], hq=8, hkv=2, splits=4)
+    p = _plan([1000, 3000], hq=8, hkv=2, splits=4, kv_dtype="e4m3")
     A = 0x10000
 
     def call(strides=(64 * 2 * 128, 2 * 128, 128), ks=0.5, vs=0.5):
@@ -269,3 +303,9 @@ def test_decode_fp8_validation_before_any_cuda_call(lib):
     assert call(vs=float("nan")) == fa.FA_ERR_INVALID_ARG
     # byte strides must be multiples of 16 (8 is fine for bf16 elements, not for bytes)
     assert call(strides=(64 * 2 * 128, 2 * 128, 8)) == fa.FA_ERR_INVALID_ARG
+
+
+def test_build_tracks_every_source_file():
+    """Every file under csrc/ is a build input, so editing any of them rebuilds."""
+    csrc = os.path.join(ROOT, "exact_attention_148_b200", "csrc")
+    assert sorted(os.listdir(csrc)) == sorted(_build.SOURCES + _build.HEADERS)
