@@ -43,7 +43,8 @@ SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill"}
 DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode",
-                    "paged_decode_batch16", "paged_decode_batch_fp8"}
+                    "paged_decode_batch16", "paged_decode_batch_fp8", "paged_decode_gqa8",
+                    "paged_decode_gqa16"}
 CHUNKED_WORKLOADS = {"chunked_prefill_batch", "tiny_chunked_prefill"}
 
 
@@ -510,14 +511,25 @@ def oracle_chunked_sample(inp: W.ChunkedPrefillInputs, budget_s: float):
 
 # ----------------------------------------------------------------------------- main
 
-def build_cases(workload, device, num_splits, kernel="auto"):
+def decode_inputs(workload, heads=None):
+    """A decode workload, optionally with its query / kv head counts replaced
+    (same cache lengths, seeded draws): heads = "HQ:HKV"."""
+    inp = W.CONFIGS[workload]()
+    if heads:
+        hq, hkv = (int(x) for x in heads.split(":"))
+        inp = W.make_decode(inp.cache_seqlens, hq, hkv, inp.head_dim, seed=hq * 1000 + hkv,
+                            name=f"{workload}_h{hq}x{hkv}")
+    return inp
+
+
+def build_cases(workload, device, num_splits, kernel="auto", heads=None):
     if workload == "default":
         return [PrefillCase(W.varlen_causal_prefill(), device),
                 DecodeCase(W.paged_decode_batch(), device, 0, kernel)]
     if workload in PREFILL_WORKLOADS:
         return [PrefillCase(W.CONFIGS[workload](), device)]
     if workload in DECODE_WORKLOADS:
-        return [DecodeCase(W.CONFIGS[workload](), device, num_splits, kernel)]
+        return [DecodeCase(decode_inputs(workload, heads), device, num_splits, kernel)]
     if workload in CHUNKED_WORKLOADS:
         st = ChunkedState(W.CONFIGS[workload](), device)
         return [AppendCase(st), ChunkedAttnCase(st)]
@@ -592,7 +604,7 @@ def run_ours(args):
     device = torch.device("cuda", dist_ctx.local if dist_ctx else 0)
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
-    cases = build_cases(args.workload, device, args.num_splits, args.decode_kernel)
+    cases = build_cases(args.workload, device, args.num_splits, args.decode_kernel, args.decode_heads)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -769,6 +781,7 @@ def main():
                                                           CHUNKED_WORKLOADS)))
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--decode-kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
+    ap.add_argument("--decode-heads", default=None, help="HQ:HKV override for a decode workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")

@@ -14,25 +14,30 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Decode-time model used to choose the split size (measured on B200, 148 SMs):
-// all resident split CTAs share the HBM bandwidth, one CTA alone cannot pull
-// more than its ring depth allows (~44 GB/s for the CUDA-core kernel's three
-// 32 KB stages; the tensor-core kernel keeps 192 KB (bf16) or 96 KB (E4M3) in
-// flight), each CTA costs ~0.5 us of fill, and a second (merge) launch costs
-// ~5 us.
+// Decode-time model used to choose the split size (fitted to B200 timings,
+// 148 SMs): all resident split CTAs share the HBM bandwidth, one CTA alone
+// cannot pull more than its ceiling, each CTA costs a fixed fill/drain time,
+// and a second (merge) launch costs ~5 us.  Per kernel (CTA ceiling, fill,
+// CTAs per SM): CUDA cores 44 GB/s, 0.5 us, 2 (1 with 8 packed heads; its
+// E4M3 ring holds as many bytes as the bf16 one); tensor cores, bf16 50 GB/s,
+// 3 us (10 us with 16 padded heads), 1 (192 KB ring); tensor cores, E4M3
+// 30 GB/s, 2 us (7 us with 16 padded heads), 2.
 constexpr double kHbmBytesPerUs148 = 6.9e6;       // bytes per microsecond, 148 SMs
-constexpr double kCtaOverheadUs = 0.5;
 constexpr double kMergeLaunchUs = 5.0;
 
 struct CtaModel {
   double bytes_per_us;   // one CTA's ceiling
+  double overhead_us;    // fill and drain of one CTA
   int ctas_per_sm;
 };
 
 CtaModel cta_model(bool tensor_cores, int kv_elem_bytes, int heads_per_cta) {
-  // (the CUDA-core kernel's E4M3 ring holds as many bytes as its bf16 one)
-  if (tensor_cores) return {kv_elem_bytes == 1 ? 7.0e4 : 1.4e5, kv_elem_bytes == 1 ? 2 : 1};
-  return {4.36e4, heads_per_cta == 8 ? 1 : 2};
+  if (tensor_cores) {
+    const bool wide = heads_per_cta > 8;   // 16 padded heads
+    return kv_elem_bytes == 1 ? CtaModel{3.0e4, wide ? 7.0 : 2.0, 2}
+                              : CtaModel{5.0e4, wide ? 10.0 : 3.0, 1};
+  }
+  return {4.36e4, 0.5, heads_per_cta == 8 ? 1 : 2};
 }
 
 // Estimated duration (us) of the split kernel (+ merge) for one chunk size:
@@ -42,10 +47,11 @@ CtaModel cta_model(bool tensor_cores, int kv_elem_bytes, int heads_per_cta) {
 // points measured in "bytes done by every running CTA" (all running CTAs
 // advance at the same rate, so that scale is shared).
 double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64_t chunk, int slots,
-                          int head_dim, int kv_elem_bytes, double cta_bytes_per_us, int num_sms) {
+                          int head_dim, int kv_elem_bytes, const CtaModel& cm, int num_sms) {
   const double bytes_per_token = 2.0 * head_dim * kv_elem_bytes;   // K and V rows of one kv head
   const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
-  const double overhead_bytes = kCtaOverheadUs * cta_bytes_per_us;
+  const double cta_bytes_per_us = cm.bytes_per_us;
+  const double overhead_bytes = cm.overhead_us * cta_bytes_per_us;
   std::priority_queue<double, std::vector<double>, std::greater<double>> running;
   double v = 0.0, t = 0.0;
   size_t b = 0;
@@ -117,9 +123,10 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
   const bool tc_ok = head_dim == 128 && pl.group <= kTensorCoreMaxGroup;
   if (kernel == kDecodeKernelTensorCores && !tc_ok) return FA_ERR_UNSUPPORTED;
   // Tensor cores by default for an E4M3 cache (the CUDA-core loop spends an
-  // integer widening and G FMAs on every byte) and for groups of 8 or more.
+  // integer widening and G FMAs on every byte) and for groups of 4 or more
+  // (measured on B200: CUDA cores ahead at G = 1 and 2, tensor cores from 4).
   pl.tensor_cores = kernel == kDecodeKernelTensorCores ||
-                    (kernel == kDecodeKernelAuto && tc_ok && (kv_elem_bytes == 1 || pl.group >= 8));
+                    (kernel == kDecodeKernelAuto && tc_ok && (kv_elem_bytes == 1 || pl.group >= 4));
   if (pl.tensor_cores) {
     pl.heads_per_cta = pl.group;
   } else {
@@ -166,8 +173,8 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     for (int64_t c : cands) {
       c = std::max<int64_t>(c, kMinChunkTokens);
       if (ceil_div(max_len, c) > kMaxSplits) continue;
-      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes,
-                                          cm.bytes_per_us, num_sms);
+      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes, cm,
+                                          num_sms);
       if (chunk == 0 || t < best_t * (1.0 - 1e-9) || (t <= best_t * (1.0 + 1e-9) && c > chunk)) {
         best_t = t;
         chunk = c;

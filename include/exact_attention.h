@@ -194,7 +194,7 @@ int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads
  * kernel.  kv_dtype: FA_KV_BF16 (plans for fa_decode_paged) or FA_KV_E4M3
  * (plans for fa_decode_paged_fp8; a plan is only accepted by the entry point
  * of its type, else FA_ERR_PLAN_MISMATCH).  kernel: FA_DECODE_AUTO picks the
- * tensor-core kernel for an E4M3 cache or a group of 8 or more heads when
+ * tensor-core kernel for an E4M3 cache or a group of 4 or more heads when
  * d = 128 and Hq/Hkv <= 16; FA_DECODE_TENSOR_CORES outside that range is
  * FA_ERR_UNSUPPORTED.  fa_decode_plan(...) is
  * fa_decode_plan_kv(..., FA_KV_BF16, FA_DECODE_AUTO, ...).

@@ -128,20 +128,23 @@ def test_plan_heads_per_cta(lib):
     assert _plan([100], hq=32, hkv=32).info.heads_per_cta == 1
     assert _plan([100], hq=32, hkv=2, **cc).info.heads_per_cta == 8     # 16 per kv head -> 2 CTAs
     assert _plan([100], hq=12, hkv=4).info.heads_per_cta == 1     # group 3
-    assert _plan([100], hq=12, hkv=2).info.heads_per_cta == 2     # group 6
+    assert _plan([100], hq=12, hkv=2, **cc).info.heads_per_cta == 2     # group 6
+    assert _plan([100], hq=12, hkv=2).info.heads_per_cta == 6     # tensor cores: whole group
 
 
 def test_plan_kernel_choice(lib):
-    """Tensor cores for an E4M3 cache or a group of 8..16 heads at d = 128."""
+    """Tensor cores for an E4M3 cache or a group of 4..16 heads at d = 128."""
     p = _plan([100], hq=32, hkv=8)
-    assert p.info.tensor_cores == 0 and p.info.kv_dtype == fa.FA_KV_BF16
+    assert p.info.tensor_cores == 1 and p.info.kv_dtype == fa.FA_KV_BF16
+    assert _plan([100], hq=32, hkv=16).info.tensor_cores == 0               # group 2
+    assert _plan([100], hq=32, hkv=32).info.tensor_cores == 0               # group 1
     p = _plan([100], hq=32, hkv=8, kv_dtype="e4m3")
     assert p.info.tensor_cores == 1 and p.info.kv_dtype == fa.FA_KV_E4M3 and p.info.heads_per_cta == 4
     p = _plan([100], hq=32, hkv=2)
     assert p.info.tensor_cores == 1 and p.info.heads_per_cta == 16
     assert _plan([100], hq=64, hkv=2).info.tensor_cores == 0                 # group 32
     assert _plan([100], hq=16, hkv=2, d=64).info.tensor_cores == 0           # d = 64
-    assert _plan([100], hq=32, hkv=8, kernel="tensor_cores").info.tensor_cores == 1
+    assert _plan([100], hq=32, hkv=16, kernel="tensor_cores").info.tensor_cores == 1
     assert _plan([100], hq=32, hkv=8, kv_dtype="e4m3", kernel="cuda_cores").info.tensor_cores == 0
     with pytest.raises(fa.FAError) as e:
         _plan([100], hq=64, hkv=2, kernel="tensor_cores")

@@ -275,6 +275,18 @@ def paged_decode_batch() -> DecodeInputs:
     return make_decode(lens, 32, 8, 128, seed=3, name="paged_decode_batch")
 
 
+def paged_decode_gqa8() -> DecodeInputs:
+    """paged_decode_batch's lengths with 64 query heads over 8 kv heads (group 8)."""
+    lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=64)
+    return make_decode(lens, 64, 8, 128, seed=8, name="paged_decode_gqa8")
+
+
+def paged_decode_gqa16() -> DecodeInputs:
+    """paged_decode_batch's lengths with 32 query heads over 2 kv heads (group 16)."""
+    lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=64)
+    return make_decode(lens, 32, 2, 128, seed=16, name="paged_decode_gqa16")
+
+
 def paged_decode_batch16_lengths() -> np.ndarray:
     return np.random.default_rng(3).integers(1024, 32768 + 1, size=16)
 
@@ -556,6 +568,8 @@ CONFIGS = {
     "long_split_decode": long_split_decode,
     "ragged_split_decode": ragged_split_decode,
     "paged_decode_batch_fp8": paged_decode_batch_fp8,
+    "paged_decode_gqa8": paged_decode_gqa8,
+    "paged_decode_gqa16": paged_decode_gqa16,
     "tiny_chunked_prefill": tiny_chunked_prefill,
     "chunked_prefill_batch": chunked_prefill_batch,
 }
