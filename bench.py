@@ -539,7 +539,7 @@ def build_cases(workload, device, num_splits, kernel="auto", heads=None):
 def kernel_source_hash(kind):
     import hashlib
     files = {"prefill": ["ptx_sm100.cuh", "prefill_pp_sm100.cuh"],
-             "decode": ["ptx_sm100.cuh", "decode_sm100.cuh"],
+             "decode": ["ptx_sm100.cuh", "decode_sm100.cuh", "decode_tc_sm100.cuh"],
              "append": ["ptx_sm100.cuh", "append_sm100.cuh"]}[kind]
     m = hashlib.sha256()
     for f in files:
