@@ -539,7 +539,8 @@ def build_cases(workload, device, num_splits, kernel="auto", heads=None):
 def kernel_source_hash(kind):
     import hashlib
     files = {"prefill": ["ptx_sm100.cuh", "prefill_pp_sm100.cuh"],
-             "decode": ["ptx_sm100.cuh", "decode_sm100.cuh", "decode_tc_sm100.cuh"],
+             "decode": ["ptx_sm100.cuh", "decode_sm100.cuh"],
+             "decode_tc": ["ptx_sm100.cuh", "decode_sm100.cuh", "decode_tc_sm100.cuh"],
              "append": ["ptx_sm100.cuh", "append_sm100.cuh"]}[kind]
     m = hashlib.sha256()
     for f in files:
@@ -561,13 +562,14 @@ def measured_traffic(kind, workload, case=None):
     rows = {}
     for ln in lines:
         parts = [x.strip() for x in ln.strip().strip("|").split("|")]
-        if len(parts) >= 5 and parts[0] in ("prefill", "decode", "append") and parts[3].isdigit():
+        if len(parts) >= 5 and parts[0] in ("prefill", "decode", "decode_tc", "append") and parts[3].isdigit():
             rows[(parts[0], parts[1])] = (parts[2], int(parts[3]) + int(parts[4]))
     sha = kernel_source_hash(kind)
     if (kind, workload) in rows and rows[(kind, workload)][0] == sha:
         return rows[(kind, workload)][1]
-    if kind == "decode" and workload == "paged_decode_batch" and ("decode", "paged_decode_batch16") in rows:
-        h, t16 = rows[("decode", "paged_decode_batch16")]
+    if kind in ("decode", "decode_tc") and workload == "paged_decode_batch" and \
+            (kind, "paged_decode_batch16") in rows:
+        h, t16 = rows[(kind, "paged_decode_batch16")]
         if h == sha and case is not None:
             kv16 = 2.0 * float(np.sum(W.paged_decode_batch16_lengths())) * 8 * 128 * 2
             return int(t16 * case.inp.kv_bytes() / kv16)
@@ -641,7 +643,8 @@ def run_ours(args):
             e["kernel"] = "fa_append_kv_kernel<%d>" % c.inp.head_dim
         else:
             e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
-                               measured_traffic("decode", c.inp.name, c))
+                               measured_traffic("decode_tc" if c.plan.info.tensor_cores else "decode",
+                                                c.inp.name, c))
             e["kernel"] = ("fa_decode_tc_kernel" if c.plan.info.tensor_cores else "fa_decode_split_kernel") + \
                 ("<e4m3>" if c.fp8 else "") + " + fa_merge_kernel (one decode call)"
         e["workload"] = c.inp.name
