@@ -44,7 +44,7 @@ SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill"}
 DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode",
                     "paged_decode_batch16", "paged_decode_batch_fp8", "paged_decode_gqa8",
-                    "paged_decode_gqa16"}
+                    "paged_decode_gqa16", "speculative_decode_batch"}
 CHUNKED_WORKLOADS = {"chunked_prefill_batch", "tiny_chunked_prefill"}
 
 
@@ -190,11 +190,11 @@ class DecodeCase:
                                    num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
                                    page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
                                    num_splits=num_splits, kv_dtype="e4m3" if self.fp8 else "bf16",
-                                   kernel=kernel)
+                                   kernel=kernel, q_len=inp.q_len)
         self.plan_ms = (time.perf_counter() - t0) * 1e3
         self.ws = torch.empty(max(self.plan.workspace_bytes, 256), dtype=torch.uint8, device=device)
         self.out = torch.empty_like(self.q)
-        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=device)
+        self.lse = torch.empty(self.q.shape[:-1], dtype=torch.float32, device=device)
         self.bytes = inp.algorithmic_bytes()
         self.launches = 1 + (1 if self.plan.info.max_splits > 1 else 0)
         self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
@@ -239,7 +239,8 @@ class DecodeCase:
     def describe(self):
         i = self.inp
         info = self.plan.info
-        return {"workload": i.name, "batch": i.batch, "cache_tokens_total": int(i.cache_seqlens.sum()),
+        return {"workload": i.name, "batch": i.batch, "q_len": i.q_len,
+                "cache_tokens_total": int(i.cache_seqlens.sum()),
                 "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads, "head_dim": i.head_dim,
                 "page_size": i.page_size, "layout": i.layout,
                 "kv_dtype": "e4m3 (per-tensor scales)" if self.fp8 else "bf16",
@@ -466,12 +467,22 @@ def oracle_decode_sample(inp: W.DecodeInputs, budget_s: float):
         ks, vs = inp.extra["k_scale"], inp.extra["v_scale"]
         conv = dict(k_to_f64=lambda a: oracle.dequantize_e4m3(a, ks),
                     v_to_f64=lambda a: oracle.dequantize_e4m3(a, vs))
+    QL = inp.q_len
     for b in range(inp.batch):
-        rws = [(b, h) for h in range(0, inp.num_q_heads, G)][:2]   # two kv heads' first q head
+        heads = list(range(0, inp.num_q_heads, G))[:2]              # two kv heads' first q head
         t0 = time.perf_counter()
-        oracle.paged_decode_rows_ref(inp.q_bits, inp.k_pages_bits, inp.v_pages_bits, inp.block_table,
-                                     inp.cache_seqlens, inp.scale, rws, inp.page_size, inp.layout,
-                                     to_f64=W.as_f64, **conv)
+        if QL == 1:
+            oracle.paged_decode_rows_ref(inp.q_bits, inp.k_pages_bits, inp.v_pages_bits,
+                                         inp.block_table, inp.cache_seqlens, inp.scale,
+                                         [(b, h) for h in heads], inp.page_size, inp.layout,
+                                         to_f64=W.as_f64, **conv)
+        else:   # multi-token decode: the chunked-prefill oracle on the packed tokens
+            qp = inp.q_bits.reshape(inp.batch * QL, inp.num_q_heads, inp.head_dim)
+            cu = np.arange(inp.batch + 1) * QL
+            oracle.paged_prefill_rows_ref(qp, cu, inp.k_pages_bits, inp.v_pages_bits, inp.block_table,
+                                          inp.cache_seqlens, True, inp.scale,
+                                          [(b * QL + t, h) for h in heads for t in range(QL)],
+                                          inp.page_size, inp.layout, to_f64=W.as_f64)
         secs += time.perf_counter() - t0
         flops_bytes += len(rws) * 2.0 * int(inp.cache_seqlens[b]) * inp.head_dim * inp.kv_elem_bytes
         rows.append(b)

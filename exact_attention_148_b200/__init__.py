@@ -39,7 +39,7 @@ EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
-    "fa_decode_paged_fp8", "fa_decode_plan_kv",
+    "fa_decode_paged_fp8", "fa_decode_plan_kv", "fa_decode_plan_ex",
 ]
 
 FA_KV_BF16, FA_KV_E4M3 = 0, 1
@@ -68,8 +68,12 @@ class _PlanInfo(ctypes.Structure):
         ("chunk_tokens", ctypes.c_int), ("max_splits", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
         ("num_work_items", ctypes.c_int), ("max_seqlen", ctypes.c_int),
         ("workspace_bytes", ctypes.c_size_t), ("kv_dtype", ctypes.c_int),
-        ("tensor_cores", ctypes.c_int),
+        ("tensor_cores", ctypes.c_int), ("q_len", ctypes.c_int),
     ]
+
+
+class _DecodeOptions(ctypes.Structure):
+    _fields_ = [("kv_dtype", ctypes.c_int), ("kernel", ctypes.c_int), ("q_len", ctypes.c_int)]
 
 
 _lib = None
@@ -93,6 +97,10 @@ def library() -> ctypes.CDLL:
     L.fa_decode_plan_kv.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, i32,
                                     ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t)]
     L.fa_decode_plan_kv.restype = i32
+    L.fa_decode_plan_ex.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                    ctypes.POINTER(_DecodeOptions), ctypes.POINTER(vp),
+                                    ctypes.POINTER(ctypes.c_size_t)]
+    L.fa_decode_plan_ex.restype = i32
     L.fa_plan_get_info.argtypes = [vp, ctypes.POINTER(_PlanInfo)]
     L.fa_plan_get_info.restype = i32
     L.fa_plan_free.argtypes = [vp]
@@ -216,6 +224,7 @@ class PlanInfo:
     workspace_bytes: int
     kv_dtype: int
     tensor_cores: int
+    q_len: int
 
 
 class DecodePlan:
@@ -246,22 +255,23 @@ class DecodePlan:
 
 def decode_plan(cache_seqlens_host, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
                 page_size: int = 64, max_pages_per_seq: int, num_sms: int | None = None,
-                num_splits: int = 0, kv_dtype: str = "bf16", kernel: str = "auto") -> DecodePlan:
+                num_splits: int = 0, kv_dtype: str = "bf16", kernel: str = "auto",
+                q_len: int = 1) -> DecodePlan:
     """Plan the split of every request's cached context (host only, no GPU needed
     when ``num_sms`` is given).  ``kv_dtype``: "bf16" (for decode_paged) or
     "e4m3" (for decode_paged_fp8); ``kernel``: "auto", "cuda_cores" or
-    "tensor_cores"."""
+    "tensor_cores"; ``q_len`` > 1: multi-token decode (q [B, q_len, Hq, d])."""
     lens = np.ascontiguousarray(np.asarray(cache_seqlens_host, dtype=np.int32))
     if num_sms is None:
         torch = _torch()
         num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     h = ctypes.c_void_p()
     ws = ctypes.c_size_t()
-    st = library().fa_decode_plan_kv(lens.ctypes.data_as(ctypes.c_void_p), len(lens), num_q_heads,
+    opts = _DecodeOptions(_KV_DTYPES[kv_dtype], _KERNELS[kernel], int(q_len))
+    st = library().fa_decode_plan_ex(lens.ctypes.data_as(ctypes.c_void_p), len(lens), num_q_heads,
                                      num_kv_heads, head_dim, page_size, max_pages_per_seq, num_sms,
-                                     num_splits, _KV_DTYPES[kv_dtype], _KERNELS[kernel],
-                                     ctypes.byref(h), ctypes.byref(ws))
-    _check(st, "fa_decode_plan_kv")
+                                     num_splits, ctypes.byref(opts), ctypes.byref(h), ctypes.byref(ws))
+    _check(st, "fa_decode_plan_ex")
     return DecodePlan(h, ws.value)
 
 
@@ -273,6 +283,15 @@ def page_strides(k_pages, layout: str):
     if layout == "HND":     # [P, Hkv, page, d]
         return a * b * d, d, b * d
     raise ValueError(layout)
+
+
+def _check_q_rows(q, plan: DecodePlan):
+    """q is [B, Hq, d], or [B, q_len, Hq, d] for a multi-token plan."""
+    i = plan.info
+    want = (i.batch, i.num_q_heads, i.head_dim) if i.q_len == 1 and q.dim() == 3 else \
+        (i.batch, i.q_len, i.num_q_heads, i.head_dim)
+    if tuple(q.shape) != want:
+        raise ValueError(f"q has shape {tuple(q.shape)}, the plan expects {want}")
 
 
 def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePlan, *,
@@ -293,12 +312,12 @@ def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, plan: DecodePl
         raise ValueError("tensors must be contiguous")
     if k_pages.shape != v_pages.shape:
         raise ValueError("k_pages and v_pages must have the same shape")
-    B, Hq, d = q.shape
+    _check_q_rows(q, plan)
     ps, ts, hs = page_strides(k_pages, layout)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     if workspace is None and plan.workspace_bytes > 0:
         workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
     st = library().fa_decode_paged(
@@ -327,12 +346,12 @@ def decode_paged_fp8(q, k_pages, v_pages, block_table, cache_seqlens, plan: Deco
         raise ValueError("tensors must be contiguous")
     if k_pages.shape != v_pages.shape:
         raise ValueError("k_pages and v_pages must have the same shape")
-    B, Hq, d = q.shape
+    _check_q_rows(q, plan)
     ps, ts, hs = page_strides(k_pages, layout)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     if workspace is None and plan.workspace_bytes > 0:
         workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=q.device)
     st = library().fa_decode_paged_fp8(
@@ -354,12 +373,12 @@ def decode_paged_static(q, k_pages, v_pages, block_table, cache_seqlens, plan: D
     Pass preallocated ``out`` (and ``lse``) to keep the call allocation-free."""
     torch = _torch()
     _require_cuda(q, k_pages, v_pages, block_table, cache_seqlens, out, lse)
-    B, Hq, d = q.shape
+    _check_q_rows(q, plan)
     ps, ts, hs = page_strides(k_pages, layout)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     st = library().fa_decode_paged_static(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(block_table),
         _ptr(cache_seqlens), plan.handle, _scale_arg(scale), _ptr(out), _ptr(lse), _stream_ptr(stream))

@@ -48,15 +48,16 @@ constexpr int kDecodeThreads = 160;
 struct DecodeParams {
   CUtensorMap tm_k;   // 4-D over the page pool, dims sorted by stride: {d, ., ., .}
   CUtensorMap tm_v;
-  CUtensorMap tm_q;   // tensor-core kernel, bf16: 3-D {d, Hq, B}, box {64, NPAD, 1}
-  const __nv_bfloat16* q;        // [B, Hq, d]
+  CUtensorMap tm_q;   // tensor-core kernel, bf16: 4-D {d, Hq, q_len, B}, box {64, G, q_len, 1}
+  const __nv_bfloat16* q;        // [B, q_len, Hq, d]
   const int32_t* block_table;    // [B, max_pages]
   const int32_t* cache_seqlens;  // [B]
-  __nv_bfloat16* out;            // [B, Hq, d]
-  float* lse;                    // [B, Hq] or null
-  float* ws_o;                   // [max_splits, B, Hq, d]
-  float* ws_lse;                 // [max_splits, B, Hq]
+  __nv_bfloat16* out;            // [B, q_len, Hq, d]
+  float* lse;                    // [B, q_len, Hq] or null
+  float* ws_o;                   // [max_splits, B, q_len, Hq, d]
+  float* ws_lse;                 // [max_splits, B, q_len, Hq]
   int batch;
+  int q_len;                     // query tokens per request (1, or more on tensor cores)
   int num_q_heads;
   int group;                     // Hq / Hkv
   int subgroups;                 // group / GC
@@ -472,6 +473,7 @@ struct MergeParams {
   __nv_bfloat16* out;          // [rows, H, D]
   float* lse;                  // [rows, H] or null
   const int32_t* cache_seqlens;// null for a plain merge
+  int q_len;                   // rows per request (row r belongs to request r / q_len)
   int num_states;
   int rows;
   int num_heads;
@@ -488,7 +490,7 @@ __global__ void __launch_bounds__(128) fa_merge_kernel(const MergeParams p) {
   const int r = rh / p.num_heads;
   int ns = p.num_states;
   if (p.cache_seqlens != nullptr) {
-    int seqlen = p.cache_seqlens[r];
+    int seqlen = p.cache_seqlens[r / p.q_len];
     seqlen = max(0, min(seqlen, p.max_pages * kDecodePage));
     ns = min(p.num_states, (seqlen + p.chunk_tokens - 1) / p.chunk_tokens);
     if (ns <= 1) return;

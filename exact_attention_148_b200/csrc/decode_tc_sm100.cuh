@@ -9,8 +9,10 @@
 //   S^T (128 keys x N) = K_tile (128 x d) . Q^T (d x N)          SS, K-major
 //   O^T (d x N)       += V_tile^T (d x 128) . P^T (128 x N)      SS, A MN-major
 //
-// N = the G heads padded to NPAD (a multiple of 8, which an SS MMA with 128
-// rows accepts).  The CUDA cores then only run the online softmax: thread i
+// N = the q_len * G (token, head) rows of the request's queries padded to NPAD
+// (a multiple of 8, which an SS MMA with 128 rows accepts); with q_len > 1
+// (multi-token decode) token t of the chunk sees keys up to
+// cache_seqlens - q_len + t.  The CUDA cores then only run the online softmax: thread i
 // of the four softmax warps owns key i of the tile (TMEM lane i of S^T) and,
 // at the end, dimension i of O^T.  A K/V element is never touched by a CUDA
 // core, so the loop is bound by the TMA stream, not by per-element FMAs.
@@ -208,7 +210,9 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
   const int split = blockIdx.x;
   const int kv_head = blockIdx.y;
   const int b = blockIdx.z;
-  const int G = p.group;                       // real heads (<= NPAD)
+  const int G = p.group;                       // heads of the kv head
+  const int QL = p.q_len;                      // query tokens per request
+  const int R = QL * G;                        // real operand rows (<= NPAD): row = t * G + h
   const int qh0 = kv_head * G;
 
   int seqlen = p.cache_seqlens[b];
@@ -231,9 +235,12 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
   const int n_tiles = (num_pg + 1) / 2;
   const bool direct = (nsplit_eff == 1);
 
+  // Multi-token decode: the chunk's own tokens must be in the cache.
+  if (QL > 1 && seqlen < QL && split == 0 && threadIdx.x == 0) record_status(FA_ERR_PLAN_MISMATCH);
   if (n_tiles == 0) {   // empty cache: O = 0, LSE = -inf (only reachable with one split)
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-      const size_t row = static_cast<size_t>(b) * p.num_q_heads + qh0 + e / D;
+    for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
+      const int rr = e / D;
+      const size_t row = (static_cast<size_t>(b) * QL + rr / G) * p.num_q_heads + qh0 + rr % G;
       p.out[row * D + e % D] = __float2bfloat16_rn(0.0f);
       if (e % D == 0 && p.lse != nullptr) p.lse[row] = -INFINITY;
     }
@@ -283,11 +290,14 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
       if constexpr (!KV8) {
+        // R = q_len * G rows (token-major), 128 bytes each, per 64-column chunk;
+        // rows R..NPAD-1 of the operand are never read back (their S^T
+        // columns are masked and their P^T rows are zero).
         tma_prefetch_desc(&p.tm_q);
-        mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+        mbar_arrive_expect_tx(bar_q, C::CHUNKS * R * 128);
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(base + C::Q_OFF + c * NPAD * 128, &p.tm_q, bar_q, c * 64, qh0, b);
+          tma_load_4d(base + C::Q_OFF + c * NPAD * 128, &p.tm_q, bar_q, c * 64, qh0, 0, b);
       }
     }
     const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages + page_begin;
@@ -447,12 +457,12 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
     if constexpr (KV8) {
       // Q^T operand: heads h = quad, quad + 4, ...; lane holds d = 4 lane .. 4 lane + 3.
       uint8_t* qs = smem + C::Q_OFF;
-      for (int h = quad; h < NPAD; h += 4) {
+      for (int h = quad; h < NPAD; h += 4) {      // h = operand row t * G + head
         uint32_t hi = 0, lo = 0;
         float sq = 1.0f;
-        if (h < G) {
+        if (h < R) {
           const uint2 u = *reinterpret_cast<const uint2*>(
-              p.q + (static_cast<size_t>(b) * p.num_q_heads + qh0 + h) * D + 4 * lane);
+              p.q + ((static_cast<size_t>(b) * QL + h / G) * p.num_q_heads + qh0 + h % G) * D + 4 * lane);
           const float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
                               __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
           float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
@@ -488,11 +498,13 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
     }
     softmax_sync();
     float c[NPAD], m[NPAD], l[NPAD];
+    int lim[NPAD];                 // last visible key of each row (token t of the chunk)
 #pragma unroll
     for (int h = 0; h < NPAD; ++h) {
       c[h] = scl[h];
       m[h] = -INFINITY;
       l[h] = 0.0f;
+      lim[h] = h < R ? seqlen - QL + h / G : -1;
     }
 
     // Every softmax warp passes the named barrier once per tile and once in
@@ -507,12 +519,13 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         uint32_t sr[NB];
         tmem_ld_n<NB>(tmem + lane_base + static_cast<uint32_t>((j & 1) * NB), sr);
         tmem_ld_n_wait<NB>(sr);
-        const bool valid = t_begin + j * C::KEYS + r < t_end;
+        const int key = t_begin + j * C::KEYS + r;
+        const bool valid = key < t_end;
 #pragma unroll
         for (int h = 0; h < NPAD; ++h) {
           const float raw = KV8 ? __uint_as_float(sr[h]) + __uint_as_float(sr[NPAD + h])
                                 : __uint_as_float(sr[h]);
-          s[h] = (valid && h < G) ? raw * c[h] : -INFINITY;
+          s[h] = (valid && key <= lim[h]) ? raw * c[h] : -INFINITY;
         }
       } else {
 #pragma unroll
@@ -595,19 +608,19 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
       tmem_ld_n_wait<NB>(o);
 #pragma unroll
       for (int h = 0; h < NPAD; ++h) {
-        if (h >= G) continue;
+        if (h >= R) continue;
         const float4 w = *reinterpret_cast<const float4*>(lred + h * 4);
         const float lsum = (w.x + w.y) + (w.z + w.w);
         float ov = KV8 ? (__uint_as_float(o[h]) + __uint_as_float(o[NPAD + h])) * (p.v_scale * (1.0f / 256.0f))
                        : __uint_as_float(o[h]);
         ov = lsum > 0.0f ? ov / lsum : 0.0f;
         const float lse_v = (lsum > 0.0f) ? (m[h] + log2f(lsum)) * 0.69314718055994530942f : -INFINITY;
-        const size_t row = static_cast<size_t>(b) * p.num_q_heads + qh0 + h;
+        const size_t row = (static_cast<size_t>(b) * QL + h / G) * p.num_q_heads + qh0 + h % G;
         if (direct) {
           p.out[row * D + r] = __float2bfloat16_rn(ov);
           if (r == 0 && p.lse != nullptr) p.lse[row] = lse_v;
         } else {
-          const size_t srow = static_cast<size_t>(split) * p.batch * p.num_q_heads + row;
+          const size_t srow = static_cast<size_t>(split) * p.batch * QL * p.num_q_heads + row;
           p.ws_o[srow * D + r] = ov;
           if (r == 0) p.ws_lse[srow] = lse_v;
         }

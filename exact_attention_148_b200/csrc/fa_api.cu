@@ -423,17 +423,18 @@ FA_API int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_
   return FA_OK;
 }
 
-FA_API int fa_decode_plan_kv(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+FA_API int fa_decode_plan_ex(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
                              int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
-                             int num_sms, int num_splits_override, int kv_dtype, int kernel,
+                             int num_sms, int num_splits_override, const fa_decode_options* options,
                              fa_plan** plan_out, size_t* workspace_bytes) {
-  if (plan_out == nullptr) return FA_ERR_INVALID_ARG;
+  if (plan_out == nullptr || options == nullptr) return FA_ERR_INVALID_ARG;
   *plan_out = nullptr;
+  const int kv_dtype = options->kv_dtype;
   if (kv_dtype != FA_KV_BF16 && kv_dtype != FA_KV_E4M3) return FA_ERR_INVALID_ARG;
   fa::DecodePlan p;
   int st = fa::make_decode_plan(cache_seqlens_host, batch, num_q_heads, num_kv_heads, head_dim,
                                 page_size, max_pages_per_seq, num_sms, num_splits_override,
-                                kv_dtype == FA_KV_E4M3 ? 1 : 2, kernel, &p);
+                                kv_dtype == FA_KV_E4M3 ? 1 : 2, options->kernel, options->q_len, &p);
   if (st != FA_OK) return st;
   fa_plan* plan = new (std::nothrow) fa_plan;
   if (plan == nullptr) return FA_ERR_INVALID_ARG;
@@ -441,6 +442,16 @@ FA_API int fa_decode_plan_kv(const int32_t* cache_seqlens_host, int batch, int n
   *plan_out = plan;
   if (workspace_bytes) *workspace_bytes = plan->p.workspace_bytes;
   return FA_OK;
+}
+
+FA_API int fa_decode_plan_kv(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                             int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                             int num_sms, int num_splits_override, int kv_dtype, int kernel,
+                             fa_plan** plan_out, size_t* workspace_bytes) {
+  const fa_decode_options o = {kv_dtype, kernel, 1};
+  return fa_decode_plan_ex(cache_seqlens_host, batch, num_q_heads, num_kv_heads, head_dim, page_size,
+                           max_pages_per_seq, num_sms, num_splits_override, &o, plan_out,
+                           workspace_bytes);
 }
 
 FA_API int fa_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
@@ -469,6 +480,7 @@ FA_API int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info) {
   info->workspace_bytes = p.workspace_bytes;
   info->kv_dtype = p.kv_elem_bytes == 1 ? FA_KV_E4M3 : FA_KV_BF16;
   info->tensor_cores = p.tensor_cores ? 1 : 0;
+  info->q_len = p.q_len;
   return FA_OK;
 }
 
@@ -523,14 +535,18 @@ int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, i
                             pl.page_size, pl.num_kv_heads, pl.head_dim, box_cols, swz,
                             &prm.head_coord, &prm.page_coord, elem_bytes);
   if (st != FA_OK) return st;
-  const int npad = pl.group <= 8 ? 8 : 16;
+  const int npad = pl.q_len * pl.group <= 8 ? 8 : 16;
   if (pl.tensor_cores && !kv8) {
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(pl.head_dim),
-                                static_cast<cuuint64_t>(pl.num_q_heads), static_cast<cuuint64_t>(pl.batch)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pl.head_dim) * 2,
-                                   static_cast<cuuint64_t>(pl.num_q_heads) * pl.head_dim * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(npad), 1};
-    st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    // q [B, q_len, Hq, d]: a box is the G heads of one kv head for every token
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(pl.head_dim),
+                                static_cast<cuuint64_t>(pl.num_q_heads),
+                                static_cast<cuuint64_t>(pl.q_len), static_cast<cuuint64_t>(pl.batch)};
+    const cuuint64_t strides[3] = {
+        static_cast<cuuint64_t>(pl.head_dim) * 2,
+        static_cast<cuuint64_t>(pl.num_q_heads) * pl.head_dim * 2,
+        static_cast<cuuint64_t>(pl.q_len) * pl.num_q_heads * pl.head_dim * 2};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(pl.group), static_cast<cuuint32_t>(pl.q_len), 1};
+    st = encode_map(&prm.tm_q, q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
   }
 
@@ -545,6 +561,7 @@ int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, i
                    ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.ws_lse_offset)
                    : nullptr;
   prm.batch = pl.batch;
+  prm.q_len = pl.q_len;
   prm.num_q_heads = pl.num_q_heads;
   prm.group = pl.group;
   prm.subgroups = pl.subgroups;
@@ -576,8 +593,9 @@ int decode_paged_impl(const void* q, const void* k_pages, const void* v_pages, i
     mp.out = prm.out;
     mp.lse = lse;
     mp.cache_seqlens = cache_seqlens_dev;
+    mp.q_len = pl.q_len;
     mp.num_states = pl.max_splits;
-    mp.rows = pl.batch;
+    mp.rows = pl.batch * pl.q_len;
     mp.num_heads = pl.num_q_heads;
     mp.chunk_tokens = pl.chunk_tokens;
     mp.max_pages = pl.max_pages_per_seq;
@@ -623,6 +641,7 @@ FA_API int fa_merge_states(const float* o_parts, const float* lse_parts, int num
   mp.out = static_cast<__nv_bfloat16*>(out);
   mp.lse = lse;
   mp.cache_seqlens = nullptr;
+  mp.q_len = 1;
   mp.num_states = num_states;
   mp.rows = rows;
   mp.num_heads = num_heads;

@@ -97,8 +97,9 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
 int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
                      int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
                      int num_sms, int num_splits_override, int kv_elem_bytes, int kernel,
-                     DecodePlan* plan) {
+                     int q_len, DecodePlan* plan) {
   if (plan == nullptr || cache_seqlens_host == nullptr) return FA_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > kTensorCoreMaxGroup) return FA_ERR_INVALID_ARG;
   if (kv_elem_bytes != 1 && kv_elem_bytes != 2) return FA_ERR_INVALID_ARG;
   if (kernel < kDecodeKernelAuto || kernel > kDecodeKernelTensorCores) return FA_ERR_INVALID_ARG;
   if (batch < 1 || batch > 65535 || num_q_heads < 1 || num_kv_heads < 1 ||
@@ -120,12 +121,15 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
   pl.num_sms = num_sms;
   pl.group = num_q_heads / num_kv_heads;
   pl.kv_elem_bytes = kv_elem_bytes;
-  const bool tc_ok = head_dim == 128 && pl.group <= kTensorCoreMaxGroup;
-  if (kernel == kDecodeKernelTensorCores && !tc_ok) return FA_ERR_UNSUPPORTED;
+  pl.q_len = q_len;
+  const bool tc_ok = head_dim == 128 && q_len * pl.group <= kTensorCoreMaxGroup;
+  if ((kernel == kDecodeKernelTensorCores || q_len > 1) && !tc_ok) return FA_ERR_UNSUPPORTED;
+  if (q_len > 1 && kernel == kDecodeKernelCudaCores) return FA_ERR_UNSUPPORTED;
   // Tensor cores by default for an E4M3 cache (the CUDA-core loop spends an
   // integer widening and G FMAs on every byte) and for groups of 4 or more
   // (measured on B200: CUDA cores ahead at G = 1 and 2, tensor cores from 4).
-  pl.tensor_cores = kernel == kDecodeKernelTensorCores ||
+  // Several query tokens per request (multi-token decode) only run on tensor cores.
+  pl.tensor_cores = kernel == kDecodeKernelTensorCores || q_len > 1 ||
                     (kernel == kDecodeKernelAuto && tc_ok && (kv_elem_bytes == 1 || pl.group >= 4));
   if (pl.tensor_cores) {
     pl.heads_per_cta = pl.group;
@@ -146,6 +150,8 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     const int32_t L = pl.seqlens[b];
     // Cache-overflow check: a length the block table cannot address is an error.
     if (L < 0 || L > capacity) return FA_ERR_INVALID_ARG;
+    // The chunk's own tokens are in the cache already.
+    if (q_len > 1 && L < q_len) return FA_ERR_INVALID_ARG;
     total += L;
     max_len = std::max(max_len, static_cast<int>(L));
   }
@@ -161,7 +167,7 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     // Try split counts s (chunk = ceil(max_len / s) rounded to a page, at
     // least kMinChunkTokens keys) plus the many-small-items rule, and keep the
     // one the decode-time model estimates fastest (ties: fewer splits).
-    const CtaModel cm = cta_model(pl.tensor_cores, kv_elem_bytes, pl.heads_per_cta);
+    const CtaModel cm = cta_model(pl.tensor_cores, kv_elem_bytes, q_len * pl.heads_per_cta);
     const int slots = num_sms * cm.ctas_per_sm;
     std::vector<int64_t> cands;
     for (int s : {1, 2, 3, 4, 5, 6, 8, 10, 12, 16, 20, 24, 32, 48, 64, 96, 128})
@@ -192,7 +198,7 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
   pl.num_work_items = static_cast<int>(items * units);
 
   if (pl.max_splits > 1) {
-    const size_t rows = static_cast<size_t>(batch) * num_q_heads;
+    const size_t rows = static_cast<size_t>(batch) * q_len * num_q_heads;
     pl.ws_o_offset = 0;
     pl.ws_lse_offset = align256(static_cast<size_t>(pl.max_splits) * rows * head_dim * 4);
     pl.workspace_bytes = align256(pl.ws_lse_offset + static_cast<size_t>(pl.max_splits) * rows * 4);

@@ -22,6 +22,7 @@ struct DecodePlan {
   int page_size = 0, max_pages_per_seq = 0, num_sms = 0;
   int group = 1;          // Hq / Hkv
   int kv_elem_bytes = 2;  // 2 = bf16 cache, 1 = E4M3 cache
+  int q_len = 1;          // query tokens per request (multi-token decode on tensor cores)
   bool tensor_cores = false;  // tcgen05 split kernel (all G heads of a kv head per CTA)
   int heads_per_cta = 1;  // GC: G on tensor cores, else largest of 8, 4, 2, 1 dividing the group
   int subgroups = 1;      // group / GC
@@ -35,12 +36,12 @@ struct DecodePlan {
 
 // kernel: 0 = choose, 1 = CUDA-core split kernel, 2 = tensor-core split kernel.
 constexpr int kDecodeKernelAuto = 0, kDecodeKernelCudaCores = 1, kDecodeKernelTensorCores = 2;
-constexpr int kTensorCoreMaxGroup = 16;
+constexpr int kTensorCoreMaxGroup = 16;   // q_len * G operand rows per CTA
 
 // Returns an fa_status.  Pure host code (no CUDA calls).
 int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
                      int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
                      int num_sms, int num_splits_override, int kv_elem_bytes, int kernel,
-                     DecodePlan* plan);
+                     int q_len, DecodePlan* plan);
 
 }  // namespace fa

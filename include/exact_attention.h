@@ -81,7 +81,15 @@ typedef struct {
   size_t workspace_bytes;
   int kv_dtype;          /* fa_kv_dtype the plan was made for */
   int tensor_cores;      /* 1 if the plan runs the tensor-core split kernel */
+  int q_len;             /* query tokens per request */
 } fa_plan_info;
+
+/* Options of fa_decode_plan_ex. */
+typedef struct {
+  int kv_dtype;          /* fa_kv_dtype */
+  int kernel;            /* fa_decode_kernel */
+  int q_len;             /* query tokens per request, >= 1 (see fa_decode_plan_ex) */
+} fa_decode_options;
 
 /*
  * fa_prefill — causal or full exact attention over packed variable-length
@@ -204,6 +212,20 @@ int fa_decode_plan_kv(const int32_t* cache_seqlens_host, int batch, int num_q_he
                       int num_sms, int num_splits_override, int kv_dtype, int kernel,
                       fa_plan** plan_out, size_t* workspace_bytes);
 
+/*
+ * fa_decode_plan_ex — fa_decode_plan_kv plus multi-token decode.  With
+ * options->q_len = n > 1 each request brings n query tokens (e.g. speculative
+ * decoding) whose K/V are already the last n entries of its cache: q and out
+ * are [batch, n, Hq, d], lse [batch, n, Hq], and token t of request b sees
+ * cached keys 0 .. cache_seqlens[b] - n + t (the chunked-prefill mask).  Needs
+ * the tensor-core kernel: d = 128 and n * Hq/Hkv <= 16 (else
+ * FA_ERR_UNSUPPORTED); every planned length must be >= n.
+ */
+int fa_decode_plan_ex(const int32_t* cache_seqlens_host, int batch, int num_q_heads,
+                      int num_kv_heads, int head_dim, int page_size, int max_pages_per_seq,
+                      int num_sms, int num_splits_override, const fa_decode_options* options,
+                      fa_plan** plan_out, size_t* workspace_bytes);
+
 int fa_plan_get_info(const fa_plan* plan, fa_plan_info* info);
 void fa_plan_free(fa_plan* plan);
 
@@ -211,7 +233,8 @@ void fa_plan_free(fa_plan* plan);
  * fa_decode_paged — one query token per request against its paged KV cache
  * (the "run" stage; Flash-Decoding split kernel + LSE merge kernel).
  *
- *   q [batch, Hq, d] bf16.
+ *   q [batch, Hq, d] bf16 ([batch, q_len, Hq, d] with a multi-token plan,
+ *       fa_decode_plan_ex; out and lse then carry the q_len axis too).
  *   k_pages, v_pages: a pool of num_pages pages of page_size tokens; element
  *       (page p, slot t, kv head g, dim c) is at
  *       p*page_stride + t*token_stride + g*head_stride + c   (elements).

@@ -340,13 +340,18 @@ def _chunk_causal_mask(q_len: int, k_len: int) -> np.ndarray:
 
 def paged_prefill_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens,
                       causal: bool, scale=None, page_size: int = 64, layout: str = "NHD",
-                      to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+                      to_f64=lambda a: np.asarray(a, dtype=np.float64),
+                      k_to_f64=None, v_to_f64=None):
     """Chunked prefill: each request's new queries against its whole paged cache.
 
     q: [Tq, Hq, d] packed by ``cu_seqlens_q``; request b's cache holds
     cache_seqlens[b] >= q_len_b tokens (the chunk's own K/V included).
+    ``k_to_f64`` / ``v_to_f64`` replace ``to_f64`` for the gathered K and V
+    (as in ``paged_decode_rows_ref``).
     Returns (O [Tq, Hq, d], LSE [Tq, Hq]).
     """
+    k_conv = k_to_f64 if k_to_f64 is not None else to_f64
+    v_conv = v_to_f64 if v_to_f64 is not None else to_f64
     q = np.asarray(q)
     Tq, Hq, d = q.shape
     Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
@@ -362,7 +367,7 @@ def paged_prefill_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seql
             raise ValueError("cache length shorter than the chunk")
         for g in range(Hkv):
             K, V = gather_paged_kv(k_pages, v_pages, block_table[b], Lk, g, page_size, layout)
-            K, V = to_f64(K), to_f64(V)
+            K, V = k_conv(K), v_conv(V)
             for h in range(Hq):
                 if kv_head_of(h, Hq, Hkv) != g:
                     continue
@@ -377,11 +382,14 @@ def paged_prefill_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seql
 
 def paged_prefill_rows_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens,
                            causal: bool, scale, rows, page_size: int = 64, layout: str = "NHD",
-                           to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+                           to_f64=lambda a: np.asarray(a, dtype=np.float64),
+                           k_to_f64=None, v_to_f64=None):
     """Selected rows (token, q_head) of ``paged_prefill_ref``, each on its own.
 
     Returns (O [n, d], LSE [n]).
     """
+    k_conv = k_to_f64 if k_to_f64 is not None else to_f64
+    v_conv = v_to_f64 if v_to_f64 is not None else to_f64
     q = np.asarray(q)
     Tq, Hq, d = q.shape
     Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
@@ -399,7 +407,7 @@ def paged_prefill_rows_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache
         g = kv_head_of(h, Hq, Hkv)
         if (b, g) not in cache:
             K, V = gather_paged_kv(k_pages, v_pages, block_table[b], Lk, g, page_size, layout)
-            cache = {(b, g): (to_f64(K), to_f64(V))}
+            cache = {(b, g): (k_conv(K), v_conv(V))}
         K, V = cache[(b, g)]
         nk = visible_key_count(i, Lq, Lk, causal)
         P, l = _softmax_with_lse(_scores(to_f64(q[t, h])[None, :], K[:nk], scale))

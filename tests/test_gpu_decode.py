@@ -16,7 +16,10 @@ def oracle_rows(inp, rows):
 
 
 def check_all_rows(inp, num_splits=0, what="", kernel="auto"):
+    import exact_attention_148_b200 as fa
+    assert fa.device_status(clear=True) == 0
     out, lse, plan = decode_on_gpu(inp, num_splits, kernel=kernel)
+    assert fa.device_status(clear=True) == 0, what
     rows = [(b, h) for b in range(inp.batch) for h in range(inp.num_q_heads)]
     o_ref, l_ref = oracle_rows(inp, rows)
     compare(bf16_to_f64(out).reshape(-1, inp.head_dim), lse.cpu().numpy().reshape(-1), o_ref, l_ref,

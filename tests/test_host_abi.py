@@ -312,3 +312,29 @@ def test_build_tracks_every_source_file():
     """Every file under csrc/ is a build input, so editing any of them rebuilds."""
     csrc = os.path.join(ROOT, "exact_attention_148_b200", "csrc")
     assert sorted(os.listdir(csrc)) == sorted(_build.SOURCES + _build.HEADERS)
+
+
+def test_multi_token_plans(lib):
+    mk = lambda **kw: fa.decode_plan(np.array([100, 2000], dtype=np.int32), num_q_heads=kw.get("hq", 8),
+                                     num_kv_heads=kw.get("hkv", 2), head_dim=kw.get("d", 128),
+                                     max_pages_per_seq=40, num_sms=148, num_splits=kw.get("s", 0),
+                                     q_len=kw.get("q_len", 1), kernel=kw.get("kernel", "auto"),
+                                     kv_dtype=kw.get("kv", "bf16"))
+    p = mk(q_len=4)
+    assert p.info.q_len == 4 and p.info.tensor_cores == 1
+    p1 = mk(q_len=1, s=4, kernel="tensor_cores")
+    p4 = mk(q_len=4, s=4)
+    assert p4.workspace_bytes >= 4 * p1.workspace_bytes - 1024            # partials scale with q_len
+    assert mk(q_len=4, kv="e4m3").info.tensor_cores == 1
+    for kw, status in [(dict(q_len=3, hq=16, hkv=2), fa.FA_ERR_UNSUPPORTED),   # 24 rows > 16
+                       (dict(q_len=2, d=64), fa.FA_ERR_UNSUPPORTED),
+                       (dict(q_len=2, kernel="cuda_cores"), fa.FA_ERR_UNSUPPORTED),
+                       (dict(q_len=0), fa.FA_ERR_INVALID_ARG),
+                       (dict(q_len=17), fa.FA_ERR_INVALID_ARG)]:
+        with pytest.raises(fa.FAError) as e:
+            mk(**kw)
+        assert e.value.status == status, kw
+    with pytest.raises(fa.FAError) as e:      # a cache shorter than the chunk
+        fa.decode_plan(np.array([3, 2000], dtype=np.int32), num_q_heads=8, num_kv_heads=2,
+                       head_dim=128, max_pages_per_seq=40, num_sms=148, q_len=4)
+    assert e.value.status == fa.FA_ERR_INVALID_ARG

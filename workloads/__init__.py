@@ -175,7 +175,7 @@ def long_gqa_prefill() -> PrefillInputs:
 @dataclass
 class DecodeInputs:
     name: str
-    q_bits: np.ndarray            # [B, Hq, d]
+    q_bits: np.ndarray            # [B, Hq, d], or [B, q_len, Hq, d] for multi-token decode
     k_pages_bits: np.ndarray      # NHD: [P, page, Hkv, d]; HND: [P, Hkv, page, d]
     v_pages_bits: np.ndarray
     block_table: np.ndarray       # [B, max_pages] int32 (unused slots = -1)
@@ -190,12 +190,16 @@ class DecodeInputs:
         return self.q_bits.shape[0]
 
     @property
+    def q_len(self):
+        return self.q_bits.shape[1] if self.q_bits.ndim == 4 else 1
+
+    @property
     def num_q_heads(self):
-        return self.q_bits.shape[1]
+        return self.q_bits.shape[-2]
 
     @property
     def head_dim(self):
-        return self.q_bits.shape[2]
+        return self.q_bits.shape[-1]
 
     @property
     def num_kv_heads(self):
@@ -224,14 +228,15 @@ class DecodeInputs:
 
     def algorithmic_bytes(self) -> float:
         """KV read once + q read + out/lse written + block_table entries used."""
-        B, Hq, d = self.q_bits.shape
+        B, Hq, d = self.batch, self.num_q_heads, self.head_dim
+        rows = B * self.q_len * Hq
         pages_used = int(np.sum((self.cache_seqlens.astype(np.int64) + self.page_size - 1) // self.page_size))
-        return self.kv_bytes() + B * Hq * d * 2 * 2 + B * Hq * 4 + pages_used * 4 + B * 4
+        return self.kv_bytes() + rows * d * 2 * 2 + rows * 4 + pages_used * 4 + B * 4
 
 
 def make_decode(cache_seqlens, num_q_heads, num_kv_heads, head_dim, *, seed=3,
                 page_size=PAGE_SIZE, layout="NHD", scale=None, extra_pages=0,
-                name="decode") -> DecodeInputs:
+                name="decode", q_len=1) -> DecodeInputs:
     """Paged KV cache whose physical pages are a seeded random permutation.
 
     Request b owns ceil(seqlen_b / page_size) logical pages; the physical page
@@ -260,7 +265,8 @@ def make_decode(cache_seqlens, num_q_heads, num_kv_heads, head_dim, *, seed=3,
         shape = (total, num_kv_heads, page_size, head_dim)
     else:
         raise ValueError(layout)
-    q = _normal_bf16_bits(s_q, (B, num_q_heads, head_dim))
+    q_shape = (B, num_q_heads, head_dim) if q_len == 1 else (B, q_len, num_q_heads, head_dim)
+    q = _normal_bf16_bits(s_q, q_shape)
     kp = _normal_bf16_bits(s_k, shape)
     vp = _normal_bf16_bits(s_v, shape)
     if scale is None:
@@ -285,6 +291,13 @@ def paged_decode_gqa16() -> DecodeInputs:
     """paged_decode_batch's lengths with 32 query heads over 2 kv heads (group 16)."""
     lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=64)
     return make_decode(lens, 32, 2, 128, seed=16, name="paged_decode_gqa16")
+
+
+def speculative_decode_batch() -> DecodeInputs:
+    """paged_decode_batch's 64 requests with 4 query tokens each (multi-token
+    decode, e.g. speculative verification), 32 q / 8 kv heads, d=128."""
+    lens = np.random.default_rng(3).integers(1024, 32768 + 1, size=64)
+    return make_decode(lens, 32, 8, 128, seed=17, q_len=4, name="speculative_decode_batch")
 
 
 def paged_decode_batch16_lengths() -> np.ndarray:
@@ -570,6 +583,7 @@ CONFIGS = {
     "paged_decode_batch_fp8": paged_decode_batch_fp8,
     "paged_decode_gqa8": paged_decode_gqa8,
     "paged_decode_gqa16": paged_decode_gqa16,
+    "speculative_decode_batch": speculative_decode_batch,
     "tiny_chunked_prefill": tiny_chunked_prefill,
     "chunked_prefill_batch": chunked_prefill_batch,
 }
