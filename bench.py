@@ -46,6 +46,7 @@ DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_dec
                     "paged_decode_batch16", "paged_decode_batch_fp8", "paged_decode_gqa8",
                     "paged_decode_gqa16", "speculative_decode_batch"}
 CHUNKED_WORKLOADS = {"chunked_prefill_batch", "tiny_chunked_prefill"}
+CASCADE_WORKLOADS = {"cascade_decode_batch"}
 
 
 def load_peaks():
@@ -355,6 +356,62 @@ class ChunkedAttnCase:
                 "algorithmic_tflop": round(self.flops / 1e12, 4)}
 
 
+class CascadeCase:
+    """fa_cascade_decode: shared prefix read once for the batch + own suffixes."""
+
+    def __init__(self, inp: W.CascadeInputs, device, kernel="auto"):
+        import torch
+        import exact_attention_148_b200 as fa
+        self.inp = inp
+        self.q = _dev_bf16(inp.q_bits, device)
+        self.kp = _dev_bf16(inp.k_pages_bits, device)
+        self.vp = _dev_bf16(inp.v_pages_bits, device)
+        self.pre = _dev_i32(inp.prefix_block_table, device)
+        self.bt = _dev_i32(inp.block_table, device)
+        self.lens = _dev_i32(inp.suffix_lens, device)
+        self.plan = fa.decode_plan(inp.suffix_lens, num_q_heads=inp.num_q_heads,
+                                   num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
+                                   max_pages_per_seq=inp.block_table.shape[1], kernel=kernel)
+        self.ws = torch.empty(max(fa.cascade_workspace_bytes(self.plan, inp.prefix_len), 256),
+                              dtype=torch.uint8, device=device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:-1], dtype=torch.float32, device=device)
+        self.bytes = inp.algorithmic_bytes()
+        self.launches = 3 + (1 if self.plan.info.max_splits > 1 else 0)
+        self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
+        self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def run(self):
+        import exact_attention_148_b200 as fa
+        fa.cascade_decode(self.q, self.kp, self.vp, self.pre, self.inp.prefix_len, self.bt, self.lens,
+                          self.plan, layout=self.inp.layout, scale=self.inp.scale, out=self.out,
+                          lse=self.lse, workspace=self.ws)
+
+    def run_e2e(self):
+        """The step's input is the batch's query rows; the paged cache is resident."""
+        import torch
+        self.q.view(torch.int16).copy_(self.h_q, non_blocking=True)
+        self.run()
+        self.h_out.copy_(self.out.view(torch.int16), non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def h2d_bytes(self):
+        return 2 * self.inp.q_bits.size
+
+    def d2h_bytes(self):
+        return 2 * self.inp.q_bits.size + 4 * self.lse.numel()
+
+    def describe(self):
+        i = self.inp
+        return {"workload": i.name, "batch": i.batch, "prefix_len": i.prefix_len,
+                "suffix_tokens_total": int(i.suffix_lens.sum()), "num_q_heads": i.num_q_heads,
+                "num_kv_heads": i.num_kv_heads, "head_dim": i.head_dim,
+                "algorithmic_gb": round(self.bytes / 1e9, 4),
+                "suffix_split_kernel": "tensor cores (tcgen05)" if self.plan.info.tensor_cores
+                else "CUDA cores"}
+
+
 # ----------------------------------------------------------------------------- timing
 
 def time_cases(cases, steps, warmup, flush, dist_ctx, e2e=False):
@@ -520,6 +577,25 @@ def oracle_chunked_sample(inp: W.ChunkedPrefillInputs, budget_s: float):
                          f"(prefix, chunk) = {done}")
 
 
+def oracle_cascade_sample(inp: W.CascadeInputs, budget_s: float):
+    """The oracle's cascade decode, one request at a time, until about budget_s;
+    work is counted in the cascade's own algorithmic bytes per request."""
+    import oracle
+    secs, done = 0.0, []
+    per_req = inp.algorithmic_bytes() / inp.batch
+    for b in range(inp.batch):
+        t0 = time.perf_counter()
+        oracle.cascade_decode_ref(inp.q_bits[b:b + 1], inp.k_pages_bits, inp.v_pages_bits,
+                                  inp.prefix_block_table, inp.prefix_len, inp.block_table[b:b + 1],
+                                  inp.suffix_lens[b:b + 1], inp.scale, inp.page_size, inp.layout,
+                                  to_f64=W.as_f64)
+        secs += time.perf_counter() - t0
+        done.append(b)
+        if secs >= budget_s:
+            break
+    return per_req * len(done), secs, f"oracle cascade_decode_ref on requests {done}"
+
+
 # ----------------------------------------------------------------------------- main
 
 def decode_inputs(workload, heads=None):
@@ -544,6 +620,9 @@ def build_cases(workload, device, num_splits, kernel="auto", heads=None):
     if workload in CHUNKED_WORKLOADS:
         st = ChunkedState(W.CONFIGS[workload](), device)
         return [AppendCase(st), ChunkedAttnCase(st)]
+    if workload in CASCADE_WORKLOADS:
+        inp = W.CONFIGS[workload]()
+        return [CascadeCase(inp, device, kernel), DecodeCase(inp.as_plain_decode(), device, 0, kernel)]
     raise SystemExit(f"unknown workload {workload}")
 
 
@@ -648,6 +727,9 @@ def run_ours(args):
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
                                measured_traffic("prefill", c.inp.name))
             e["kernel"] = "fa_prefill_pp_kernel<%d, paged>" % c.inp.head_dim
+        elif isinstance(c, CascadeCase):
+            e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src, None)
+            e["kernel"] = "fa_prefill_pp_kernel<paged, key ranges> + decode split + fa_cascade_merge_kernel"
         elif isinstance(c, AppendCase):
             e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
                                measured_traffic("append", c.inp.name))
@@ -662,7 +744,11 @@ def run_ours(args):
         e["ms_per_launch"] = round(ms / c.launches, 4)
         rooflines.append(e)
     chunked = isinstance(main, AppendCase)
-    if chunked:
+    cascade = isinstance(main, CascadeCase)
+    if cascade:
+        value = aggregate_throughput(main.bytes, ms_case[0], N, 1e9)
+        unit = "GB/s"
+    elif chunked:
         # the whole chunked step (append + attention) against the attention FLOPs
         value = aggregate_throughput(cases[1].flops, ms_step, N, 1e12)
         unit = "TFLOP/s"
@@ -685,11 +771,16 @@ def run_ours(args):
            "parallelism": f"replicas x{N}" if N > 1 else "single GPU"}
     for i, c in enumerate(cases):
         key = {PrefillCase: "prefill", DecodeCase: "decode", AppendCase: "append",
-               ChunkedAttnCase: "chunked_prefill"}[type(c)]
+               ChunkedAttnCase: "chunked_prefill", CascadeCase: "cascade"}[type(c)]
         cfg[key] = c.describe()
     line["config"] = cfg
     line["roofline"] = rl
-    if chunked:
+    if cascade:
+        line["plain_decode_same_contexts"] = {
+            "ms": round(ms_case[1], 4), "speedup_of_cascade": round(ms_case[1] / ms_case[0], 3),
+            "note": "fa_decode_paged over prefix+suffix table rows (prefix read per request)"}
+        line["ms_per_step"] = round(ms_case[0], 4)
+    elif chunked:
         line["append"] = {"value": round(N * main.bytes / (ms_case[0] * 1e-3) / 1e9, 1), "unit": "GB/s",
                           "ms": round(ms_case[0], 4), "roofline": rooflines[0]}
         line["chunked_prefill_ms"] = round(ms_case[1], 4)
@@ -702,7 +793,9 @@ def run_ours(args):
         line["prefill_ms"] = round(ms_case[0], 4)
         line["prefill_roofline"] = rooflines[0]
     if e2e_case is not None:
-        if chunked:
+        if cascade:
+            e2e_v = N * main.bytes / (e2e_case[0] * 1e-3) / 1e9
+        elif chunked:
             e2e_v = N * cases[1].flops / (sum(e2e_case) * 1e-3) / 1e12
         elif isinstance(main, PrefillCase):
             e2e_v = N * main.flops / (e2e_case[0] * 1e-3) / 1e12
@@ -733,6 +826,9 @@ def cpu_baseline(case, budget):
     elif isinstance(case, ChunkedAttnCase):
         work, secs, desc = oracle_chunked_sample(case.inp, budget)
         val, unit = work / secs / 1e12, "TFLOP/s"
+    elif isinstance(case, CascadeCase):
+        work, secs, desc = oracle_cascade_sample(case.inp, budget)
+        val, unit = work / secs / 1e9, "GB/s"
     else:
         work, secs, desc = oracle_decode_sample(case.inp, budget)
         val, unit = work / secs / 1e9, "GB/s"
@@ -760,6 +856,8 @@ def run_reference(args):
     fn = oracle_prefill_sample if is_prefill else oracle_decode_sample
     if main in CHUNKED_WORKLOADS:
         fn = oracle_chunked_sample
+    if main in CASCADE_WORKLOADS:
+        fn = oracle_cascade_sample
     for _ in range(args.warmup and 1):
         fn(inp, 0.0)
     work, secs = 0.0, 0.0
@@ -792,7 +890,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
                     help="default | " + " | ".join(sorted(PREFILL_WORKLOADS | DECODE_WORKLOADS |
-                                                          CHUNKED_WORKLOADS)))
+                                                          CHUNKED_WORKLOADS | CASCADE_WORKLOADS)))
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--decode-kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
     ap.add_argument("--decode-heads", default=None, help="HQ:HKV override for a decode workload")

@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
     "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
-    "append_kv", "prefill_paged", "decode_paged_fp8",
+    "append_kv", "prefill_paged", "decode_paged_fp8", "cascade_decode", "cascade_workspace_bytes",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -39,7 +39,8 @@ EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
-    "fa_decode_paged_fp8", "fa_decode_plan_kv", "fa_decode_plan_ex",
+    "fa_decode_paged_fp8", "fa_decode_plan_kv", "fa_decode_plan_ex", "fa_cascade_workspace_bytes",
+    "fa_cascade_decode",
 ]
 
 FA_KV_BF16, FA_KV_E4M3 = 0, 1
@@ -101,6 +102,11 @@ def library() -> ctypes.CDLL:
                                     ctypes.POINTER(_DecodeOptions), ctypes.POINTER(vp),
                                     ctypes.POINTER(ctypes.c_size_t)]
     L.fa_decode_plan_ex.restype = i32
+    L.fa_cascade_workspace_bytes.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_size_t)]
+    L.fa_cascade_workspace_bytes.restype = i32
+    L.fa_cascade_decode.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, i32, vp, vp, vp, f32, vp, vp,
+                                    vp, ctypes.c_size_t, vp]
+    L.fa_cascade_decode.restype = i32
     L.fa_plan_get_info.argtypes = [vp, ctypes.POINTER(_PlanInfo)]
     L.fa_plan_get_info.restype = i32
     L.fa_plan_free.argtypes = [vp]
@@ -463,6 +469,43 @@ def prefill_paged(q, cu_seqlens_q, k_pages, v_pages, block_table, cache_seqlens,
         _ptr(cache_seqlens), len_h.ctypes.data_as(ctypes.c_void_p), batch, Hq, Hkv, d, page_size,
         1 if causal else 0, _scale_arg(scale), _ptr(out), _ptr(lse), _stream_ptr(stream))
     _check(st, "fa_prefill_paged")
+    return out, lse
+
+
+def cascade_workspace_bytes(plan: DecodePlan, prefix_len: int) -> int:
+    n = ctypes.c_size_t()
+    _check(library().fa_cascade_workspace_bytes(plan.handle, int(prefix_len), ctypes.byref(n)),
+           "fa_cascade_workspace_bytes")
+    return n.value
+
+
+def cascade_decode(q, k_pages, v_pages, prefix_block_table, prefix_len: int, block_table,
+                   cache_seqlens, plan: DecodePlan, *, layout: str = "NHD",
+                   scale: float | None = None, out=None, lse=None, workspace=None,
+                   return_lse: bool = True, stream=None):
+    """Decode where every request's context is a shared prefix (prefix_len
+    tokens in the pages of prefix_block_table) followed by its own suffix
+    (cache_seqlens[b] tokens through block_table[b]).  ``plan`` is a bf16 plan
+    for the suffix lengths.  Returns (out, lse)."""
+    torch = _torch()
+    _require_cuda(q, k_pages, v_pages, prefix_block_table, block_table, cache_seqlens, out, lse,
+                  workspace)
+    _check_pool(k_pages, v_pages, block_table)
+    _check_q_rows(q, plan)
+    ps, ts, hs = page_strides(k_pages, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    need = cascade_workspace_bytes(plan, prefix_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = library().fa_cascade_decode(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], ps, ts, hs, _ptr(prefix_block_table),
+        int(prefix_len), _ptr(block_table), _ptr(cache_seqlens), plan.handle, _scale_arg(scale),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream))
+    _check(st, "fa_cascade_decode")
     return out, lse
 
 

@@ -535,3 +535,63 @@ __global__ void __launch_bounds__(128) fa_merge_kernel(const MergeParams p) {
 }
 
 }  // namespace fa
+
+namespace fa {
+
+// ----------------------------------------------------------------------------
+// Cascade merge: for every (row, head), the LSE merge of the shared prefix's
+// key-range states (fp32) and the row's own suffix state (bf16 O + LSE), one
+// warp per (row, head).  An empty suffix carries LSE = -inf and zero weight.
+// ----------------------------------------------------------------------------
+struct CascadeMergeParams {
+  const float* prefix_o;          // [S, rows, H, D] normalised
+  const float* prefix_lse;        // [S, rows, H]
+  const __nv_bfloat16* suffix_o;  // [rows, H, D] normalised
+  const float* suffix_lse;        // [rows, H]
+  __nv_bfloat16* out;             // [rows, H, D]
+  float* lse;                     // [rows, H] or null
+  int num_prefix;
+  int rows;
+  int num_heads;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) fa_cascade_merge_kernel(const CascadeMergeParams p) {
+  constexpr int V = D / 32;   // columns per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rh = blockIdx.x * 4 + warp;
+  if (rh >= p.rows * p.num_heads) return;
+  const size_t stride = static_cast<size_t>(p.rows) * p.num_heads;
+  const float ls = p.suffix_lse[rh];
+  float M = ls;
+  for (int i = lane; i < p.num_prefix; i += 32) M = fmaxf(M, p.prefix_lse[i * stride + rh]);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+  float o[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) o[v] = 0.0f;
+  float wsum = 0.0f;
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (M != -INFINITY) {
+    for (int i = 0; i < p.num_prefix; ++i) {
+      const float w = ex2_approx((p.prefix_lse[i * stride + rh] - M) * kLog2e);
+      wsum += w;
+      const float* src = p.prefix_o + (i * stride + rh) * D + lane * V;
+#pragma unroll
+      for (int v = 0; v < V; ++v) o[v] = fmaf(w, src[v], o[v]);
+    }
+    const float w = ex2_approx((ls - M) * kLog2e);   // -inf -> 0
+    wsum += w;
+    const __nv_bfloat16* src = p.suffix_o + static_cast<size_t>(rh) * D + lane * V;
+#pragma unroll
+    for (int v = 0; v < V; ++v) o[v] = fmaf(w, __bfloat162float(src[v]), o[v]);
+  }
+  const float inv = (wsum > 0.0f) ? 1.0f / wsum : 0.0f;
+  __nv_bfloat16* dst = p.out + static_cast<size_t>(rh) * D + lane * V;
+#pragma unroll
+  for (int v = 0; v < V; v += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + v) = __floats2bfloat162_rn(o[v] * inv, o[v + 1] * inv);
+  if (lane == 0 && p.lse != nullptr) p.lse[rh] = (wsum > 0.0f) ? M + logf(wsum) : -INFINITY;
+}
+
+}  // namespace fa

@@ -739,3 +739,148 @@ FA_API int fa_decode_paged_static(const void* q, const void* k_pages, const void
                          block_table, cache_seqlens_dev, plan, scale, out, lse, scratch,
                          kStaticScratchBytes, stream);
 }
+
+// ============================================================================
+// Cascade (prefix-sharing) decode: every request's query attends to one shared
+// prefix (read once for the whole batch by the paged prefill kernel, the
+// requests acting as the query tokens of one full-attention sequence, cut into
+// key ranges to fill the SMs) and to its own suffix (the paged decode); the
+// two states are merged by LSE.
+namespace {
+
+struct CascadeLayout {
+  int splits = 0, split_tiles = 0;
+  size_t off_so = 0, off_sl = 0, off_po = 0, off_pl = 0, total = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+CascadeLayout cascade_layout(const fa::DecodePlan& pl, int prefix_len) {
+  CascadeLayout c;
+  const size_t rows = static_cast<size_t>(pl.batch) * pl.num_q_heads;
+  c.off_so = align256(pl.workspace_bytes);
+  c.off_sl = align256(c.off_so + rows * pl.head_dim * 2);
+  c.off_po = align256(c.off_sl + rows * 4);
+  if (prefix_len > 0) {
+    const int n_ktiles = (prefix_len + 127) / 128;
+    const int n_qtiles = (pl.batch + 127) / 128;
+    const int g = pl.group;
+    const int per_head = (g % 2 == 0) ? n_qtiles * (g / 2) : ((n_qtiles + 1) / 2) * g;
+    const int base = per_head * pl.num_kv_heads;             // CTAs per key range
+    const int want = std::max(1, (pl.num_sms + base - 1) / base);
+    c.splits = std::min(want, n_ktiles);
+    c.split_tiles = (n_ktiles + c.splits - 1) / c.splits;
+    c.splits = (n_ktiles + c.split_tiles - 1) / c.split_tiles;
+  }
+  c.off_pl = align256(c.off_po + static_cast<size_t>(c.splits) * rows * pl.head_dim * 4);
+  c.total = align256(c.off_pl + static_cast<size_t>(c.splits) * rows * 4);
+  return c;
+}
+
+}  // namespace
+
+FA_API int fa_cascade_workspace_bytes(const fa_plan* plan, int prefix_len, size_t* bytes) {
+  if (plan == nullptr || plan->p.magic != fa::kPlanMagic || bytes == nullptr || prefix_len < 0)
+    return FA_ERR_INVALID_ARG;
+  *bytes = cascade_layout(plan->p, prefix_len).total;
+  return FA_OK;
+}
+
+FA_API int fa_cascade_decode(const void* q, const void* k_pages, const void* v_pages,
+                             int64_t num_pages, int64_t page_stride, int64_t token_stride,
+                             int64_t head_stride, const int32_t* prefix_block_table,
+                             int prefix_len, const int32_t* block_table,
+                             const int32_t* cache_seqlens_dev, const fa_plan* plan, float scale,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (plan == nullptr || plan->p.magic != fa::kPlanMagic) return FA_ERR_INVALID_ARG;
+  const fa::DecodePlan& pl = plan->p;
+  if (pl.kv_elem_bytes != 2 || pl.q_len != 1) return FA_ERR_PLAN_MISMATCH;
+  if (!q || !out || !workspace || prefix_len < 0 || (prefix_len > 0 && !prefix_block_table))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(workspace, 256) ||
+      !aligned(prefix_block_table, 4))
+    return FA_ERR_INVALID_ARG;
+  if (!valid_pool(k_pages, v_pages, num_pages, page_stride, token_stride, head_stride))
+    return FA_ERR_INVALID_ARG;
+  const CascadeLayout c = cascade_layout(pl, prefix_len);
+  if (workspace_bytes < c.total) return FA_ERR_WORKSPACE;
+  scale = resolve_scale(scale, pl.head_dim);
+  if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prefix_len == 0)   // nothing shared: the plain decode
+    return decode_paged_impl(q, k_pages, v_pages, num_pages, page_stride, token_stride, head_stride,
+                             block_table, cache_seqlens_dev, plan, scale, false, 1.0f, 1.0f, out,
+                             lse, workspace, pl.workspace_bytes, stream);
+
+  // 1. shared prefix: B "tokens" (one per request) x Hq heads, full attention
+  static thread_local fa::PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  {
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(pl.head_dim), static_cast<cuuint64_t>(pl.num_q_heads),
+                                static_cast<cuuint64_t>(pl.batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pl.head_dim) * 2,
+                                   static_cast<cuuint64_t>(pl.num_q_heads) * pl.head_dim * 2};
+    int st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
+  int st = encode_page_pool_map(&prm.tm_k, k_pages, num_pages, page_stride, token_stride, head_stride,
+                                pl.page_size, pl.num_kv_heads, pl.head_dim, 64,
+                                CU_TENSOR_MAP_SWIZZLE_128B, &prm.head_coord, &prm.page_coord);
+  if (st != FA_OK) return st;
+  st = encode_page_pool_map(&prm.tm_v, v_pages, num_pages, page_stride, token_stride, head_stride,
+                            pl.page_size, pl.num_kv_heads, pl.head_dim, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                            &prm.head_coord, &prm.page_coord);
+  if (st != FA_OK) return st;
+  prm.cu_seqlens = nullptr;
+  prm.uniform_q_len = pl.batch;
+  prm.cache_seqlens = nullptr;
+  prm.uniform_k_len = prefix_len;
+  prm.block_table = prefix_block_table;
+  prm.max_pages = (prefix_len + pl.page_size - 1) / pl.page_size;
+  prm.num_pages = static_cast<int>(num_pages);
+  prm.num_q_heads = pl.num_q_heads;
+  prm.group = pl.group;
+  prm.causal = 0;
+  prm.scale_log2 = scale * kLog2e;
+  prm.kv_splits = c.splits;
+  prm.kv_split_tiles = c.split_tiles;
+  prm.total_q = pl.batch;
+  prm.part_o = reinterpret_cast<float*>(ws + c.off_po);
+  prm.part_lse = reinterpret_cast<float*>(ws + c.off_pl);
+  std::vector<std::pair<uint32_t, int>> groups;
+  build_prefill_groups({static_cast<int64_t>(pl.batch)}, {static_cast<int64_t>(prefix_len)},
+                       pl.num_q_heads, pl.num_kv_heads, false, &groups);
+  for (auto& g : groups) g.second *= c.splits;
+  st = pl.head_dim == 128 ? launch_prefill<128, true>(prm, groups, s) : launch_prefill<64, true>(prm, groups, s);
+  if (st != FA_OK) return st;
+
+  // 2. each request's own suffix
+  __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(ws + c.off_so);
+  float* sl = reinterpret_cast<float*>(ws + c.off_sl);
+  st = decode_paged_impl(q, k_pages, v_pages, num_pages, page_stride, token_stride, head_stride,
+                         block_table, cache_seqlens_dev, plan, scale, false, 1.0f, 1.0f, so, sl,
+                         workspace, pl.workspace_bytes, stream);
+  if (st != FA_OK) return st;
+
+  // 3. LSE merge of the prefix ranges and the suffix
+  fa::CascadeMergeParams mp;
+  mp.prefix_o = prm.part_o;
+  mp.prefix_lse = prm.part_lse;
+  mp.suffix_o = so;
+  mp.suffix_lse = sl;
+  mp.out = static_cast<__nv_bfloat16*>(out);
+  mp.lse = lse;
+  mp.num_prefix = c.splits;
+  mp.rows = pl.batch;
+  mp.num_heads = pl.num_q_heads;
+  dim3 grid((pl.batch * pl.num_q_heads + 3) / 4);
+  if (pl.head_dim == 128)
+    fa::fa_cascade_merge_kernel<128><<<grid, 128, 0, s>>>(mp);
+  else
+    fa::fa_cascade_merge_kernel<64><<<grid, 128, 0, s>>>(mp);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}

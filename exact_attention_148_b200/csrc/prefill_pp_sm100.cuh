@@ -60,9 +60,20 @@ struct PrefillParams {
   CUtensorMap tm_v;   //   64 columns x one 64-token page, 128B swizzle
   __nv_bfloat16* out;        // [T, Hq, d]
   float* lse;                // [T, Hq] or null
-  const int32_t* cu_seqlens; // [B+1] query offsets
+  const int32_t* cu_seqlens; // [B+1] query offsets, or null: one sequence of uniform_q_len
   const int32_t* block_table;    // paged: [B, max_pages]
-  const int32_t* cache_seqlens;  // paged: [B] keys per request
+  const int32_t* cache_seqlens;  // paged: [B] keys per request, or null: uniform_k_len
+  int uniform_q_len;
+  int uniform_k_len;
+  // Key-range splits (full attention only): the key tiles of every q tile are
+  // cut into kv_splits ranges of kv_split_tiles; each range's normalised O and
+  // LSE go to part_o [kv_splits, total_q, Hq, d] / part_lse [kv_splits, total_q, Hq]
+  // (fp32) for an LSE merge.  part_o null: bf16 out / lse as usual (kv_splits 1).
+  int kv_splits;
+  int kv_split_tiles;
+  int total_q;
+  float* part_o;
+  float* part_lse;
   int max_pages;
   int num_pages;
   int head_coord;            // paged: tensor-map dimension (1..3) of the kv head
@@ -180,22 +191,34 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   }
   const int seq = static_cast<int>(p.group_id[lo] >> 16);
   const int kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
-  const int rank = bid - p.group_start[lo];
-  const int s0 = p.cu_seqlens[seq];
-  const int L = p.cu_seqlens[seq + 1] - s0;     // queries
+  int rank = bid - p.group_start[lo];
+  const int s0 = p.cu_seqlens != nullptr ? p.cu_seqlens[seq] : 0;
+  const int L = p.cu_seqlens != nullptr ? p.cu_seqlens[seq + 1] - s0 : p.uniform_q_len;   // queries
   const int n_qtiles = (L + C::BM - 1) / C::BM;
   int Lk = L;                                   // keys
   if constexpr (PAGED) {
-    Lk = p.cache_seqlens[seq];
+    Lk = p.cache_seqlens != nullptr ? p.cache_seqlens[seq] : p.uniform_k_len;
+    // A causal chunk's own tokens are among the keys (k_len >= q_len); full
+    // attention (the shared prefix of a cascade) may have fewer keys than queries.
     const int cap = p.max_pages * kPrefillPage;
-    if (Lk < L || Lk > cap) {
+    if ((p.causal && Lk < L) || Lk > cap || Lk < 0) {
       if (rank == 0 && threadIdx.x == 0) record_status(FA_ERR_PLAN_MISMATCH);
-      Lk = min(max(Lk, L), cap);
+      Lk = min(max(Lk, p.causal ? L : 0), cap);
     }
   }
   const int off = p.causal ? Lk - L : 0;        // query i sits at key position i + off
-  const int n_ktiles = (Lk + C::BN - 1) / C::BN;
+  const int n_ktiles_all = (Lk + C::BN - 1) / C::BN;
   const int G = p.group;
+  // Key-range split: a group holds kv_splits copies of its q-tile CTAs, one
+  // per range of kv_split_tiles key tiles (tiles [kt0, n_ktiles)).
+  int kt0 = 0, n_ktiles = n_ktiles_all, split = 0;
+  if (p.kv_splits > 1) {
+    const int base_ctas = ((G & 1) == 0) ? n_qtiles * (G >> 1) : ((n_qtiles + 1) >> 1) * G;
+    split = rank / base_ctas;
+    rank -= split * base_ctas;
+    kt0 = split * p.kv_split_tiles;
+    n_ktiles = min(n_ktiles_all, kt0 + p.kv_split_tiles);
+  }
   int qtile[2], head[2];
   if ((G & 1) == 0) {            // two heads of the group, same rows
     const int half = G >> 1;
@@ -217,7 +240,8 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     const bool active = qtile[k] >= 0 && qtile[k] < n_qtiles;
     n_kv[k] = !active ? 0
                       : (p.causal ? min(n_ktiles, (qtile[k] * C::BM + C::BM - 1 + off) / C::BN + 1)
-                                  : n_ktiles);
+                                  : n_ktiles) - kt0;
+    if (n_kv[k] < 0) n_kv[k] = 0;
   }
   if (n_kv[0] == 0 && n_kv[1] == 0) return;   // uniform; nothing allocated yet
   const int n_max = max(n_kv[0], n_kv[1]);
@@ -288,12 +312,12 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       if (n_kv[1] > 0) load_q(1, head[1], qtile[1]);
     }
     const int32_t* bt_row = p.block_table + static_cast<size_t>(seq) * p.max_pages;
-    const int tail_tile = (Lk % kPrefillPage != 0) ? (Lk - 1) / C::BN : -1;
+    const int tail_tile = (Lk % kPrefillPage != 0) ? (Lk - 1) / C::BN - kt0 : -1;   // split-relative
     int pg_base = -1, pg_mine = 0, issued = 0, tail_item = -1;
     bool ok = true;
     for (int item = 0; item < 2 * n_max; ++item) {
-      const int jt = item >> 1;
-      const int lp0 = 2 * jt;
+      const int jt = item >> 1;                       // split-relative key tile
+      const int lp0 = 2 * (kt0 + jt);
       if ((lp0 & ~31) != pg_base) {
         pg_base = lp0 & ~31;
         const int lp = pg_base + lane;
@@ -340,8 +364,8 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       tail_landed = __all_sync(0xffffffffu, mbar_wait(bar_vtail, 0, abort_flag));
       if (tail_landed) {
         // rows [Lk, end of its page) of the tile, in every 64-column chunk
-        const int r0 = Lk - (tail_item >> 1) * C::BN;
-        const int r1 = ((Lk + kPrefillPage - 1) / kPrefillPage) * kPrefillPage - (tail_item >> 1) * C::BN;
+        const int r0 = Lk - (kt0 + (tail_item >> 1)) * C::BN;
+        const int r1 = ((Lk + kPrefillPage - 1) / kPrefillPage) * kPrefillPage - (kt0 + (tail_item >> 1)) * C::BN;
         uint4* tile = reinterpret_cast<uint4*>(smem + C::KV_OFF + (tail_item % C::NS) * C::TILE_BYTES);
         const int per_chunk = (r1 - r0) * 8;          // 16-byte stores per chunk
         for (int e = lane; e < C::CHUNKS * per_chunk; e += 32) {
@@ -384,7 +408,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
         if (!mbar_wait(bar_kv_empty(item), ((item / C::NS) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar_kv_full(item), C::TILE_BYTES);
         const CUtensorMap* map = (item & 1) ? &p.tm_v : &p.tm_k;
-        const int row = s0 + (item >> 1) * C::BN;
+        const int row = s0 + (kt0 + (item >> 1)) * C::BN;
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c)
           tma_load_3d(kv_s(item) + c * C::CHUNK_BYTES, map, bar_kv_full(item), c * 64, kv_head, row);
@@ -500,9 +524,9 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       reg_dep(s[2]);
       reg_dep(s[3]);
 
-      const bool masked = j * C::BN + C::BN - 1 > tile_last;
+      const bool masked = (kt0 + j) * C::BN + C::BN - 1 > tile_last;
       if (masked) {
-        const int lim = row_last - j * C::BN;
+        const int lim = row_last - (kt0 + j) * C::BN;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -595,6 +619,24 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       const bool valid = q_row < L;
       __nv_bfloat16* orow =
           p.out + (static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head) * D;
+      if (p.part_o != nullptr) {
+        // key-range split: normalised fp32 O and LSE of this range
+        const size_t prow = (static_cast<size_t>(split) * p.total_q + s0 + q_row) * p.num_q_heads + my_head;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld_x32(oc + c * 32, o);
+          tmem_ld_wait(o);
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + c * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                   __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+          }
+        }
+        if (valid) p.part_lse[prow] = (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
+      } else {
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -614,6 +656,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       if (valid && p.lse != nullptr)
         p.lse[static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head] =
             (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
+      }
     }
   }
 

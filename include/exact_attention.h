@@ -317,6 +317,32 @@ int fa_decode_paged_static(const void* q, const void* k_pages, const void* v_pag
                            void* out, float* lse, void* stream);
 
 /*
+ * fa_cascade_decode — decode with a prefix shared by every request of the
+ * batch (prefix sharing: wsisp.com "FIA / FlashAttention", section 三, MLA/GQA
+ * row), computed as two partial states merged by their LSE (niuteng5618.github.io,
+ * section "FA对decode阶段的影响", steps 3-4).
+ *
+ *   The context of request b is the shared prefix (prefix_len tokens in the
+ *   pages listed by prefix_block_table, device [ceil(prefix_len / page_size)])
+ *   followed by its own suffix (cache_seqlens_dev[b] tokens through row b of
+ *   block_table).  The result equals fa_decode_paged over that concatenation.
+ *   plan: a bf16, single-token plan made for the suffix lengths.
+ *   workspace: >= fa_cascade_workspace_bytes(plan, prefix_len), 256-byte aligned.
+ * The prefix is read once for the whole batch: the requests act as the query
+ * tokens of one full-attention sequence over the prefix (the paged prefill
+ * kernel, its key range cut to fill the SMs); the suffixes run through the
+ * paged decode; one kernel merges the states.  prefix_len == 0 is the plain
+ * decode.  q, out [batch, Hq, d] bf16; lse [batch, Hq] fp32 or NULL.
+ */
+int fa_cascade_workspace_bytes(const fa_plan* plan, int prefix_len, size_t* bytes);
+int fa_cascade_decode(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                      int64_t page_stride, int64_t token_stride, int64_t head_stride,
+                      const int32_t* prefix_block_table, int prefix_len,
+                      const int32_t* block_table, const int32_t* cache_seqlens_dev,
+                      const fa_plan* plan, float scale, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
  * fa_merge_states — combine partial attention states by their LSE (the light
  * reduction kernel of Flash-Decoding: niuteng5618.github.io, section
  * "FA对decode阶段的影响", step 4).

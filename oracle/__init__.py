@@ -15,6 +15,7 @@ from .attention import (  # noqa: F401
     attention_probs_ref,
     attention_ref,
     attention_rows_ref,
+    cascade_decode_ref,
     gather_paged_kv,
     kv_head_of,
     merge_states_ref,

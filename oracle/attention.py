@@ -414,3 +414,37 @@ def paged_prefill_rows_ref(q, cu_seqlens_q, k_pages, v_pages, block_table, cache
         out[n] = (P @ V[:nk])[0]
         lse[n] = l[0]
     return out, lse
+
+
+def cascade_decode_ref(q, k_pages, v_pages, prefix_block_table, prefix_len: int, block_table,
+                       suffix_lens, scale=None, page_size: int = 64, layout: str = "NHD",
+                       to_f64=lambda a: np.asarray(a, dtype=np.float64)):
+    """Decode over a shared prefix followed by each request's own suffix.
+
+    Request b's keys are the prefix_len tokens of the shared pages, then the
+    suffix_lens[b] tokens of its own pages (prefix sharing, wsisp.com
+    "FIA / FlashAttention", section 三): plain attention of its query row over
+    that concatenation.  Returns (O [B, Hq, d], LSE [B, Hq]).
+    """
+    q = np.asarray(q)
+    B, Hq, d = q.shape
+    Hkv = k_pages.shape[2] if layout == "NHD" else k_pages.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for g in range(Hkv):
+        Kp, Vp = gather_paged_kv(k_pages, v_pages, prefix_block_table, int(prefix_len), g,
+                                 page_size, layout)
+        for b in range(B):
+            Ks, Vs = gather_paged_kv(k_pages, v_pages, block_table[b], int(suffix_lens[b]), g,
+                                     page_size, layout)
+            K = to_f64(np.concatenate([Kp, Ks], axis=0))
+            V = to_f64(np.concatenate([Vp, Vs], axis=0))
+            for h in range(Hq):
+                if kv_head_of(h, Hq, Hkv) != g:
+                    continue
+                P, l = _softmax_with_lse(_scores(to_f64(q[b, h])[None, :], K, scale))
+                out[b, h] = (P @ V)[0] if K.shape[0] else 0.0
+                lse[b, h] = l[0]
+    return out, lse

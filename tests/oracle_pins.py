@@ -440,3 +440,48 @@ def pin_golden_fp8_decode(paged_decode_ref, dequantize_e4m3):
                             v_to_f64=lambda a: dequantize_e4m3(a, g["v_scale"]))
     _close(o, g["o"], 1e-13, "fp8 decode O")
     _close(l, g["lse"], 1e-13, "fp8 decode LSE")
+
+
+# --- cascade (shared-prefix) decode -------------------------------------------
+
+def pin_cascade_matches_concatenation(cascade_decode_ref, partial_state_ref, layout="NHD", seed=161):
+    """Hand-built contiguous context = prefix rows then suffix rows; the cascade
+    must equal plain attention of each query over it (prefix not a page multiple)."""
+    g = np.random.default_rng(seed)
+    hq, hkv, d, ps = 4, 2, 5, 4
+    P, suf = 7, [0, 3, 9]
+    pre_k, pre_v = g.standard_normal((P, hkv, d)), g.standard_normal((P, hkv, d))
+    seqs = [(pre_k, pre_v)] + [(g.standard_normal((L, hkv, d)), g.standard_normal((L, hkv, d)))
+                               for L in suf]
+    kp, vp, bt = _scatter_to_pages(seqs, ps, layout, g)
+    q = g.standard_normal((len(suf), hq, d))
+    o, l = cascade_decode_ref(q, kp, vp, bt[0][:(P + ps - 1) // ps], P, bt[1:], suf, 0.7,
+                              page_size=ps, layout=layout)
+    for b, L in enumerate(suf):
+        K = np.concatenate([pre_k, seqs[b + 1][0]])
+        V = np.concatenate([pre_v, seqs[b + 1][1]])
+        for h in range(hq):
+            gh = h // (hq // hkv)
+            ob, lb = partial_state_ref(q[b, h][None], K[:, gh], V[:, gh], 0.7)
+            _close(o[b, h], ob[0], 1e-13, f"cascade O b={b} h={h}")
+            _close(l[b, h], lb[0], 1e-13, f"cascade LSE b={b} h={h}")
+
+
+def pin_cascade_aligned_is_decode(cascade_decode_ref, paged_decode_ref, seed=171):
+    """With a page-aligned prefix the cascade equals the plain paged decode whose
+    table rows list the prefix pages and then the suffix pages."""
+    g = np.random.default_rng(seed)
+    hq, hkv, d, ps = 6, 3, 4, 4
+    P, suf = 8, [1, 0, 6]
+    seqs = [(g.standard_normal((P, hkv, d)), g.standard_normal((P, hkv, d)))] + \
+        [(g.standard_normal((L, hkv, d)), g.standard_normal((L, hkv, d))) for L in suf]
+    kp, vp, bt = _scatter_to_pages(seqs, ps, "HND", g)
+    q = g.standard_normal((len(suf), hq, d))
+    pre = bt[0][:P // ps]
+    o, l = cascade_decode_ref(q, kp, vp, pre, P, bt[1:], suf, 0.5, page_size=ps, layout="HND")
+    full = np.full((len(suf), len(pre) + bt.shape[1]), -1)
+    full[:, :len(pre)] = pre
+    full[:, len(pre):] = bt[1:]
+    od, ld = paged_decode_ref(q, kp, vp, full, [P + L for L in suf], 0.5, page_size=ps, layout="HND")
+    _close(o, od, 1e-13, "cascade vs decode O")
+    _close(l, ld, 1e-13, "cascade vs decode LSE")

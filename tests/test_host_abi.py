@@ -338,3 +338,27 @@ def test_multi_token_plans(lib):
         fa.decode_plan(np.array([3, 2000], dtype=np.int32), num_q_heads=8, num_kv_heads=2,
                        head_dim=128, max_pages_per_seq=40, num_sms=148, q_len=4)
     assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+def test_cascade_validation_before_any_cuda_call(lib):
+    A = 0x10000
+    p = _plan([100, 2000], hq=8, hkv=2)
+    n = ctypes.c_size_t()
+    assert lib.fa_cascade_workspace_bytes(p.handle, 1000, ctypes.byref(n)) == fa.FA_OK
+    n0 = ctypes.c_size_t()
+    assert lib.fa_cascade_workspace_bytes(p.handle, 0, ctypes.byref(n0)) == fa.FA_OK
+    assert n.value > n0.value >= p.workspace_bytes
+    assert lib.fa_cascade_workspace_bytes(p.handle, -1, ctypes.byref(n)) == fa.FA_ERR_INVALID_ARG
+
+    def call(plan=p.handle, ws_bytes=None, prefix=1000, pre=A, ws=A):
+        return lib.fa_cascade_decode(_fake(A), _fake(A), _fake(A), 100, 64 * 2 * 128, 2 * 128, 128,
+                                     _fake(pre), prefix, _fake(A), _fake(A), plan, float("nan"),
+                                     _fake(A), None, _fake(ws), n.value if ws_bytes is None else ws_bytes,
+                                     None)
+    n.value = 0
+    lib.fa_cascade_workspace_bytes(p.handle, 1000, ctypes.byref(n))
+    assert call(ws_bytes=n.value - 256) == fa.FA_ERR_WORKSPACE
+    assert call(pre=0) == fa.FA_ERR_INVALID_ARG
+    assert call(ws=A + 16) == fa.FA_ERR_INVALID_ARG
+    p8 = _plan([100, 2000], hq=8, hkv=2, kv_dtype="e4m3")
+    assert call(plan=p8.handle) == fa.FA_ERR_PLAN_MISMATCH

@@ -219,3 +219,26 @@ def test_fp8_scales_swapped_is_caught():
     except AssertionError:
         return
     raise AssertionError("swapped K/V scales not caught")
+
+
+def test_cascade_mutants_are_caught(monkeypatch):
+    """A cascade that drops the prefix, or counts it twice, must be caught."""
+    real = A.cascade_decode_ref
+
+    def no_prefix(q, kp, vp, pre, P, bt, suf, scale=None, page_size=64, layout="NHD", **kw):
+        return real(q, kp, vp, pre[:0], 0, bt, suf, scale, page_size, layout, **kw)
+
+    def double_prefix(q, kp, vp, pre, P, bt, suf, scale=None, page_size=64, layout="NHD", **kw):
+        n = len(pre)
+        bt2 = np.full((bt.shape[0], n + bt.shape[1]), -1)
+        bt2[:, :n] = pre
+        bt2[:, n:] = bt
+        if P % page_size:     # only page-aligned prefixes can be doubled through the table
+            return real(q, kp, vp, pre, P, bt, suf, scale * 1.01, page_size, layout, **kw)
+        return real(q, kp, vp, pre, P, bt2, np.asarray(suf) + P, scale, page_size, layout, **kw)
+
+    for bad in (no_prefix, double_prefix):
+        pins = [lambda: P.pin_cascade_matches_concatenation(bad, A.partial_state_ref),
+                lambda: P.pin_cascade_aligned_is_decode(bad, A.paged_decode_ref)]
+        with np.errstate(all="ignore"):
+            assert _some_pin_fires(pins), bad.__name__

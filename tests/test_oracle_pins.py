@@ -202,3 +202,12 @@ def test_empty_cache_decodes_to_zero():
     ob, lb = oracle.partial_state_ref(q[0], K, V, 0.5)
     np.testing.assert_allclose(o[0], ob, atol=1e-14)
     np.testing.assert_allclose(l[0], lb, atol=1e-14)
+
+
+@pytest.mark.parametrize("layout", ["NHD", "HND"])
+def test_cascade_matches_concatenation(layout):
+    P.pin_cascade_matches_concatenation(oracle.cascade_decode_ref, oracle.partial_state_ref, layout)
+
+
+def test_cascade_aligned_is_decode():
+    P.pin_cascade_aligned_is_decode(oracle.cascade_decode_ref, oracle.paged_decode_ref)

@@ -572,6 +572,100 @@ def poison_chunked(inp: ChunkedPrefillInputs) -> ChunkedPrefillInputs:
     return out
 
 
+# ---------------------------------------------------------------------------
+# Cascade (shared-prefix) decode workloads
+# ---------------------------------------------------------------------------
+
+@dataclass
+class CascadeInputs:
+    """Decode where every request shares one prefix (its pages listed once in
+    ``prefix_block_table``) and then has its own suffix (``block_table`` rows,
+    ``suffix_lens``)."""
+    name: str
+    q_bits: np.ndarray            # [B, Hq, d]
+    k_pages_bits: np.ndarray      # NHD [P, page, Hkv, d] or HND [P, Hkv, page, d]
+    v_pages_bits: np.ndarray
+    prefix_block_table: np.ndarray   # [ceil(prefix_len / page)] int32
+    prefix_len: int
+    block_table: np.ndarray       # [B, max_suffix_pages] int32 (unused = -1)
+    suffix_lens: np.ndarray       # [B] int32
+    scale: float
+    layout: str = "NHD"
+    page_size: int = PAGE_SIZE
+
+    @property
+    def batch(self):
+        return self.q_bits.shape[0]
+
+    @property
+    def num_q_heads(self):
+        return self.q_bits.shape[1]
+
+    @property
+    def head_dim(self):
+        return self.q_bits.shape[2]
+
+    @property
+    def num_kv_heads(self):
+        return self.k_pages_bits.shape[2] if self.layout == "NHD" else self.k_pages_bits.shape[1]
+
+    def strides(self):
+        P, a, b, d = self.k_pages_bits.shape
+        if self.layout == "NHD":
+            return a * b * d, b * d, d
+        return a * b * d, d, b * d
+
+    def algorithmic_bytes(self) -> float:
+        """The shared prefix's K/V once, every suffix's K/V once, q and out."""
+        B, Hq, d = self.q_bits.shape
+        tokens = self.prefix_len + float(self.suffix_lens.astype(np.int64).sum())
+        return 2.0 * tokens * self.num_kv_heads * d * 2 + B * Hq * d * 2 * 2 + B * Hq * 4
+
+    def as_plain_decode(self) -> "DecodeInputs":
+        """The same contexts as a plain paged decode (each request's table row =
+        prefix pages then suffix pages); needs a page-aligned prefix."""
+        assert self.prefix_len % self.page_size == 0
+        n_pre = len(self.prefix_block_table)
+        bt = np.full((self.batch, n_pre + self.block_table.shape[1]), -1, dtype=np.int32)
+        bt[:, :n_pre] = self.prefix_block_table
+        bt[:, n_pre:] = self.block_table
+        return DecodeInputs(self.name + "_plain", self.q_bits, self.k_pages_bits, self.v_pages_bits,
+                            bt, (self.suffix_lens + self.prefix_len).astype(np.int32), self.scale,
+                            self.layout, self.page_size)
+
+
+def make_cascade(prefix_len, suffix_lens, num_q_heads, num_kv_heads, head_dim, *, seed=21,
+                 layout="NHD", extra_pages=0, name="cascade") -> CascadeInputs:
+    suffix_lens = np.asarray(suffix_lens, dtype=np.int64)
+    B = len(suffix_lens)
+    ps = PAGE_SIZE
+    n_pre = (int(prefix_len) + ps - 1) // ps
+    n_suf = (suffix_lens + ps - 1) // ps
+    P = n_pre + int(n_suf.sum()) + int(extra_pages)
+    ss = np.random.SeedSequence(seed)
+    s_perm, s_q, s_k, s_v = ss.spawn(4)
+    perm = np.random.Generator(np.random.PCG64(s_perm)).permutation(P).astype(np.int32)
+    pre_bt = perm[:n_pre].copy()
+    bt = np.full((B, int(max(1, n_suf.max()))), -1, dtype=np.int32)
+    off = n_pre
+    for b in range(B):
+        bt[b, :n_suf[b]] = perm[off:off + n_suf[b]]
+        off += int(n_suf[b])
+    shape = (P, ps, num_kv_heads, head_dim) if layout == "NHD" else (P, num_kv_heads, ps, head_dim)
+    q = _normal_bf16_bits(s_q, (B, num_q_heads, head_dim))
+    kp = _normal_bf16_bits(s_k, shape)
+    vp = _normal_bf16_bits(s_v, shape)
+    return CascadeInputs(name, q, kp, vp, pre_bt, int(prefix_len), bt, suffix_lens.astype(np.int32),
+                         1.0 / math.sqrt(head_dim), layout, ps)
+
+
+def cascade_decode_batch() -> CascadeInputs:
+    """64 requests sharing an 8192-token prefix, own suffixes U[64, 2048],
+    32 q / 8 kv heads, d=128, shuffled pages."""
+    suf = np.random.default_rng(21).integers(64, 2048 + 1, size=64)
+    return make_cascade(8192, suf, 32, 8, 128, seed=21, name="cascade_decode_batch")
+
+
 CONFIGS = {
     "tiny_causal_prefill": tiny_causal_prefill,
     "varlen_causal_prefill": varlen_causal_prefill,
@@ -584,6 +678,7 @@ CONFIGS = {
     "paged_decode_gqa8": paged_decode_gqa8,
     "paged_decode_gqa16": paged_decode_gqa16,
     "speculative_decode_batch": speculative_decode_batch,
+    "cascade_decode_batch": cascade_decode_batch,
     "tiny_chunked_prefill": tiny_chunked_prefill,
     "chunked_prefill_batch": chunked_prefill_batch,
 }
