@@ -767,7 +767,7 @@ CascadeLayout cascade_layout(const fa::DecodePlan& pl, int prefix_len) {
     const int g = pl.group;
     const int per_head = (g % 2 == 0) ? n_qtiles * (g / 2) : ((n_qtiles + 1) / 2) * g;
     const int base = per_head * pl.num_kv_heads;             // CTAs per key range
-    const int want = std::max(1, (pl.num_sms + base - 1) / base);
+    const int want = std::max(1, pl.num_sms / base);     // one wave of CTAs
     c.splits = std::min(want, n_ktiles);
     c.split_tiles = (n_ktiles + c.splits - 1) / c.splits;
     c.splits = (n_ktiles + c.split_tiles - 1) / c.split_tiles;
