@@ -112,8 +112,9 @@ struct PrefillPPCfg {
   static constexpr int Q_OFF = 0;                          // two Q tiles
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final, v_tail
-  static constexpr int NUM_BARS = 1 + 2 * NS + 8;
+  // q_full (slot 0), kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final, v_tail,
+  // q_full (slot 1)
+  static constexpr int NUM_BARS = 1 + 2 * NS + 9;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * C::NS + k); };
   const uint32_t bar_final = bars + 8 * (7 + 2 * C::NS);
   const uint32_t bar_vtail = bars + 8 * (8 + 2 * C::NS);
+  const uint32_t bar_q1 = bars + 8 * (9 + 2 * C::NS);   // slot 1's Q tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     }
     mbar_init(bar_final, 1);
     mbar_init(bar_vtail, 1);
+    mbar_init(bar_q1, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -300,17 +303,24 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
-      const int nq = (n_kv[0] > 0) + (n_kv[1] > 0);
-      mbar_arrive_expect_tx(bar_q, nq * C::TILE_BYTES);
-      auto load_q = [&](int k, int h, int t) {
+      // slot 0's Q first (its first S needs only Q0 and K0); slot 1's Q
+      // follows K0 in the loop below
+      if (n_kv[0] > 0) {
+        mbar_arrive_expect_tx(bar_q, C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(q_s + k * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tm_q, bar_q, c * 64, h,
-                      s0 + t * C::BM);
-      };
-      if (n_kv[0] > 0) load_q(0, head[0], qtile[0]);
-      if (n_kv[1] > 0) load_q(1, head[1], qtile[1]);
+          tma_load_3d(q_s + c * C::CHUNK_BYTES, &p.tm_q, bar_q, c * 64, head[0], s0 + qtile[0] * C::BM);
+      }
     }
+    auto load_q1 = [&] {
+      if (lane == 0 && n_kv[1] > 0) {
+        mbar_arrive_expect_tx(bar_q1, C::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_3d(q_s + C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tm_q, bar_q1, c * 64, head[1],
+                      s0 + qtile[1] * C::BM);
+      }
+    };
     const int32_t* bt_row = p.block_table + static_cast<size_t>(seq) * p.max_pages;
     const int tail_tile = (Lk % kPrefillPage != 0) ? (Lk - 1) / C::BN - kt0 : -1;   // split-relative
     int pg_base = -1, pg_mine = 0, issued = 0, tail_item = -1;
@@ -356,6 +366,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
           ok = false;
         }
       }
+      if (item == 0) load_q1();
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
     }
     tail_item = __shfl_sync(0xffffffffu, tail_item, 0);
@@ -393,16 +404,15 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
-      const int nq = (n_kv[0] > 0) + (n_kv[1] > 0);
-      mbar_arrive_expect_tx(bar_q, nq * C::TILE_BYTES);
-      auto load_q = [&](int k, int h, int t) {
+      // slot 0's Q, then K0, then slot 1's Q: the first S needs only Q0 and K0
+      auto load_q = [&](int k, int h, int t, uint32_t bar) {
+        mbar_arrive_expect_tx(bar, C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(q_s + k * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tm_q, bar_q, c * 64, h,
+          tma_load_3d(q_s + k * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tm_q, bar, c * 64, h,
                       s0 + t * C::BM);
       };
-      if (n_kv[0] > 0) load_q(0, head[0], qtile[0]);
-      if (n_kv[1] > 0) load_q(1, head[1], qtile[1]);
+      if (n_kv[0] > 0) load_q(0, head[0], qtile[0], bar_q);
       int issued = 0;
       for (int item = 0; item < 2 * n_max; ++item) {
         if (!mbar_wait(bar_kv_empty(item), ((item / C::NS) & 1) ^ 1, abort_flag)) break;
@@ -413,6 +423,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
         for (int c = 0; c < C::CHUNKS; ++c)
           tma_load_3d(kv_s(item) + c * C::CHUNK_BYTES, map, bar_kv_full(item), c * 64, kv_head, row);
         ++issued;
+        if (item == 0 && n_kv[1] > 0) load_q(1, head[1], qtile[1], bar_q1);
       }
       if (*abort_flag) {
         volatile int never = 0;
@@ -462,10 +473,14 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
           tc_commit(bar_s_full(0));
         }
         if (nkv1 > 0) {
-          issue_qk(1, 0);
-          tc_commit(bar_s_full(1));
+          ok = mbar_wait(bar_q1, 0, abort_flag);
+          if (ok) {
+            tc_fence_after_sync();
+            issue_qk(1, 0);
+            tc_commit(bar_s_full(1));
+          }
         }
-        tc_commit(bar_kv_empty(0));
+        if (ok) tc_commit(bar_kv_empty(0));
       }
       // One slot's step at key tile j: O_k += P_k V_j, then S_k(j+1).
       // S_k(j+1) overwrites the columns P_k(j) occupies; the PV MMA that reads
