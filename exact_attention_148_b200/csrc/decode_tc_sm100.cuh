@@ -27,8 +27,8 @@
 // in E4M3's normal range.  Scores and outputs add the hi and lo columns.
 //
 // Roles (6 warps): warp 0 TMA producer (Q for bf16, then K and V of each
-// 128-key tile: two 64-token pages through the block table), warp 1 TMEM
-// owner and MMA issuer, warps 2-5 softmax and epilogue.
+// 128-key tile: two 64-token pages through the block table, as separate ring
+// items), warp 1 TMEM owner and MMA issuer, warps 2-5 softmax and epilogue.
 #pragma once
 
 #include "decode_sm100.cuh"
@@ -47,26 +47,30 @@ struct DecodeTcCfg {
   static constexpr int NB = KV8 ? 2 * NPAD : NPAD;       // operand rows / accumulator columns
   static constexpr int CHUNKS = D * ELEM / 128;          // 128-byte column chunks per K/V row
   static constexpr int KV_BYTES = KEYS * D * ELEM;       // one K or V tile
-  static constexpr int STAGES = 3;
+  // Ring of K and V tiles as separate items (K_0, V_0, K_1, ...).  With 8
+  // padded rows: 96 KB for either type, two CTAs per SM hiding each other's
+  // fill/drain.  With 16 the softmax of a tile takes longer and needs the
+  // deeper look-ahead of a 192 KB ring (one CTA per SM); measured on B200.
+  static constexpr int CTAS_PER_SM = NPAD == 8 ? 2 : 1;
+  static constexpr int ITEMS = (CTAS_PER_SM == 2 ? 96 : 192) * 1024 / KV_BYTES;
   static constexpr int Q_BYTES = NB * 128 * CHUNKS;      // Q^T operand
   static constexpr int P_CHUNKS = KEYS * ELEM / 128;     // 128-byte key chunks per P^T row
   static constexpr int P_BYTES = NB * 128 * P_CHUNKS;    // one P^T operand
-  static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = STAGES * KV_BYTES;
-  static constexpr int Q_OFF = 2 * STAGES * KV_BYTES;
+  static constexpr int RING_OFF = 0;
+  static constexpr int Q_OFF = ITEMS * KV_BYTES;
   static constexpr int P_OFF = Q_OFF + ((Q_BYTES + 1023) / 1024) * 1024;
   static constexpr int P_STRIDE = ((P_BYTES + 1023) / 1024) * 1024;
   static constexpr int RED_OFF = P_OFF + 2 * P_STRIDE;   // [2][NPAD][4] tile maxima
   static constexpr int SCL_OFF = RED_OFF + 2 * NPAD * 4 * 4;   // [NPAD] per-head score multipliers
   static constexpr int LRED_OFF = SCL_OFF + NPAD * 4;    // [NPAD][4] normaliser partials
   static constexpr int BAR_OFF = LRED_OFF + NPAD * 4 * 4;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], v_tail, final
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 8;
+  // q_full, kv_full[ITEMS], kv_empty[ITEMS], s_full[2], p_full[2], o_done[2], v_tail, final
+  static constexpr int NUM_BARS = 1 + 2 * ITEMS + 8;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 128;             // S^T x2 + O^T: 3 * NB <= 96
   static_assert(3 * NB <= static_cast<int>(TMEM_COLS), "TMEM budget");
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(SMEM_BYTES <= (CTAS_PER_SM == 2 ? 113 : 227) * 1024, "shared memory per CTA");
 };
 
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major) {
@@ -195,7 +199,7 @@ __device__ __forceinline__ int xpose32_base(int lane) {
 }
 
 template <bool KV8, int NPAD>
-__global__ void __launch_bounds__(kDecodeTcThreads, 1)
+__global__ void __launch_bounds__(kDecodeTcThreads, NPAD == 8 ? 2 : 1)
     fa_decode_tc_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecodeTcCfg<KV8, NPAD>;
   constexpr int D = C::D;
@@ -249,19 +253,22 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
 
   const uint32_t bars = base + C::BAR_OFF;
   const uint32_t bar_q = bars;
-  auto bar_kv_full = [&](int i) { return bars + 8 * (1 + i % C::STAGES); };
-  auto bar_kv_empty = [&](int i) { return bars + 8 * (1 + C::STAGES + i % C::STAGES); };
-  auto bar_s_full = [&](int k) { return bars + 8 * (1 + 2 * C::STAGES + k); };
-  auto bar_p_full = [&](int k) { return bars + 8 * (3 + 2 * C::STAGES + k); };
-  auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * C::STAGES + k); };
-  const uint32_t bar_vtail = bars + 8 * (7 + 2 * C::STAGES);
-  const uint32_t bar_final = bars + 8 * (8 + 2 * C::STAGES);
+  // ring item it = 2 * tile + (0: K, 1: V), slot it % ITEMS
+  auto bar_kv_full = [&](int it) { return bars + 8 * (1 + it % C::ITEMS); };
+  auto bar_kv_empty = [&](int it) { return bars + 8 * (1 + C::ITEMS + it % C::ITEMS); };
+  auto item_par = [&](int it) { return static_cast<uint32_t>((it / C::ITEMS) & 1); };
+  auto item_s = [&](int it) { return base + C::RING_OFF + (it % C::ITEMS) * C::KV_BYTES; };
+  auto bar_s_full = [&](int k) { return bars + 8 * (1 + 2 * C::ITEMS + k); };
+  auto bar_p_full = [&](int k) { return bars + 8 * (3 + 2 * C::ITEMS + k); };
+  auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * C::ITEMS + k); };
+  const uint32_t bar_vtail = bars + 8 * (7 + 2 * C::ITEMS);
+  const uint32_t bar_final = bars + 8 * (8 + 2 * C::ITEMS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, KV8 ? 4 : 1);
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < C::ITEMS; ++i) {
       mbar_init(bar_kv_full(i), 1);
       mbar_init(bar_kv_empty(i), 1);
     }
@@ -301,11 +308,14 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
       }
     }
     const int32_t* bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages + page_begin;
-    // The split's last page ends inside the page only at the cache end.
+    // The split's last page ends inside the page only at the cache end; that
+    // tile's V item lands on its own barrier, the warp zeroes its rows past
+    // the cache end (0 * NaN would otherwise reach O), then marks it full.
     const int tail_tile = (t_end % kDecodePage != 0) ? n_tiles - 1 : -1;
-    int pg_base = -1, pg_mine = 0, issued = 0;
-    bool tail_issued = false, ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
+    int pg_base = -1, pg_mine = 0, issued = 0, tail_item = -1;
+    bool ok = true;
+    for (int it = 0; it < 2 * n_tiles; ++it) {
+      const int i = it >> 1;
       const int lp0 = 2 * i;                        // split-relative logical page
       if ((lp0 & ~31) != pg_base) {
         pg_base = lp0 & ~31;
@@ -323,18 +333,11 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
       const int ph0 = __shfl_sync(0xffffffffu, pg_mine, lp0 & 31);
       const int ph1 = __shfl_sync(0xffffffffu, pg_mine, (lp0 + 1) & 31);
       if (lane == 0) {
-        if (mbar_wait(bar_kv_empty(i), ((i / C::STAGES) & 1) ^ 1, abort_flag)) {
-          const bool vtail = (i == tail_tile);
-          // K and V land on kv_full.  The tail tile's V lands on its own
-          // barrier instead, and kv_full's arrival waits until its rows past
-          // the cache end are zeroed (only K's bytes are expected here).
-          if (vtail) {
-            mbar_expect_tx(bar_kv_full(i), C::KV_BYTES);
-            mbar_arrive_expect_tx(bar_vtail, C::KV_BYTES);
-          } else {
-            mbar_arrive_expect_tx(bar_kv_full(i), 2 * C::KV_BYTES);
-          }
-          const int st = i % C::STAGES;
+        if (mbar_wait(bar_kv_empty(it), item_par(it) ^ 1, abort_flag)) {
+          const bool vtail = (it & 1) && i == tail_tile;
+          const uint32_t bar = vtail ? bar_vtail : bar_kv_full(it);
+          mbar_arrive_expect_tx(bar, C::KV_BYTES);
+          const CUtensorMap* map = (it & 1) ? &p.tm_v : &p.tm_k;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int phys = h ? ph1 : ph0;
@@ -342,32 +345,27 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
             const int c2 = (p.head_coord == 2) ? kv_head : (p.page_coord == 2 ? phys : 0);
             const int c3 = (p.head_coord == 3) ? kv_head : (p.page_coord == 3 ? phys : 0);
 #pragma unroll
-            for (int c = 0; c < C::CHUNKS; ++c) {
-              const uint32_t off = st * C::KV_BYTES + c * (C::KEYS * 128) + h * (kDecodePage * 128);
-              tma_load_4d(base + C::K_OFF + off, &p.tm_k, bar_kv_full(i), c * (128 / C::ELEM), c1, c2, c3);
-              tma_load_4d(base + C::V_OFF + off, &p.tm_v, vtail ? bar_vtail : bar_kv_full(i),
+            for (int c = 0; c < C::CHUNKS; ++c)
+              tma_load_4d(item_s(it) + c * (C::KEYS * 128) + h * (kDecodePage * 128), map, bar,
                           c * (128 / C::ELEM), c1, c2, c3);
-            }
           }
           ++issued;
-          if (vtail) tail_issued = true;
+          if (vtail) tail_item = it;
         } else {
           ok = false;
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
     }
-    // Cache end inside the last page: zero the V rows past it (0 * NaN would
-    // otherwise reach O), then release the tile's arrival on kv_full.
-    tail_issued = __shfl_sync(0xffffffffu, tail_issued, 0);
+    tail_item = __shfl_sync(0xffffffffu, tail_item, 0);
     bool tail_landed = true;
-    if (tail_issued) {
+    if (tail_item >= 0) {
       tail_landed = __all_sync(0xffffffffu, mbar_wait(bar_vtail, 0, abort_flag));
       if (tail_landed) {
-        const int i = n_tiles - 1;
+        const int i = tail_item >> 1;
         const int r0 = t_end - (t_begin + i * C::KEYS);
         const int r1 = ((t_end + kDecodePage - 1) / kDecodePage) * kDecodePage - (t_begin + i * C::KEYS);
-        uint4* tile = reinterpret_cast<uint4*>(smem + C::V_OFF + (i % C::STAGES) * C::KV_BYTES);
+        uint4* tile = reinterpret_cast<uint4*>(smem + C::RING_OFF + (tail_item % C::ITEMS) * C::KV_BYTES);
         const int per_chunk = (r1 - r0) * 8;
         for (int e = lane; e < C::CHUNKS * per_chunk; e += 32) {
           const int c = e / per_chunk, w = e % per_chunk;
@@ -375,14 +373,18 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         }
         fence_async_shared();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_kv_full(i));
+        if (lane == 0) mbar_arrive(bar_kv_full(tail_item));
       }
     }
     if (lane == 0 && *abort_flag) {
       volatile int never = 0;
-      for (int i = (issued > C::STAGES ? issued - C::STAGES : 0); i < issued; ++i)
-        mbar_wait(bar_kv_full(i), (i / C::STAGES) & 1, &never);
-      if (tail_issued && !tail_landed) mbar_wait(bar_vtail, 0, &never);
+      for (int it = (issued > C::ITEMS ? issued - C::ITEMS : 0); it < issued; ++it) {
+        if (it == tail_item) {
+          if (!tail_landed) mbar_wait(bar_vtail, 0, &never);
+        } else {
+          mbar_wait(bar_kv_full(it), item_par(it), &never);
+        }
+      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -392,12 +394,12 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
       constexpr int KSTEPS = D * C::ELEM / 32;       // 32-byte K steps over d
       constexpr int PSTEPS = C::KEYS * C::ELEM / 32; // 32-byte K steps over the keys
       auto issue_s = [&](int i) {
-        const uint32_t st = (i % C::STAGES) * C::KV_BYTES;
+        const uint32_t kt = item_s(2 * i);
         const uint32_t d_tmem = tmem + static_cast<uint32_t>((i & 1) * NB);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
           // 128-byte chunk kk/4, 32 bytes into it
-          const uint32_t a = base + C::K_OFF + st + (kk >> 2) * (C::KEYS * 128) + (kk & 3) * 32;
+          const uint32_t a = kt + (kk >> 2) * (C::KEYS * 128) + (kk & 3) * 32;
           const uint32_t bq = base + C::Q_OFF + (kk >> 2) * (NB * 128) + (kk & 3) * 32;
           const uint64_t ad = sdesc_sw128(a, 16, 1024), bd = sdesc_sw128(bq, 16, 1024);
           if constexpr (KV8) mma_e4m3_ss(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
@@ -405,39 +407,44 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         }
       };
       auto issue_pv = [&](int i) {
-        const uint32_t st = (i % C::STAGES) * C::KV_BYTES;
+        const uint32_t vt = item_s(2 * i + 1);
         const uint32_t o_tmem = tmem + static_cast<uint32_t>(2 * NB);
         const uint32_t pbuf = base + C::P_OFF + (i & 1) * C::P_STRIDE;
 #pragma unroll
         for (int kk = 0; kk < PSTEPS; ++kk) {
           // V^T, MN-major: 32 bytes of keys = 32 / ELEM keys per step, 128 bytes a key row;
           // the d direction crosses 128-byte chunks every KEYS * 128 bytes.
-          const uint32_t a = base + C::V_OFF + st + kk * (32 / C::ELEM) * 128;
+          const uint32_t a = vt + kk * (32 / C::ELEM) * 128;
           const uint32_t bp = pbuf + (kk >> 2) * (NB * 128) + (kk & 3) * 32;
           const uint64_t ad = sdesc_sw128(a, C::KEYS * 128, 1024), bd = sdesc_sw128(bp, 16, 1024);
           if constexpr (KV8) mma_e4m3_ss(o_tmem, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
           else mma_bf16_ss(o_tmem, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
         }
       };
+      // S_0, S_1, then per tile j: PV_j, S_{j+2}.  A K item is released
+      // once its S MMAs complete, a V item once its PV MMAs complete.
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       for (int i = 0; ok && i < 2 && i < n_tiles; ++i) {
-        if (!mbar_wait(bar_kv_full(i), (i / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar_kv_full(2 * i), item_par(2 * i), abort_flag)) { ok = false; break; }
         tc_fence_after_sync();
         issue_s(i);
         tc_commit(bar_s_full(i & 1));
+        tc_commit(bar_kv_empty(2 * i));
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         if (!mbar_wait(bar_p_full(j & 1), (j >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(bar_kv_full(2 * j + 1), item_par(2 * j + 1), abort_flag)) break;
         tc_fence_after_sync();
         issue_pv(j);
         tc_commit(bar_o_done(j & 1));
-        tc_commit(bar_kv_empty(j));
+        tc_commit(bar_kv_empty(2 * j + 1));
         const int n = j + 2;
         if (n < n_tiles) {
-          if (!mbar_wait(bar_kv_full(n), (n / C::STAGES) & 1, abort_flag)) break;
+          if (!mbar_wait(bar_kv_full(2 * n), item_par(2 * n), abort_flag)) break;
           tc_fence_after_sync();
           issue_s(n);
           tc_commit(bar_s_full(n & 1));
+          tc_commit(bar_kv_empty(2 * n));
         }
       }
       tc_commit(bar_final);

@@ -19,9 +19,9 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // cannot pull more than its ceiling, each CTA costs a fixed fill/drain time,
 // and a second (merge) launch costs ~5 us.  Per kernel (CTA ceiling, fill,
 // CTAs per SM): CUDA cores 44 GB/s, 0.5 us, 2 (1 with 8 packed heads; its
-// E4M3 ring holds as many bytes as the bf16 one); tensor cores, bf16 50 GB/s,
-// 3 us (10 us with 16 padded heads), 1 (192 KB ring); tensor cores, E4M3
-// 30 GB/s, 2 us (7 us with 16 padded heads), 2.
+// E4M3 ring holds as many bytes as the bf16 one); tensor cores with 8 padded
+// rows (96 KB ring of K and V tiles) 30 GB/s, 2 us, 2; with 16 padded rows
+// (192 KB ring) 50 GB/s, 10 us, 1 for bf16 and 30 GB/s, 7 us, 1 for E4M3.
 constexpr double kHbmBytesPerUs148 = 6.9e6;       // bytes per microsecond, 148 SMs
 constexpr double kMergeLaunchUs = 5.0;
 
@@ -33,9 +33,10 @@ struct CtaModel {
 
 CtaModel cta_model(bool tensor_cores, int kv_elem_bytes, int heads_per_cta) {
   if (tensor_cores) {
-    const bool wide = heads_per_cta > 8;   // 16 padded heads
-    return kv_elem_bytes == 1 ? CtaModel{3.0e4, wide ? 7.0 : 2.0, 2}
-                              : CtaModel{5.0e4, wide ? 10.0 : 3.0, 1};
+    // 8 padded rows: 96 KB ring, two CTAs per SM; 16: 192 KB ring, one
+    const bool wide = heads_per_cta > 8;
+    if (!wide) return CtaModel{3.0e4, 2.0, 2};
+    return kv_elem_bytes == 1 ? CtaModel{3.0e4, 7.0, 1} : CtaModel{5.0e4, 10.0, 1};
   }
   return {4.36e4, 0.5, heads_per_cta == 8 ? 1 : 2};
 }
