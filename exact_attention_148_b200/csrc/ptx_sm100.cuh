@@ -94,11 +94,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // by limit_ns; on expiry record FA_ERR_TIMEOUT and return.
 __global__ void fa_selftest_wait_kernel(unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int abort_flag;
   const uint32_t b = smem_addr(&bar);
   if (threadIdx.x == 0) {
     mbar_init(b, 1);
-    abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();

@@ -32,7 +32,13 @@ Readings taken where the pages are silent (each also listed in the design doc):
   mask keeps the same rule as a full prefill of the whole sequence);
 * KV append: the chunk's n new K/V rows take logical positions
   cache_seqlens[b] - n ... cache_seqlens[b] - 1 of their request and are
-  written through the page table (same page, section 2).
+  written through the page table (same page, section 2);
+* multi-token decode (several query tokens per request) is the chunked
+  prefill rule applied to a decode step: the tokens are the last q_len
+  positions of the cache;
+* cascade (prefix sharing, wsisp.com "FIA / FlashAttention", section 三): a
+  request's keys are the shared prefix followed by its own suffix, and the
+  result is plain attention over that concatenation.
 
 Split/merge (Flash-Decoding, "Flash Attention & Paged Attention", section
 "FA对decode阶段的影响", steps 3-4): each split yields a partial (O_i, LSE_i)
