@@ -494,22 +494,28 @@ def oracle_prefill_sample(inp: W.PrefillInputs, budget_s: float):
     order = np.argsort(inp.seqlens)          # shortest sequences first
     flops, secs, done = 0.0, 0.0, []
     d = inp.head_dim
-    for b in order:
-        s0, s1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
-        L = s1 - s0
-        g = 0
-        q = W.as_f64(inp.q_bits[s0:s1, 0:1])
-        k = W.as_f64(inp.k_bits[s0:s1, g:g + 1])
-        v = W.as_f64(inp.v_bits[s0:s1, g:g + 1])
-        t0 = time.perf_counter()
-        oracle.attention_ref(q, k, v, [0, L], inp.causal, inp.scale)
-        secs += time.perf_counter() - t0
-        pairs = L * (L + 1) // 2 if inp.causal else L * L
-        flops += 4.0 * d * pairs
-        done.append(L)
+    G = inp.num_q_heads // inp.num_kv_heads
+    for h in range(inp.num_q_heads):         # one (sequence, head) block at a time
+        for b in order:
+            s0, s1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
+            L = s1 - s0
+            g = h // G
+            q = W.as_f64(inp.q_bits[s0:s1, h:h + 1])
+            k = W.as_f64(inp.k_bits[s0:s1, g:g + 1])
+            v = W.as_f64(inp.v_bits[s0:s1, g:g + 1])
+            t0 = time.perf_counter()
+            oracle.attention_ref(q, k, v, [0, L], inp.causal, inp.scale)
+            secs += time.perf_counter() - t0
+            pairs = L * (L + 1) // 2 if inp.causal else L * L
+            flops += 4.0 * d * pairs
+            done.append((h, L))
+            if secs >= budget_s:
+                break
         if secs >= budget_s:
             break
-    return flops, secs, f"oracle attention_ref on head 0 of sequences with lengths {done}"
+    heads = sorted({h for h, _ in done})
+    return flops, secs, (f"oracle attention_ref on {len(done)} (sequence, head) blocks, heads "
+                         f"{heads[0]}-{heads[-1]}, sequence lengths {sorted({L for _, L in done})}")
 
 
 def oracle_decode_sample(inp: W.DecodeInputs, budget_s: float):
