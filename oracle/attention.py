@@ -14,7 +14,7 @@ contrast with tiling: "Flash Attention & Paged Attention", section 1 pseudocode)
 and the softmax is summed explicitly.  No tiling, no online softmax, no
 reordering: this is the thing the tiled kernels must reproduce.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
 
 * causal: key j is allowed for query i iff j <= i, both counted from the start
   of their sequence (one ``cu_seqlens`` for q and k, so q and k lengths match);

@@ -13,7 +13,7 @@ e with bias 7, 3 mantissa bits m, no infinities,
 
 so the largest finite magnitude is 448 (e = 15, m = 6).
 
-Reading taken for the quantised KV cache (listed in the design doc): one scale per
+Reading taken for the quantised KV cache: one scale per
 tensor, k = k_scale * E4M3(k8), v = v_scale * E4M3(v8); the query stays bf16.
 """
 from __future__ import annotations
