@@ -62,7 +62,8 @@ typedef enum { FA_KV_BF16 = 0, FA_KV_E4M3 = 1 } fa_kv_dtype;
 typedef enum {
   FA_DECODE_AUTO = 0,          /* the planner chooses */
   FA_DECODE_CUDA_CORES = 1,    /* fp32 FMAs per element, up to 8 heads per CTA */
-  FA_DECODE_TENSOR_CORES = 2   /* tcgen05 MMAs, all G <= 16 heads of a kv head per CTA; d = 128 */
+  FA_DECODE_TENSOR_CORES = 2   /* tcgen05 MMAs, all G heads (x q_len tokens, <= 16 rows) of a kv
+                                  head per CTA; d = 128 */
 } fa_decode_kernel;
 
 /* Read-only view of a plan (for tests and tools). */
