@@ -84,6 +84,24 @@ int ensure_smem(const void* kernel, int bytes) {
   return FA_OK;
 }
 
+// SM count of the current device, queried once per device.
+int sm_count(int* out) {
+  constexpr int kMaxDev = 128;
+  static std::mutex mu;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDev) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int n = 0;
+    FA_CUDA_CHECK(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev));
+    cached[dev] = n;
+  }
+  *out = cached[dev];
+  return FA_OK;
+}
+
 float resolve_scale(float scale, int head_dim) {
   return std::isnan(scale) ? 1.0f / std::sqrt(static_cast<float>(head_dim)) : scale;
 }
@@ -408,10 +426,10 @@ FA_API int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_
   ap.num_kv_heads = num_kv_heads;
   ap.max_pages = max_pages_per_seq;
   ap.num_pages = static_cast<int>(num_pages);
-  // One warp per token; at most 16 resident blocks per SM's worth of grid.
-  int dev = 0, sms = 148;
-  FA_CUDA_CHECK(cudaGetDevice(&dev));
-  FA_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  // One warp per token; a grid of at most 8 blocks per SM loops over the rest.
+  int sms = 0;
+  const int st = sm_count(&sms);
+  if (st != FA_OK) return st;
   const int64_t want = (static_cast<int64_t>(total_new) + 7) / 8;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
