@@ -41,7 +41,8 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
-PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill"}
+PREFILL_WORKLOADS = {"varlen_causal_prefill", "long_gqa_prefill", "tiny_causal_prefill",
+                     "varlen_causal_prefill_fp8"}
 DECODE_WORKLOADS = {"paged_decode_batch", "long_split_decode", "ragged_split_decode",
                     "paged_decode_batch16", "paged_decode_batch_fp8", "paged_decode_gqa8",
                     "paged_decode_gqa16", "speculative_decode_batch"}
@@ -126,38 +127,49 @@ class PrefillCase:
     def __init__(self, inp: W.PrefillInputs, device):
         import torch
         self.inp = inp
-        self.q = _dev_bf16(inp.q_bits, device)
-        self.k = _dev_bf16(inp.k_bits, device)
-        self.v = _dev_bf16(inp.v_bits, device)
+        self.fp8 = isinstance(inp, W.Fp8PrefillInputs)
+        if self.fp8:
+            self.q, self.k, self.v = (torch.from_numpy(x).to(device) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+            self.h_q, self.h_k, self.h_v = (torch.from_numpy(x).pin_memory()
+                                            for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+        else:
+            self.q = _dev_bf16(inp.q_bits, device)
+            self.k = _dev_bf16(inp.k_bits, device)
+            self.v = _dev_bf16(inp.v_bits, device)
+            # pinned host copies for the end-to-end leg
+            self.h_q, self.h_k, self.h_v = (torch.from_numpy(x.view(np.int16)).pin_memory()
+                                            for x in (inp.q_bits, inp.k_bits, inp.v_bits))
         self.cu = _dev_i32(inp.cu_seqlens, device)
-        self.out = torch.empty_like(self.q)
+        self.out = torch.empty(self.q.shape, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=device)
         self.flops = inp.causal_flops()
         self.launches = -(-sum(-(-int(L) // 128) for L in inp.seqlens) // 2048)
-        # pinned host copies for the end-to-end leg
-        self.h_q = torch.from_numpy(inp.q_bits.view(np.int16)).pin_memory()
-        self.h_k = torch.from_numpy(inp.k_bits.view(np.int16)).pin_memory()
-        self.h_v = torch.from_numpy(inp.v_bits.view(np.int16)).pin_memory()
         self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
         self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
 
     def run(self):
         import exact_attention_148_b200 as fa
-        fa.prefill(self.q, self.k, self.v, self.cu, causal=self.inp.causal, scale=self.inp.scale,
-                   out=self.out, lse=self.lse, cu_seqlens_host=self.inp.cu_seqlens)
+        i = self.inp
+        if self.fp8:
+            fa.prefill_fp8(self.q, self.k, self.v, self.cu, q_scale=i.q_scale, k_scale=i.k_scale,
+                           v_scale=i.v_scale, causal=i.causal, scale=i.scale, out=self.out,
+                           lse=self.lse, cu_seqlens_host=i.cu_seqlens)
+        else:
+            fa.prefill(self.q, self.k, self.v, self.cu, causal=i.causal, scale=i.scale,
+                       out=self.out, lse=self.lse, cu_seqlens_host=i.cu_seqlens)
 
     def run_e2e(self):
         """Host buffers in, host buffers out: H2D copies, the C-ABI call, D2H copies."""
         import torch
-        self.q.view(torch.int16).copy_(self.h_q, non_blocking=True)
-        self.k.view(torch.int16).copy_(self.h_k, non_blocking=True)
-        self.v.view(torch.int16).copy_(self.h_v, non_blocking=True)
+        for d, h in ((self.q, self.h_q), (self.k, self.h_k), (self.v, self.h_v)):
+            (d if self.fp8 else d.view(torch.int16)).copy_(h, non_blocking=True)
         self.run()
         self.h_out.copy_(self.out.view(torch.int16), non_blocking=True)
         self.h_lse.copy_(self.lse, non_blocking=True)
 
     def h2d_bytes(self):
-        return 2 * (self.inp.q_bits.size + self.inp.k_bits.size + self.inp.v_bits.size) + \
+        eb = 1 if self.fp8 else 2
+        return eb * (self.inp.q_bits.size + self.inp.k_bits.size + self.inp.v_bits.size) + \
             4 * self.inp.cu_seqlens.size
 
     def d2h_bytes(self):
@@ -168,6 +180,7 @@ class PrefillCase:
         return {"workload": i.name, "batch": int(len(i.seqlens)), "seqlens_total": int(i.seqlens.sum()),
                 "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads,
                 "head_dim": i.head_dim, "causal": bool(i.causal),
+                "inputs": "e4m3 q/k/v, per-tensor scales" if self.fp8 else "bf16",
                 "algorithmic_tflop": round(self.flops / 1e12, 4)}
 
 
@@ -500,9 +513,14 @@ def oracle_prefill_sample(inp: W.PrefillInputs, budget_s: float):
             s0, s1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
             L = s1 - s0
             g = h // G
-            q = W.as_f64(inp.q_bits[s0:s1, h:h + 1])
-            k = W.as_f64(inp.k_bits[s0:s1, g:g + 1])
-            v = W.as_f64(inp.v_bits[s0:s1, g:g + 1])
+            if isinstance(inp, W.Fp8PrefillInputs):
+                q = oracle.dequantize_e4m3(inp.q_bits[s0:s1, h:h + 1], inp.q_scale)
+                k = oracle.dequantize_e4m3(inp.k_bits[s0:s1, g:g + 1], inp.k_scale)
+                v = oracle.dequantize_e4m3(inp.v_bits[s0:s1, g:g + 1], inp.v_scale)
+            else:
+                q = W.as_f64(inp.q_bits[s0:s1, h:h + 1])
+                k = W.as_f64(inp.k_bits[s0:s1, g:g + 1])
+                v = W.as_f64(inp.v_bits[s0:s1, g:g + 1])
             t0 = time.perf_counter()
             oracle.attention_ref(q, k, v, [0, L], inp.causal, inp.scale)
             secs += time.perf_counter() - t0
@@ -675,14 +693,20 @@ def aggregate_throughput(work_per_replica: float, ms_max: float, n_replicas: int
     return n_replicas * work_per_replica / (ms_max * 1e-3) / scale
 
 
-def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=None):
+def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=None, fp8_qk=False):
     if kind == "tensor":
         achieved = algorithmic / (ms_per_launch * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
+        src = f"{peak_src} bf16 dense (burst)"
+        spec = SPEC_PEAKS["bf16_tflops"]
+        if fp8_qk:
+            # half the FLOPs (Q K^T) at the E4M3 rate, nominally 2x bf16, the
+            # other half (P V, f16) at the bf16 rate: 2 / (1/2 + 1) = 4/3
+            peak, spec = round(peak * 4.0 / 3.0, 1), spec * 4.0 / 3.0
+            src += " x 4/3 (Q K^T at the fp8 rate = 2 x bf16 nominal, P V at the f16 rate)"
         return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 dense (burst)",
-                "frac_of_spec": round(achieved / SPEC_PEAKS["bf16_tflops"], 4)}
+                "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
+                "frac_of_spec": round(achieved / spec, 4)}
     achieved = algorithmic / (ms_per_launch * 1e-3) / 1e9
     peak = peaks["hbm_gbs"]
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -724,8 +748,8 @@ def run_ours(args):
     for c, ms in zip(cases, ms_case):
         if isinstance(c, PrefillCase):
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
-                               measured_traffic("prefill", c.inp.name))
-            e["kernel"] = "fa_prefill_pp_kernel<%d>" % c.inp.head_dim
+                               measured_traffic("prefill", c.inp.name), fp8_qk=c.fp8)
+            e["kernel"] = "fa_prefill_pp_kernel<%d%s>" % (c.inp.head_dim, ", e4m3" if c.fp8 else "")
         elif isinstance(c, ChunkedAttnCase):
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
                                measured_traffic("prefill", c.inp.name))
@@ -765,7 +789,8 @@ def run_ours(args):
     rl = rooflines[int(np.argmax(ms_case))]
     line.update({"value": round(value, 3), "unit": unit, "n_gpus": N, "steps": args.steps,
                  "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
-                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                 "scaling": "weak", "vs_baseline": None,
+                 "dtype": "e4m3 in, fp32 accumulate" if getattr(main, "fp8", False) else "bf16",
                  "data": "synthetic (seeded N(0,1) rounded to bf16; see workloads/)"})
     cfg = {"workload": cases[1].inp.name + " (append + chunked prefill)" if chunked else
            " + ".join(c.inp.name for c in cases),

@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
     "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
-    "append_kv", "prefill_paged", "decode_paged_fp8", "cascade_decode", "cascade_workspace_bytes",
+    "append_kv", "prefill_paged", "prefill_fp8", "decode_paged_fp8", "cascade_decode", "cascade_workspace_bytes",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +40,7 @@ EXPORTED_SYMBOLS = [
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
     "fa_decode_paged_fp8", "fa_decode_plan_kv", "fa_decode_plan_ex", "fa_cascade_workspace_bytes",
-    "fa_cascade_decode",
+    "fa_cascade_decode", "fa_prefill_fp8",
 ]
 
 FA_KV_BF16, FA_KV_E4M3 = 0, 1
@@ -92,6 +92,9 @@ def library() -> ctypes.CDLL:
     vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
     L.fa_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp]
     L.fa_prefill.restype = i32
+    L.fa_prefill_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32,
+                                 vp, vp, vp]
+    L.fa_prefill_fp8.restype = i32
     L.fa_decode_plan.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                  ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t)]
     L.fa_decode_plan.restype = i32
@@ -209,6 +212,38 @@ def prefill(q, k, v, cu_seqlens, *, causal: bool = True, scale: float | None = N
                               1 if causal else 0, _scale_arg(scale), _ptr(out), _ptr(lse),
                               _stream_ptr(stream))
     _check(st, "fa_prefill")
+    return out, lse
+
+
+def prefill_fp8(q, k, v, cu_seqlens, *, q_scale: float, k_scale: float, v_scale: float,
+                causal: bool = True, scale: float | None = None, out=None, lse=None,
+                cu_seqlens_host=None, return_lse: bool = True, stream=None):
+    """``prefill`` over E4M3 inputs: q [T, Hq, 128], k/v [T, Hkv, 128] uint8
+    (or float8_e4m3fn) tensors of E4M3 codes, dequantised as q_scale * q8,
+    k_scale * k8 and v_scale * v8.  Returns (out [T, Hq, 128] bf16, lse fp32)."""
+    torch = _torch()
+    _require_cuda(q, k, v, cu_seqlens, out, lse)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.element_size() != 1 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous 3-D tensor of one-byte E4M3 codes")
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu().numpy()
+    cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+    batch = len(cu_h) - 1
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    st = library().fa_prefill_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                  cu_h.ctypes.data_as(ctypes.c_void_p), batch, Hq, Hkv, d,
+                                  1 if causal else 0, _scale_arg(scale), float(q_scale),
+                                  float(k_scale), float(v_scale), _ptr(out), _ptr(lse),
+                                  _stream_ptr(stream))
+    _check(st, "fa_prefill_fp8")
     return out, lse
 
 

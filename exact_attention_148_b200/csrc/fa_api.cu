@@ -110,12 +110,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------- prefill
 // groups: (sequence << 16 | kv head, number of CTAs) in launch order.
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool F8 = false>
 int launch_prefill(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t, int>>& groups,
                    cudaStream_t stream) {
-  constexpr int kSmem = fa::PrefillPPCfg<D>::SMEM_BYTES;
-  constexpr int kThreads = fa::kPrefillPPThreads;
-  auto kernel = fa::fa_prefill_pp_kernel<D, PAGED>;
+  constexpr int kSmem = fa::PrefillPPCfg<D, F8>::SMEM_BYTES;
+  constexpr int kThreads = fa::PrefillPPCfg<D, F8>::THREADS;
+  auto kernel = fa::fa_prefill_pp_kernel<D, PAGED, F8>;
   int st = ensure_smem(reinterpret_cast<const void*>(kernel), kSmem);
   if (st != FA_OK) return st;
   for (size_t off = 0; off < groups.size(); off += fa::kPrefillMaxGroups) {
@@ -252,10 +252,17 @@ int launch_merge(const fa::MergeParams& mp, int head_dim, cudaStream_t stream) {
 
 // ============================================================================ API
 
-FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
-                      const int32_t* cu_seqlens_host, int batch, int num_q_heads, int num_kv_heads,
-                      int head_dim, int causal, float scale, void* out, float* lse, void* stream) {
+namespace {
+
+// fa_prefill and fa_prefill_fp8 (f8: E4M3 Q/K/V with per-tensor scales).
+int prefill_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
+                 const int32_t* cu_seqlens_host, int batch, int num_q_heads, int num_kv_heads,
+                 int head_dim, int causal, float scale, bool f8, float q_scale, float k_scale,
+                 float v_scale, void* out, float* lse, void* stream) {
   if (!q || !k || !v || !cu_seqlens_dev || !cu_seqlens_host || !out) return FA_ERR_INVALID_ARG;
+  if (f8 && head_dim != 128) return FA_ERR_UNSUPPORTED;
+  for (float sc : {q_scale, k_scale, v_scale})
+    if (!(sc > 0.0f) || std::isinf(sc)) return FA_ERR_INVALID_ARG;
   if (batch < 1 || batch > 65535 || num_q_heads < 1 || num_kv_heads < 1 ||
       num_q_heads > 65535 || num_q_heads % num_kv_heads != 0)
     return FA_ERR_INVALID_ARG;
@@ -282,23 +289,26 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
 
   static thread_local fa::PrefillParams prm;   // ~17 KB; kept off the stack
   std::memset(&prm, 0, sizeof(prm));
-  const cuuint32_t box[3] = {64, 1, 128};
+  // 128-byte boxes: 64 bf16 columns, or all 128 E4M3 columns, of 128 rows
+  const int eb = f8 ? 1 : 2;
+  const CUtensorMapDataType dt = f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 1, 128};
   {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
                                 static_cast<cuuint64_t>(T)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
-                                   static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
-    int st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * eb,
+                                   static_cast<cuuint64_t>(num_q_heads) * head_dim * eb};
+    int st = encode_map(&prm.tm_q, q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, dt);
     if (st != FA_OK) return st;
   }
   {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),
                                 static_cast<cuuint64_t>(T)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
-                                   static_cast<cuuint64_t>(num_kv_heads) * head_dim * 2};
-    int st = encode_map(&prm.tm_k, k, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * eb,
+                                   static_cast<cuuint64_t>(num_kv_heads) * head_dim * eb};
+    int st = encode_map(&prm.tm_k, k, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, dt);
     if (st != FA_OK) return st;
-    st = encode_map(&prm.tm_v, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = encode_map(&prm.tm_v, v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, dt);
     if (st != FA_OK) return st;
   }
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -307,10 +317,29 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
   prm.num_q_heads = num_q_heads;
   prm.group = group;
   prm.causal = causal ? 1 : 0;
-  prm.scale_log2 = scale * kLog2e;
+  prm.scale_log2 = scale * kLog2e * q_scale * k_scale;
+  prm.v_scale = v_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (f8) return launch_prefill<128, false, true>(prm, groups, s);
   return head_dim == 128 ? launch_prefill<128, false>(prm, groups, s)
                          : launch_prefill<64, false>(prm, groups, s);
+}
+
+}  // namespace
+
+FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
+                      const int32_t* cu_seqlens_host, int batch, int num_q_heads, int num_kv_heads,
+                      int head_dim, int causal, float scale, void* out, float* lse, void* stream) {
+  return prefill_impl(q, k, v, cu_seqlens_dev, cu_seqlens_host, batch, num_q_heads, num_kv_heads,
+                      head_dim, causal, scale, false, 1.0f, 1.0f, 1.0f, out, lse, stream);
+}
+
+FA_API int fa_prefill_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
+                          const int32_t* cu_seqlens_host, int batch, int num_q_heads,
+                          int num_kv_heads, int head_dim, int causal, float scale, float q_scale,
+                          float k_scale, float v_scale, void* out, float* lse, void* stream) {
+  return prefill_impl(q, k, v, cu_seqlens_dev, cu_seqlens_host, batch, num_q_heads, num_kv_heads,
+                      head_dim, causal, scale, true, q_scale, k_scale, v_scale, out, lse, stream);
 }
 
 FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,

@@ -74,6 +74,7 @@ struct PrefillParams {
   int total_q;
   float* part_o;
   float* part_lse;
+  float v_scale;             // E4M3 inputs: V dequantisation scale
   int max_pages;
   int num_pages;
   int head_coord;            // paged: tensor-map dimension (1..3) of the kv head
@@ -100,21 +101,31 @@ constexpr int kPrefillPPThreads = 320;
 #define FA_PREFILL_F16EX2_MASK 0x0
 #endif
 
-template <int D>
+// F8: Q, K and V are E4M3 bytes (one scale per tensor).  S = Q K^T runs as a
+// kind::f8f6f4 MMA on them as stored (exact products, half the tensor time of
+// bf16); P is kept as f16 and V is widened to f16 in shared memory by two
+// converter warps (E4M3 -> f16 is exact), so P V stays a kind::f16 MMA and
+// the softmax does no more work than with bf16 inputs.
+template <int D, bool F8 = false>
 struct PrefillPPCfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(!F8 || D == 128, "E4M3 inputs: head_dim 128");
+  static constexpr int ELEM = F8 ? 1 : 2;
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int CHUNKS = D / 64;
+  static constexpr int CHUNKS = D * ELEM / 128;            // 128-byte column chunks of a row
   static constexpr int CHUNK_BYTES = 128 * 128;
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
-  static constexpr int NS = (D == 128) ? 5 : 8;           // K/V ring slots
+  static constexpr int NS = F8 ? 8 : (D == 128) ? 5 : 8;   // K/V ring slots
   static constexpr int Q_OFF = 0;                          // two Q tiles
   static constexpr int KV_OFF = 2 * TILE_BYTES;
-  static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
+  static constexpr int VH_OFF = KV_OFF + NS * TILE_BYTES;  // F8: two f16 V tiles (2 chunks each)
+  static constexpr int VH_TILE = 2 * CHUNK_BYTES;
+  static constexpr int BAR_OFF = VH_OFF + (F8 ? 2 * VH_TILE : 0);
   // q_full (slot 0), kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final, v_tail,
-  // q_full (slot 1)
-  static constexpr int NUM_BARS = 1 + 2 * NS + 9;
+  // q_full (slot 1), F8: vh_full[2], vh_empty[2]
+  static constexpr int NUM_BARS = 1 + 2 * NS + 9 + (F8 ? 4 : 0);
+  static constexpr int THREADS = F8 ? 384 : 320;           // F8: + two converter warps
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -159,6 +170,40 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+__host__ __device__ constexpr uint32_t idesc_e4m3_k(int M, int N) {
+  // F32 accumulate, A and B E4M3 (format 0), both K-major
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
+  // F32 accumulate, A and B f16 (format 0)
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Four E4M3 bytes (low byte first) -> two f16x2 words (exact).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(w));
+}
+
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -171,10 +216,11 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
 
 constexpr int kPrefillPage = 64;
 
-template <int D, bool PAGED>
-__global__ void __launch_bounds__(kPrefillPPThreads, 1)
+template <int D, bool PAGED, bool F8 = false>
+__global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
     fa_prefill_pp_kernel(const __grid_constant__ PrefillParams p) {
-  using C = PrefillPPCfg<D>;
+  static_assert(!(F8 && PAGED), "E4M3 inputs: packed K/V only");
+  using C = PrefillPPCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -259,6 +305,8 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   const uint32_t bar_final = bars + 8 * (7 + 2 * C::NS);
   const uint32_t bar_vtail = bars + 8 * (8 + 2 * C::NS);
   const uint32_t bar_q1 = bars + 8 * (9 + 2 * C::NS);   // slot 1's Q tile
+  auto bar_vh_full = [&](int sl) { return bars + 8 * (10 + 2 * C::NS + sl); };
+  auto bar_vh_empty = [&](int sl) { return bars + 8 * (12 + 2 * C::NS + sl); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -266,12 +314,18 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     mbar_init(bar_q, 1);
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(bar_kv_full(i), 1);
-      mbar_init(bar_kv_empty(i), 1);
+      // F8: the V tiles (odd items, odd slots since NS is even) are released
+      // by the two converter warps, the K tiles by the MMA issuer
+      mbar_init(bar_kv_empty(i), (F8 && (i & 1)) ? 2 : 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s_full(k), 1);
       mbar_init(bar_p_full(k), 4);
       mbar_init(bar_o_done(k), 1);
+      if constexpr (F8) {
+        mbar_init(bar_vh_full(k), 2);
+        mbar_init(bar_vh_empty(k), 1);
+      }
     }
     mbar_init(bar_final, 1);
     mbar_init(bar_vtail, 1);
@@ -434,8 +488,8 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(C::BM, C::BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(C::BM, D, true);
+      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_k(C::BM, C::BN) : idesc_bf16_f32(C::BM, C::BN, false);
+      constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(C::BM, D, true) : idesc_bf16_f32(C::BM, D, true);
       // k is always a literal below, so per-slot values stay in registers.
       // This thread's issue rate is on the per-tile critical path (it shares
       // its SMSP with two softmax warps), so descriptors are built once and
@@ -443,22 +497,25 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       // units; no carry leaves the 14-bit field inside shared memory).
       const uint64_t q_desc = sdesc_sw128(q_s, 16, 1024);
       const uint64_t k_desc0 = sdesc_sw128(base + C::KV_OFF, 16, 1024);
-      const uint64_t v_desc0 = sdesc_sw128(base + C::KV_OFF, C::CHUNK_BYTES, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(base + (F8 ? C::VH_OFF : C::KV_OFF), C::CHUNK_BYTES, 1024);
       auto ring_off = [&](int item) { return static_cast<uint64_t>((item % C::NS) * (C::TILE_BYTES >> 4)); };
       auto issue_qk = [&](int k, int item) {
         const uint64_t qd = q_desc + (k ? (C::TILE_BYTES >> 4) : 0);
         const uint64_t kd = k_desc0 + ring_off(item);
         const uint32_t d_tmem = tmem + (k ? 128u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D * C::ELEM / 32; ++kk) {   // 32-byte K steps
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32) >> 4);
-          mma_bf16_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+          if constexpr (F8) mma_f8_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+          else mma_bf16_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int k, int item, bool accumulate) {
         const uint32_t o_tmem = tmem + 256u + (k ? D : 0);
         const uint32_t p_tmem = tmem + (k ? 128u : 0u);
-        const uint64_t vd = v_desc0 + ring_off(item);
+        // F8: the f16 copy of V_j in slot j & 1 (item = 2j + 1)
+        const uint64_t vd = F8 ? v_desc0 + static_cast<uint64_t>((((item >> 1) & 1) * C::VH_TILE) >> 4)
+                               : v_desc0 + ring_off(item);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
           mma_bf16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
@@ -500,16 +557,53 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
       for (int j = 0; ok && j < n_max; ++j) {
         const int v_item = 2 * j + 1, k_item = 2 * j + 2;
         const bool need_k = (j + 1 < nkv0) || (j + 1 < nkv1);
-        if (!mbar_wait(bar_kv_full(v_item), (v_item / C::NS) & 1, abort_flag)) break;
+        if (F8 ? !mbar_wait(bar_vh_full(j & 1), (j >> 1) & 1, abort_flag)
+               : !mbar_wait(bar_kv_full(v_item), (v_item / C::NS) & 1, abort_flag))
+          break;
         if (need_k && !mbar_wait(bar_kv_full(k_item), (k_item / C::NS) & 1, abort_flag)) break;
         ok = slot_step(0, nkv0, j, v_item, k_item) && slot_step(1, nkv1, j, v_item, k_item);
         if (!ok) break;
-        tc_commit(bar_kv_empty(v_item));
+        if constexpr (F8) tc_commit(bar_vh_empty(j & 1));
+        else tc_commit(bar_kv_empty(v_item));
         if (need_k) tc_commit(bar_kv_empty(k_item));
       }
       tc_commit(bar_final);
       volatile int never = 0;
       mbar_wait(bar_final, 0, &never);
+    }
+  } else if (F8 && warp >= 10) {
+    // ---------------------------------------------------------------- V converters
+    // Warp 10 widens keys 0-63 of V_j, warp 11 keys 64-127: each 16-byte
+    // E4M3 unit (16 columns of one key) becomes two 16-byte f16 units of the
+    // 128-byte-swizzled, two-chunk f16 tile the P V MMA reads.
+    const int half = warp - 10;
+    for (int j = 0; j < n_max; ++j) {
+      const int v_item = 2 * j + 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_kv_full(v_item), (v_item / C::NS) & 1, abort_flag))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_vh_empty(j & 1), ((j >> 1) & 1) ^ 1, abort_flag))) break;
+      const uint8_t* src = smem + C::KV_OFF + (v_item % C::NS) * C::TILE_BYTES;
+      uint8_t* dst = smem + C::VH_OFF + (j & 1) * C::VH_TILE;
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int e = lane + 32 * i;             // 0..511
+        const int key = half * 64 + (e >> 3), u = e & 7, sw = key & 7;
+        const uint4 b = *reinterpret_cast<const uint4*>(src + key * 128 + ((u ^ sw) << 4));
+        uint4 lo4, hi4;
+        e4m3x4_to_f16x4(b.x, lo4.x, lo4.y);
+        e4m3x4_to_f16x4(b.y, lo4.z, lo4.w);
+        e4m3x4_to_f16x4(b.z, hi4.x, hi4.y);
+        e4m3x4_to_f16x4(b.w, hi4.z, hi4.w);
+        const int c = u >> 2, w0 = 2 * (u & 3);   // f16 chunk and unit of columns 16u..16u+7
+        uint8_t* row = dst + c * C::CHUNK_BYTES + key * 128;
+        *reinterpret_cast<uint4*>(row + ((w0 ^ sw) << 4)) = lo4;
+        *reinterpret_cast<uint4*>(row + (((w0 + 1) ^ sw) << 4)) = hi4;
+      }
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_vh_full(j & 1));
+        mbar_arrive(bar_kv_empty(v_item));
+      }
     }
   } else {
     // ---------------------------------------------------------------- softmax warpgroups
@@ -597,7 +691,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
           }
           ps[i & 3].x += p0;
           ps[i & 3].y += p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          pk[i] = F8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
         }
         // P chunk c (16 packed columns) lands on S columns already in registers.
         tmem_st_x16(sc + c * 16, pk);
@@ -630,7 +724,7 @@ __global__ void __launch_bounds__(kPrefillPPThreads, 1)
     }
     if (nk > 0 && ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (nk - 1) & 1, abort_flag))) {
       tc_fence_after_sync();
-      const float inv_l = 1.0f / l_sum;
+      const float inv_l = F8 ? p.v_scale / l_sum : 1.0f / l_sum;
       const bool valid = q_row < L;
       __nv_bfloat16* orow =
           p.out + (static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head) * D;

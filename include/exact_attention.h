@@ -114,6 +114,29 @@ int fa_prefill(const void* q, const void* k, const void* v,
                void* out, float* lse, void* stream);
 
 /*
+ * fa_prefill_fp8 — fa_prefill over E4M3 inputs (FP8 inference kernels:
+ * wsisp.com "FIA / FlashAttention", section 三, FP8 row; the operation is
+ * fa_prefill's on the dequantised tensors).
+ *
+ *   q [T, Hq, 128], k, v [T, Hkv, 128]: E4M3 bytes (OCP FP8 E4M3), same
+ *       layouts as fa_prefill; base addresses 16-byte aligned.
+ *   q_scale, k_scale, v_scale: per-tensor dequantisation scales (> 0,
+ *       finite): the query is q_scale * E4M3(q8), and likewise for k and v.
+ *   Other arguments as fa_prefill; head_dim must be 128 (else
+ *   FA_ERR_UNSUPPORTED).
+ * Q K^T multiplies the E4M3 codes exactly and accumulates in fp32; the
+ * probabilities are rounded to f16 (bf16 in fa_prefill) and V is widened to f16
+ * exactly, so P V also accumulates in fp32; out is bf16, lse fp32.  The NaN
+ * code S.1111.111 must not occur in the inputs (a saturating quantiser never
+ * writes it); it propagates as NaN into the rows that read it.
+ */
+int fa_prefill_fp8(const void* q, const void* k, const void* v,
+                   const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host, int batch,
+                   int num_q_heads, int num_kv_heads, int head_dim, int causal, float scale,
+                   float q_scale, float k_scale, float v_scale, void* out, float* lse,
+                   void* stream);
+
+/*
  * fa_append_kv — write new K/V rows into a paged KV cache (the cache that
  * prefill fills for later steps: niuteng5618.github.io "Flash Attention &
  * Paged Attention", section "FA对Prefill阶段的影响"; fixed-size pages behind a

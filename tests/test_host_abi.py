@@ -196,6 +196,24 @@ def _fake(addr):
     return ctypes.c_void_p(addr)
 
 
+def test_prefill_fp8_validation_before_any_cuda_call(lib):
+    cu = np.array([0, 128], dtype=np.int32)
+    cuh = cu.ctypes.data_as(ctypes.c_void_p)
+    A = 0x10000   # never dereferenced: validation fails first
+    call = lambda q=A, d=128, qs=1.0, ks=1.0, vs=1.0, cuh=cuh: lib.fa_prefill_fp8(
+        _fake(q), _fake(A), _fake(A), _fake(A), cuh, 1, 4, 2, d, 1, float("nan"), qs, ks, vs,
+        _fake(A), None, None)
+    assert call(q=0) == fa.FA_ERR_INVALID_ARG
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED                      # E4M3 inputs: d = 128 only
+    for bad_scale in (0.0, -1.0, float("nan"), float("inf")):
+        assert call(qs=bad_scale) == fa.FA_ERR_INVALID_ARG
+        assert call(ks=bad_scale) == fa.FA_ERR_INVALID_ARG
+        assert call(vs=bad_scale) == fa.FA_ERR_INVALID_ARG
+    assert call(q=A + 8) == fa.FA_ERR_INVALID_ARG                   # 16-byte alignment
+    bad = np.array([0, 0], dtype=np.int32)
+    assert call(cuh=bad.ctypes.data_as(ctypes.c_void_p)) == fa.FA_ERR_INVALID_ARG
+
+
 def test_prefill_validation_before_any_cuda_call(lib):
     cu = np.array([0, 128], dtype=np.int32)
     cuh = cu.ctypes.data_as(ctypes.c_void_p)

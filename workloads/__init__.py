@@ -349,6 +349,30 @@ def paged_decode_batch_fp8() -> DecodeInputs:
     return to_fp8_cache(paged_decode_batch())
 
 
+@dataclass
+class Fp8PrefillInputs(PrefillInputs):
+    """A prefill workload in FP8 E4M3: q_bits / k_bits / v_bits hold uint8
+    codes; the tensors are q_scale * E4M3(q8) and likewise for k and v."""
+    q_scale: float = 1.0
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+
+
+def to_fp8_prefill(inp: PrefillInputs, amax: float = 4.0) -> Fp8PrefillInputs:
+    """The same prefill inputs quantised to E4M3, one scale per tensor
+    (scale = amax / 448, as for the FP8 cache)."""
+    s = amax / E4M3_MAX
+    q8, k8, v8 = (quantize_e4m3(bf16_bits_to_f32(x), s) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    return Fp8PrefillInputs(inp.name + "_fp8", q8, k8, v8, inp.cu_seqlens, inp.causal, inp.scale,
+                            None, float(s), float(s), float(s))
+
+
+def varlen_causal_prefill_fp8() -> Fp8PrefillInputs:
+    """varlen_causal_prefill (8 sequences in [512, 4096], 32 heads, d=128,
+    causal) with Q, K and V in FP8 E4M3, per-tensor scales."""
+    return to_fp8_prefill(varlen_causal_prefill())
+
+
 def relayout(inp: DecodeInputs, layout: str) -> DecodeInputs:
     """Same cache contents in the other page layout (NHD <-> HND)."""
     if layout == inp.layout:
@@ -675,6 +699,7 @@ CONFIGS = {
     "long_split_decode": long_split_decode,
     "ragged_split_decode": ragged_split_decode,
     "paged_decode_batch_fp8": paged_decode_batch_fp8,
+    "varlen_causal_prefill_fp8": varlen_causal_prefill_fp8,
     "paged_decode_gqa8": paged_decode_gqa8,
     "paged_decode_gqa16": paged_decode_gqa16,
     "speculative_decode_batch": speculative_decode_batch,
