@@ -121,3 +121,36 @@ def test_append_chunked_prefill_and_cascade_in_graphs():
     torch.cuda.synchronize()
     assert torch.equal(co, want[0]) and torch.equal(cl, want[1])
     assert fa.device_status(clear=True) == 0
+
+
+def test_prefill_fp8_in_a_graph():
+    import torch
+    import exact_attention_148_b200 as fa
+    inp = W.to_fp8_prefill(W.make_prefill([129, 700], 4, 2, 128, causal=True, seed=2002))
+    q, k, v = (torch.from_numpy(x).cuda() for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    cu = to_dev_i32(inp.cu_seqlens)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    l = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+
+    def step():
+        fa.prefill_fp8(q, k, v, cu, q_scale=inp.q_scale, k_scale=inp.k_scale, v_scale=inp.v_scale,
+                       causal=True, scale=inp.scale, out=o, lse=l, cu_seqlens_host=inp.cu_seqlens,
+                       stream=torch.cuda.current_stream())
+
+    step()
+    torch.cuda.synchronize()
+    want = (o.clone(), l.clone())
+    g = _capture(step)
+    o.zero_()
+    l.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, want[0]) and torch.equal(l, want[1])
+    k.copy_(torch.flip(k, dims=[0]))        # new keys in place: the replay follows them
+    g.replay()
+    o2, l2 = fa.prefill_fp8(q, k, v, cu, q_scale=inp.q_scale, k_scale=inp.k_scale,
+                            v_scale=inp.v_scale, causal=True, scale=inp.scale,
+                            cu_seqlens_host=inp.cu_seqlens)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(l, l2)
+    assert fa.device_status(clear=True) == 0
