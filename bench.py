@@ -500,6 +500,18 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name and logical core count (/proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    return f"{ln.split(':', 1)[1].strip()}, {os.cpu_count()} logical cores"
+    except OSError:
+        pass
+    return f"unknown, {os.cpu_count()} logical cores"
+
+
 def oracle_prefill_sample(inp: W.PrefillInputs, budget_s: float):
     """Run the oracle on whole (sequence, head) blocks until about budget_s has
     passed; returns (flops done, seconds, description)."""
@@ -862,7 +874,7 @@ def cpu_baseline(case, budget):
         work, secs, desc = oracle_decode_sample(case.inp, budget)
         val, unit = work / secs / 1e9, "GB/s"
     return {"value": val, "unit": unit, "cores": threads, "kind": "oracle",
-            "sample": f"{desc}; {secs:.1f} s of CPU time"}
+            "sample": f"{desc}; {secs:.1f} s of CPU time", "cpu": cpu_model()}
 
 
 def run_reference(args):
@@ -906,7 +918,7 @@ def run_reference(args):
             "config": {"workload": inp.name if not (main == "default") else
                        "varlen_causal_prefill + paged_decode_batch (prefill half sampled)"},
             "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(), "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "cpu": cpu_model()},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
