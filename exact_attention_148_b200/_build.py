@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
 SOURCES = ["fa_api.cu", "planner.cpp"]
 HEADERS = ["ptx_sm100.cuh", "prefill_pp_sm100.cuh", "decode_sm100.cuh", "decode_tc_sm100.cuh",
-           "append_sm100.cuh", "planner.h"]
+           "append_sm100.cuh", "prefill_persist_sm100.cuh", "planner.h"]
 
 
 def nvcc_path() -> str:

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -18,6 +19,7 @@
 #include "decode_sm100.cuh"
 #include "decode_tc_sm100.cuh"
 #include "planner.h"
+#include "prefill_persist_sm100.cuh"
 #include "prefill_pp_sm100.cuh"
 
 #define FA_API extern "C" __attribute__((visibility("default")))
@@ -25,6 +27,10 @@
 struct fa_plan {
   fa::DecodePlan p;
 };
+
+// Work counters of the persistent prefill, {next item, CTAs finished} per
+// slot; zero at load, and reset to zero by the last CTA of every launch.
+__device__ uint32_t g_prefill_sched[fa::kSchedSlots][2];
 
 namespace {
 
@@ -133,6 +139,85 @@ int launch_prefill(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t,
     FA_CUDA_CHECK(cudaGetLastError());
   }
   return FA_OK;
+}
+
+// Persistent prefill (packed Q/K/V): one CTA per SM, items from a counter.
+template <int D, bool F8>
+int launch_prefill_persistent(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t, int>>& groups,
+                              cudaStream_t stream, uint32_t* sched, int num_sms) {
+  constexpr int kSmem = fa::PrefillPersistCfg<D, F8>::SMEM_BYTES;
+  constexpr int kThreads = fa::PrefillPersistCfg<D, F8>::THREADS;
+  auto kernel = fa::fa_prefill_persist_kernel<D, F8>;
+  int st = ensure_smem(reinterpret_cast<const void*>(kernel), kSmem);
+  if (st != FA_OK) return st;
+  for (size_t off = 0; off < groups.size(); off += fa::kPrefillMaxGroups) {
+    const int n = static_cast<int>(std::min<size_t>(fa::kPrefillMaxGroups, groups.size() - off));
+    int64_t total = 0;
+    for (int i = 0; i < n; ++i) {
+      prm.group_start[i] = static_cast<int>(total);
+      prm.group_id[i] = groups[off + i].first;
+      total += groups[off + i].second;
+    }
+    if (total > INT32_MAX) return FA_ERR_UNSUPPORTED;
+    prm.group_start[n] = static_cast<int>(total);
+    prm.num_groups = n;
+    prm.total_items = static_cast<int>(total);
+    prm.sched = sched;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(total, num_sms));
+    kernel<<<grid, kThreads, kSmem, stream>>>(prm);
+    FA_CUDA_CHECK(cudaGetLastError());
+  }
+  return FA_OK;
+}
+
+// FA_PREFILL_SCHEDULE=persistent selects the persistent prefill; anything
+// else (or unset) the grid form.
+bool prefill_persistent_requested() {
+  const char* s = std::getenv("FA_PREFILL_SCHEDULE");
+  return s != nullptr && std::strcmp(s, "persistent") == 0;
+}
+
+// The persistent prefill's counter pair for a launch on `stream`: one pair per
+// (device, stream), so launches that can overlap (other streams) never share
+// one, and launches on one stream run one after the other.  Null, and the grid
+// form is used, while the stream is being captured (a graph keeps the pointer,
+// and its replays could overlap eager launches on the same pair), when the
+// stream's id cannot be read, or once every pair of the device is taken.
+uint32_t* prefill_sched_slot(cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return nullptr;
+  unsigned long long id = 0;
+  int dev = 0;
+  if (cudaStreamGetId(stream, &id) != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  static std::mutex mu;
+  static std::map<std::pair<int, unsigned long long>, int> slot_of;
+  static std::map<int, int> taken;
+  static std::map<int, uint32_t*> base_of;
+  std::lock_guard<std::mutex> lock(mu);
+  auto b = base_of.find(dev);
+  if (b == base_of.end()) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_prefill_sched) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    b = base_of.emplace(dev, static_cast<uint32_t*>(ptr)).first;
+  }
+  const auto key = std::make_pair(dev, id);
+  auto it = slot_of.find(key);
+  if (it == slot_of.end()) {
+    int& t = taken[dev];
+    if (t >= fa::kSchedSlots) return nullptr;
+    it = slot_of.emplace(key, t++).first;
+  }
+  return b->second + 2 * it->second;
 }
 
 // Launch order of the prefill CTAs: sequences heaviest first (most query-key
@@ -320,6 +405,15 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* cu_
   prm.scale_log2 = scale * kLog2e * q_scale * k_scale;
   prm.v_scale = v_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prefill_persistent_requested()) {
+    uint32_t* sched = prefill_sched_slot(s);
+    int sms = 0;
+    if (sched != nullptr && sm_count(&sms) == FA_OK) {
+      if (f8) return launch_prefill_persistent<128, true>(prm, groups, s, sched, sms);
+      return head_dim == 128 ? launch_prefill_persistent<128, false>(prm, groups, s, sched, sms)
+                             : launch_prefill_persistent<64, false>(prm, groups, s, sched, sms);
+    }
+  }
   if (f8) return launch_prefill<128, false, true>(prm, groups, s);
   return head_dim == 128 ? launch_prefill<128, false>(prm, groups, s)
                          : launch_prefill<64, false>(prm, groups, s);

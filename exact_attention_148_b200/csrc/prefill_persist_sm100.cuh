@@ -1,0 +1,559 @@
+// Persistent form of the ping-pong prefill (packed Q/K/V, bf16 or E4M3).
+//
+// Same roles, tiles, TMEM columns and per-tile math as fa_prefill_pp_kernel;
+// the difference is what happens between work items.  In the grid form every
+// (q tile pair, head pair) item is its own CTA, and each CTA pays for its
+// launch, barrier and TMEM set-up, the latency of its first Q and K tiles,
+// a first softmax with no second slot to overlap, and its last P V and
+// epilogue with the tensor core idle.  Here one CTA per SM takes items from a
+// global counter in launch order (heaviest first, so the greedy fill of the
+// grid form is kept) and every pipeline runs on across items:
+//
+//   * the K/V ring, its barrier phases and the MMA stream never drain: the
+//     producer loads K_0 of the next item as soon as a ring slot frees;
+//   * a slot's Q tile is reloaded once the last S MMA of its previous item
+//     has completed (q_empty, committed by the MMA warp after that MMA);
+//   * the MMA warp issues S(i+1, 0) of a slot right after PV(i, last) of that
+//     slot (the P columns it overwrites are consumed by then: the tcgen05
+//     MMAs of one thread run in order), so the tensor core computes the next
+//     item's first scores while the softmax warps write the current O;
+//   * the softmax warps write O(i) and only then read S(i+1, 0) and arrive for
+//     PV(i+1, 0), which overwrites O, so the O columns need no new barrier.
+//
+// Item ids pass from the producer warp (which takes them from the counter)
+// to the other roles through a small shared-memory queue guarded by
+// item_full / item_empty mbarriers.  Every role takes every item, so all
+// per-role counters (ring entries, Q loads, tiles per slot, f16 V tiles)
+// advance identically.  The counter pair {next item, CTAs finished} is reset
+// by the last CTA to finish, ready for the next launch on the same stream;
+// the host gives each stream its own pair.
+#pragma once
+
+#include "prefill_pp_sm100.cuh"
+
+namespace fa {
+
+constexpr int kPersistQueue = 4;     // item ids in flight between the producer and the others
+constexpr int kSchedSlots = 64;      // counter pairs: one per stream that launches this kernel
+
+template <int D, bool F8 = false>
+struct PrefillPersistCfg {
+  using B = PrefillPPCfg<D, F8>;
+  // B's barriers, then q_empty[2], item_full[kPersistQueue], item_empty[kPersistQueue]
+  static constexpr int NUM_BARS = B::NUM_BARS + 2 + 2 * kPersistQueue;
+  static constexpr int QUEUE_OFF = B::BAR_OFF + NUM_BARS * 8;
+  static constexpr int MISC_OFF = QUEUE_OFF + 4 * kPersistQueue;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr int THREADS = B::THREADS;
+  // roles that take each item from the queue: the MMA thread, 8 softmax warps,
+  // and with E4M3 inputs the 2 converter warps
+  static constexpr int CONSUMERS = 1 + 8 + (F8 ? 2 : 0);
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(!F8 || B::NS % 2 == 0, "E4M3: V tiles must stay on odd ring slots");
+};
+
+// One work item: two 128-row query slots of one sequence that read the same
+// K/V tiles (two heads of a kv head at one q tile when the GQA group is even,
+// else two consecutive q tiles of one head).  Same numbering as the grid
+// form's CTA index: groups in launch order, heaviest q tiles first in a group.
+struct PrefillItem {
+  int s0;          // first token of the sequence
+  int L;           // its length (queries = keys)
+  int kv_head;
+  int qtile[2];
+  int head[2];
+  int n_kv[2];     // key tiles of each slot (0: slot unused)
+};
+
+__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int idx, int BM, int BN) {
+  int lo = 0, hi = p.num_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.group_start[mid] <= idx) lo = mid; else hi = mid - 1;
+  }
+  PrefillItem w;
+  const int seq = static_cast<int>(p.group_id[lo] >> 16);
+  w.kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
+  const int rank = idx - p.group_start[lo];
+  w.s0 = p.cu_seqlens[seq];
+  w.L = p.cu_seqlens[seq + 1] - w.s0;
+  const int n_qtiles = (w.L + BM - 1) / BM;
+  const int n_ktiles = (w.L + BN - 1) / BN;
+  const int G = p.group;
+  if ((G & 1) == 0) {
+    const int half = G >> 1;
+    const int t = n_qtiles - 1 - rank / half;
+    w.qtile[0] = w.qtile[1] = t;
+    w.head[0] = w.kv_head * G + 2 * (rank % half);
+    w.head[1] = w.head[0] + 1;
+  } else {
+    const int npairs = (n_qtiles + 1) >> 1;
+    const int pr = npairs - 1 - rank / G;
+    w.qtile[0] = 2 * pr;
+    w.qtile[1] = 2 * pr + 1;
+    w.head[0] = w.head[1] = w.kv_head * G + rank % G;
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const bool active = w.qtile[k] >= 0 && w.qtile[k] < n_qtiles;
+    w.n_kv[k] = !active ? 0 : (p.causal ? min(n_ktiles, (w.qtile[k] * BM + BM - 1) / BN + 1) : n_ktiles);
+  }
+  return w;
+}
+
+template <int D, bool F8 = false>
+__global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
+    fa_prefill_persist_kernel(const __grid_constant__ PrefillParams p) {
+  using B = PrefillPPCfg<D, F8>;
+  using C = PrefillPersistCfg<D, F8>;
+  constexpr int NS = B::NS;
+  constexpr int QD = kPersistQueue;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t q_s = base + B::Q_OFF;
+  auto kv_s = [&](uint32_t e) { return base + B::KV_OFF + (e % NS) * B::TILE_BYTES; };
+  const uint32_t bars = base + B::BAR_OFF;
+  const uint32_t bar_q = bars;
+  auto bar_kv_full = [&](uint32_t e) { return bars + 8 * (1 + e % NS); };
+  auto bar_kv_empty = [&](uint32_t e) { return bars + 8 * (1 + NS + e % NS); };
+  auto bar_s_full = [&](int k) { return bars + 8 * (1 + 2 * NS + k); };
+  auto bar_p_full = [&](int k) { return bars + 8 * (3 + 2 * NS + k); };
+  auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * NS + k); };
+  const uint32_t bar_final = bars + 8 * (7 + 2 * NS);
+  const uint32_t bar_q1 = bars + 8 * (9 + 2 * NS);
+  auto bar_vh_full = [&](int sl) { return bars + 8 * (10 + 2 * NS + sl); };
+  auto bar_vh_empty = [&](int sl) { return bars + 8 * (12 + 2 * NS + sl); };
+  auto bar_q_empty = [&](int k) { return bars + 8 * (B::NUM_BARS + k); };
+  auto bar_item_full = [&](int i) { return bars + 8 * (B::NUM_BARS + 2 + i); };
+  auto bar_item_empty = [&](int i) { return bars + 8 * (B::NUM_BARS + 2 + QD + i); };
+  volatile int* queue = reinterpret_cast<volatile int*>(smem + C::QUEUE_OFF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    mbar_init(bar_q1, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bar_kv_full(i), 1);
+      // E4M3: the V tiles (odd ring entries, odd slots since NS is even and
+      // every item has an even number of entries) are released by the two
+      // converter warps, the K tiles by the MMA thread
+      mbar_init(bar_kv_empty(i), (F8 && (i & 1)) ? 2 : 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar_s_full(k), 1);
+      mbar_init(bar_p_full(k), 4);
+      mbar_init(bar_o_done(k), 1);
+      mbar_init(bar_q_empty(k), 1);
+      if constexpr (F8) {
+        mbar_init(bar_vh_full(k), 2);
+        mbar_init(bar_vh_empty(k), 1);
+      }
+    }
+    for (int i = 0; i < QD; ++i) {
+      mbar_init(bar_item_full(i), 1);
+      mbar_init(bar_item_empty(i), C::CONSUMERS);
+    }
+    mbar_init(bar_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_addr(tmem_slot), B::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  // A consumer warp's next item id (-1: no more work; -2: aborted).  All
+  // lanes wait; lane 0 releases the queue entry once the id is in registers.
+  auto take_item_warp = [&](int n) -> int {
+    const int qi = n % QD;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_item_full(qi), (n / QD) & 1, abort_flag))) return -2;
+    const int it = queue[qi];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_item_empty(qi));
+    return it;
+  };
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- TMA producer + scheduler
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      auto load_q = [&](int k, int h, int row0, uint32_t bar) {
+        mbar_arrive_expect_tx(bar, B::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < B::CHUNKS; ++c)
+          tma_load_3d(q_s + k * B::TILE_BYTES + c * B::CHUNK_BYTES, &p.tm_q, bar, c * 64, h, row0);
+      };
+      uint32_t issued = 0;          // ring entries issued
+      int qc0 = 0, qc1 = 0;         // Q loads of each slot
+      int next = static_cast<int>(atomicAdd(p.sched, 1u));
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        const int it = next < p.total_items ? next : -1;
+        const int qi = n % QD;
+        if (!mbar_wait(bar_item_empty(qi), ((n / QD) & 1) ^ 1, abort_flag)) break;
+        queue[qi] = it;
+        mbar_arrive(bar_item_full(qi));
+        if (it < 0) break;
+        next = static_cast<int>(atomicAdd(p.sched, 1u));   // claimed now, started after this item
+        const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+        const int n_max = max(w.n_kv[0], w.n_kv[1]);
+        // ring entries K_0, V_0, K_1, V_1, ...; both Q tiles right after K_0
+        for (int e = 0; e < 2 * n_max; ++e) {
+          const uint32_t R = issued;
+          if (!mbar_wait(bar_kv_empty(R), ((R / NS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar_kv_full(R), B::TILE_BYTES);
+          const CUtensorMap* map = (e & 1) ? &p.tm_v : &p.tm_k;
+          const int row = w.s0 + (e >> 1) * B::BN;
+#pragma unroll
+          for (int c = 0; c < B::CHUNKS; ++c)
+            tma_load_3d(kv_s(R) + c * B::CHUNK_BYTES, map, bar_kv_full(R), c * 64, w.kv_head, row);
+          ++issued;
+          if (e == 0) {
+            // a slot's Q tile is free once the last S MMA of its previous item completed
+            if (w.n_kv[0] > 0) {
+              if (!mbar_wait(bar_q_empty(0), (qc0 & 1) ^ 1, abort_flag)) { ok = false; break; }
+              load_q(0, w.head[0], w.s0 + w.qtile[0] * B::BM, bar_q);
+              ++qc0;
+            }
+            if (w.n_kv[1] > 0) {
+              if (!mbar_wait(bar_q_empty(1), (qc1 & 1) ^ 1, abort_flag)) { ok = false; break; }
+              load_q(1, w.head[1], w.s0 + w.qtile[1] * B::BM, bar_q1);
+              ++qc1;
+            }
+          }
+        }
+      }
+      if (*abort_flag) {
+        // let the copies in flight land before the CTA's shared memory goes away
+        volatile int never = 0;
+        for (uint32_t i = (issued > static_cast<uint32_t>(NS) ? issued - NS : 0u); i < issued; ++i)
+          mbar_wait(bar_kv_full(i), (i / NS) & 1, &never);
+        if (qc0 > 0) mbar_wait(bar_q, (qc0 - 1) & 1, &never);
+        if (qc1 > 0) mbar_wait(bar_q1, (qc1 - 1) & 1, &never);
+      }
+      __threadfence();   // this thread's counter updates precede the CTA's finish count
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_k(B::BM, B::BN) : idesc_bf16_f32(B::BM, B::BN, false);
+      constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(B::BM, D, true) : idesc_bf16_f32(B::BM, D, true);
+      const uint64_t q_desc = sdesc_sw128(q_s, 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(base + B::KV_OFF, 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(base + (F8 ? B::VH_OFF : B::KV_OFF), B::CHUNK_BYTES, 1024);
+      auto ring_off = [&](uint32_t e) { return static_cast<uint64_t>((e % NS) * (B::TILE_BYTES >> 4)); };
+      auto issue_qk = [&](int k, uint32_t R) {
+        const uint64_t qd = q_desc + (k ? (B::TILE_BYTES >> 4) : 0);
+        const uint64_t kd = k_desc0 + ring_off(R);
+        const uint32_t d_tmem = tmem + (k ? 128u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D * B::ELEM / 32; ++kk) {   // 32-byte K steps
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * B::CHUNK_BYTES + (kk & 3) * 32) >> 4);
+          if constexpr (F8) mma_f8_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+          else mma_bf16_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      // V operand: ring entry R (bf16) or f16 tile vslot (E4M3)
+      auto issue_pv = [&](int k, uint32_t R, int vslot, bool accumulate) {
+        const uint32_t o_tmem = tmem + 256u + (k ? D : 0);
+        const uint32_t p_tmem = tmem + (k ? 128u : 0u);
+        const uint64_t vd = F8 ? v_desc0 + static_cast<uint64_t>((vslot * B::VH_TILE) >> 4)
+                               : v_desc0 + ring_off(R);
+#pragma unroll
+        for (int kk = 0; kk < B::BN / 16; ++kk)
+          mma_bf16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
+                      (accumulate || kk > 0) ? 1u : 0u);
+      };
+      uint32_t ring = 0;      // first ring entry of the current item
+      int qc0 = 0, qc1 = 0;   // Q tiles consumed per slot
+      int t0 = 0, t1 = 0;     // key tiles done per slot before the current item
+      int vcount = 0;         // f16 V tiles consumed (E4M3)
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        const int qi = n % QD;
+        if (!mbar_wait(bar_item_full(qi), (n / QD) & 1, abort_flag)) break;
+        const int it = queue[qi];
+        mbar_arrive(bar_item_empty(qi));
+        if (it < 0) break;
+        const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+        const int nk0 = w.n_kv[0], nk1 = w.n_kv[1];
+        const int n_max = max(nk0, nk1);
+        // first scores of both slots (K_0 is entry `ring`)
+        if (!mbar_wait(bar_kv_full(ring), (ring / NS) & 1, abort_flag)) break;
+        if (nk0 > 0) {
+          if (!mbar_wait(bar_q, qc0 & 1, abort_flag)) break;
+          tc_fence_after_sync();
+          issue_qk(0, ring);
+          tc_commit(bar_s_full(0));
+          if (nk0 == 1) tc_commit(bar_q_empty(0));
+          ++qc0;
+        }
+        if (nk1 > 0) {
+          if (!mbar_wait(bar_q1, qc1 & 1, abort_flag)) break;
+          tc_fence_after_sync();
+          issue_qk(1, ring);
+          tc_commit(bar_s_full(1));
+          if (nk1 == 1) tc_commit(bar_q_empty(1));
+          ++qc1;
+        }
+        tc_commit(bar_kv_empty(ring));
+        // One slot's step at key tile j: O_k += P_k V_j, then S_k(j+1).
+        auto slot_step = [&](int k, int nk, int tb, int j, uint32_t v_R, int vslot, uint32_t k_R) -> bool {
+          if (j >= nk) return true;
+          if (!mbar_wait(bar_p_full(k), (tb + j) & 1, abort_flag)) return false;
+          tc_fence_after_sync();
+          issue_pv(k, v_R, vslot, j > 0);
+          tc_commit(bar_o_done(k));
+          if (j + 1 < nk) {
+            issue_qk(k, k_R);
+            tc_commit(bar_s_full(k));
+            if (j + 2 == nk) tc_commit(bar_q_empty(k));   // that was the slot's last S of this item
+          }
+          return true;
+        };
+        for (int j = 0; j < n_max; ++j) {
+          const uint32_t v_R = ring + 2 * j + 1, k_R = ring + 2 * j + 2;
+          const int vslot = vcount & 1;
+          const bool need_k = (j + 1 < nk0) || (j + 1 < nk1);
+          if (F8 ? !mbar_wait(bar_vh_full(vslot), (vcount >> 1) & 1, abort_flag)
+                 : !mbar_wait(bar_kv_full(v_R), (v_R / NS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (need_k && !mbar_wait(bar_kv_full(k_R), (k_R / NS) & 1, abort_flag)) { ok = false; break; }
+          if (!slot_step(0, nk0, t0, j, v_R, vslot, k_R) || !slot_step(1, nk1, t1, j, v_R, vslot, k_R)) {
+            ok = false;
+            break;
+          }
+          if constexpr (F8) tc_commit(bar_vh_empty(vslot));
+          else tc_commit(bar_kv_empty(v_R));
+          if (need_k) tc_commit(bar_kv_empty(k_R));
+          ++vcount;
+        }
+        ring += 2 * n_max;
+        t0 += nk0;
+        t1 += nk1;
+      }
+      tc_commit(bar_final);
+      volatile int never = 0;
+      mbar_wait(bar_final, 0, &never);
+    }
+  } else if (F8 && warp >= 10) {
+    // ---------------------------------------------------------------- V converters (E4M3 -> f16)
+    // Warp 10 widens keys 0-63 of V_j, warp 11 keys 64-127 (layouts as in
+    // fa_prefill_pp_kernel's converter warps).
+    const int half = warp - 10;
+    uint32_t ring = 0;
+    int vcount = 0;
+    for (int n = 0;; ++n) {
+      const int it = take_item_warp(n);
+      if (it < 0) break;
+      const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+      const int n_max = max(w.n_kv[0], w.n_kv[1]);
+      bool ok = true;
+      for (int j = 0; j < n_max; ++j, ++vcount) {
+        const uint32_t v_R = ring + 2 * j + 1;
+        const int vslot = vcount & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_kv_full(v_R), (v_R / NS) & 1, abort_flag)) ||
+            !__all_sync(0xffffffffu, mbar_wait(bar_vh_empty(vslot), ((vcount >> 1) & 1) ^ 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = smem + B::KV_OFF + (v_R % NS) * B::TILE_BYTES;
+        uint8_t* dst = smem + B::VH_OFF + vslot * B::VH_TILE;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int e = lane + 32 * i;             // 0..511
+          const int key = half * 64 + (e >> 3), u = e & 7, sw = key & 7;
+          const uint4 b = *reinterpret_cast<const uint4*>(src + key * 128 + ((u ^ sw) << 4));
+          uint4 lo4, hi4;
+          e4m3x4_to_f16x4(b.x, lo4.x, lo4.y);
+          e4m3x4_to_f16x4(b.y, lo4.z, lo4.w);
+          e4m3x4_to_f16x4(b.z, hi4.x, hi4.y);
+          e4m3x4_to_f16x4(b.w, hi4.z, hi4.w);
+          const int c = u >> 2, w0 = 2 * (u & 3);
+          uint8_t* row = dst + c * B::CHUNK_BYTES + key * 128;
+          *reinterpret_cast<uint4*>(row + ((w0 ^ sw) << 4)) = lo4;
+          *reinterpret_cast<uint4*>(row + (((w0 + 1) ^ sw) << 4)) = hi4;
+        }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar_vh_full(vslot));
+          mbar_arrive(bar_kv_empty(v_R));
+        }
+      }
+      if (!ok) break;
+      ring += 2 * n_max;
+    }
+  } else if (warp < 8) {
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int k = warp >> 2;                       // slot
+    const int r = threadIdx.x & 127;               // row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sc = tmem + lane_base + (k ? 128u : 0u);
+    const uint32_t oc = tmem + lane_base + 256u + (k ? D : 0);
+    int tiles = 0;                                 // key tiles of this slot before the item
+    for (int n = 0;; ++n) {
+      const int it = take_item_warp(n);
+      if (it < 0) break;
+      const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+      const int nk = k ? w.n_kv[1] : w.n_kv[0];   // (k is not a compile-time index)
+      if (nk == 0) continue;
+      const int my_qtile = k ? w.qtile[1] : w.qtile[0];
+      const int my_head = k ? w.head[1] : w.head[0];
+      const int q_row = my_qtile * B::BM + r;
+      const int row_last = p.causal ? min(q_row, w.L - 1) : w.L - 1;
+      const int tile_last = p.causal ? min(my_qtile * B::BM, w.L - 1) : w.L - 1;
+      float m_ref = 0.0f, l_sum = 0.0f;
+      bool ok = true;
+      for (int j = 0; j < nk; ++j) {
+        const int g = tiles + j;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(k), g & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after_sync();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_x32(sc + c * 32, s[c]);
+        tmem_ld_wait(s[0]);
+        reg_dep(s[1]);
+        reg_dep(s[2]);
+        reg_dep(s[3]);
+
+        const bool masked = j * B::BN + B::BN - 1 > tile_last;
+        if (masked) {
+          const int lim = row_last - j * B::BN;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i > lim) s[c][i] = __float_as_uint(-INFINITY);
+        }
+        float mx[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          mx[c] = fmax3(__uint_as_float(s[c][0]), __uint_as_float(s[c][1]), __uint_as_float(s[c][2]));
+#pragma unroll
+          for (int i = 3; i < 31; i += 2)
+            mx[c] = fmax3(mx[c], __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
+          mx[c] = fmaxf(mx[c], __uint_as_float(s[c][31]));
+        }
+        const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float m_tile = rmax * p.scale_log2;
+        float alpha = 1.0f;
+        bool rescale = false;
+        if (j == 0) {
+          m_ref = (m_tile == -INFINITY) ? 0.0f : m_tile;
+        } else {
+          const bool need = m_tile > m_ref + kRescaleThreshold;
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2_approx(m_ref - m_tile);
+            m_ref = m_tile;
+          }
+        }
+        const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 neg_m2 = make_float2(-m_ref, -m_ref);
+        float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), scale2, neg_m2);
+            const float p0 = ex2_approx(x.x);
+            const float p1 = ex2_approx(x.y);
+            ps[i & 3].x += p0;
+            ps[i & 3].y += p1;
+            pk[i] = F8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+          }
+          tmem_st_x16(sc + c * 16, pk);
+        }
+        l_sum = l_sum * alpha + (((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
+                                 ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y)));
+        if (rescale) {
+          // O holds P V of tiles < j against the old reference maximum: once
+          // PV(j - 1) has landed, scale it by alpha
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (g - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_x32(oc + c * 32, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_x32(oc + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p_full(k));
+      }
+      if (!ok) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (tiles + nk - 1) & 1, abort_flag))) break;
+      tc_fence_after_sync();
+      const float inv_l = F8 ? p.v_scale / l_sum : 1.0f / l_sum;
+      const bool valid = q_row < w.L;
+      __nv_bfloat16* orow = p.out + (static_cast<size_t>(w.s0 + q_row) * p.num_q_heads + my_head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_x32(oc + c * 32, o);
+        tmem_ld_wait(o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[static_cast<size_t>(w.s0 + q_row) * p.num_q_heads + my_head] =
+            (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
+      // O is read out: the next item's first P V may overwrite it (the
+      // p_full arrival of its first tile follows this in program order)
+      tc_fence_before_sync();
+      tiles += nk;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, B::TMEM_COLS);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA to finish resets the counters for the next launch
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
+  }
+}
+
+}  // namespace fa
