@@ -143,7 +143,8 @@ class PrefillCase:
         self.out = torch.empty(self.q.shape, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=device)
         self.flops = inp.causal_flops()
-        self.launches = -(-sum(-(-int(L) // 128) for L in inp.seqlens) // 2048)
+        # one launch per 2048 (sequence, kv head) groups
+        self.launches = -(-len(inp.seqlens) * inp.num_kv_heads // 2048)
         self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
         self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
 
@@ -181,6 +182,7 @@ class PrefillCase:
                 "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads,
                 "head_dim": i.head_dim, "causal": bool(i.causal),
                 "inputs": "e4m3 q/k/v, per-tensor scales" if self.fp8 else "bf16",
+                "schedule": os.environ.get("FA_PREFILL_SCHEDULE") == "persistent" and "persistent" or "grid",
                 "algorithmic_tflop": round(self.flops / 1e12, 4)}
 
 
@@ -662,6 +664,7 @@ def build_cases(workload, device, num_splits, kernel="auto", heads=None):
 def kernel_source_hash(kind):
     import hashlib
     files = {"prefill": ["ptx_sm100.cuh", "prefill_pp_sm100.cuh"],
+             "prefill_persist": ["ptx_sm100.cuh", "prefill_pp_sm100.cuh", "prefill_persist_sm100.cuh"],
              "decode": ["ptx_sm100.cuh", "decode_sm100.cuh"],
              "decode_tc": ["ptx_sm100.cuh", "decode_sm100.cuh", "decode_tc_sm100.cuh"],
              "append": ["ptx_sm100.cuh", "append_sm100.cuh"]}[kind]
@@ -685,7 +688,8 @@ def measured_traffic(kind, workload, case=None):
     rows = {}
     for ln in lines:
         parts = [x.strip() for x in ln.strip().strip("|").split("|")]
-        if len(parts) >= 5 and parts[0] in ("prefill", "decode", "decode_tc", "append") and parts[3].isdigit():
+        if len(parts) >= 5 and parts[0] in ("prefill", "prefill_persist", "decode", "decode_tc", "append") \
+                and parts[3].isdigit():
             rows[(parts[0], parts[1])] = (parts[2], int(parts[3]) + int(parts[4]))
     sha = kernel_source_hash(kind)
     if (kind, workload) in rows and rows[(kind, workload)][0] == sha:
@@ -759,9 +763,12 @@ def run_ours(args):
     rooflines = []
     for c, ms in zip(cases, ms_case):
         if isinstance(c, PrefillCase):
+            pers = os.environ.get("FA_PREFILL_SCHEDULE") == "persistent"
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
-                               measured_traffic("prefill", c.inp.name), fp8_qk=c.fp8)
-            e["kernel"] = "fa_prefill_pp_kernel<%d%s>" % (c.inp.head_dim, ", e4m3" if c.fp8 else "")
+                               measured_traffic("prefill_persist" if pers else "prefill", c.inp.name),
+                               fp8_qk=c.fp8)
+            e["kernel"] = "%s<%d%s>" % ("fa_prefill_persist_kernel" if pers else "fa_prefill_pp_kernel",
+                                        c.inp.head_dim, ", e4m3" if c.fp8 else "")
         elif isinstance(c, ChunkedAttnCase):
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
                                measured_traffic("prefill", c.inp.name))
@@ -938,7 +945,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--prefill-schedule", default=None, choices=["grid", "persistent"],
+                    help="packed prefill: one CTA per work item (grid) or one per SM (persistent); "
+                         "default: the library's (FA_PREFILL_SCHEDULE, else grid)")
     args = ap.parse_args()
+    if args.prefill_schedule is not None:
+        os.environ["FA_PREFILL_SCHEDULE"] = args.prefill_schedule
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
