@@ -161,10 +161,12 @@ int launch_prefill_persistent(fa::PrefillParams& prm, const std::vector<std::pai
     if (total > INT32_MAX) return FA_ERR_UNSUPPORTED;
     prm.group_start[n] = static_cast<int>(total);
     prm.num_groups = n;
-    prm.total_items = static_cast<int>(total);
-    prm.sched = sched;
+    static thread_local fa::PrefillPersistParams pp;   // ~17 KB; kept off the stack
+    pp.p = prm;
+    pp.sched = sched;
+    pp.total_items = static_cast<int>(total);
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(total, num_sms));
-    kernel<<<grid, kThreads, kSmem, stream>>>(prm);
+    kernel<<<grid, kThreads, kSmem, stream>>>(pp);
     FA_CUDA_CHECK(cudaGetLastError());
   }
   return FA_OK;

@@ -52,6 +52,13 @@ struct PrefillPersistCfg {
   static_assert(!F8 || B::NS % 2 == 0, "E4M3: V tiles must stay on odd ring slots");
 };
 
+// Launch arguments: the grid form's, plus the work counter.
+struct PrefillPersistParams {
+  PrefillParams p;
+  uint32_t* sched;     // {next item, CTAs finished}; zero at launch, zero again at exit
+  int total_items;     // work items of this launch
+};
+
 // One work item: two 128-row query slots of one sequence that read the same
 // K/V tiles (two heads of a kv head at one q tile when the GQA group is even,
 // else two consecutive q tiles of one head).  Same numbering as the grid
@@ -103,7 +110,8 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
 
 template <int D, bool F8 = false>
 __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
-    fa_prefill_persist_kernel(const __grid_constant__ PrefillParams p) {
+    fa_prefill_persist_kernel(const __grid_constant__ PrefillPersistParams pp) {
+  const PrefillParams& p = pp.p;
   using B = PrefillPPCfg<D, F8>;
   using C = PrefillPersistCfg<D, F8>;
   constexpr int NS = B::NS;
@@ -198,16 +206,16 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
       };
       uint32_t issued = 0;          // ring entries issued
       int qc0 = 0, qc1 = 0;         // Q loads of each slot
-      int next = static_cast<int>(atomicAdd(p.sched, 1u));
+      int next = static_cast<int>(atomicAdd(pp.sched, 1u));
       bool ok = true;
       for (int n = 0; ok; ++n) {
-        const int it = next < p.total_items ? next : -1;
+        const int it = next < pp.total_items ? next : -1;
         const int qi = n % QD;
         if (!mbar_wait(bar_item_empty(qi), ((n / QD) & 1) ^ 1, abort_flag)) break;
         queue[qi] = it;
         mbar_arrive(bar_item_full(qi));
         if (it < 0) break;
-        next = static_cast<int>(atomicAdd(p.sched, 1u));   // claimed now, started after this item
+        next = static_cast<int>(atomicAdd(pp.sched, 1u));   // claimed now, started after this item
         const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
         const int n_max = max(w.n_kv[0], w.n_kv[1]);
         // ring entries K_0, V_0, K_1, V_1, ...; both Q tiles right after K_0
@@ -549,9 +557,9 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
   if (threadIdx.x == 0) {
     // the last CTA to finish resets the counters for the next launch
     __threadfence();
-    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-      atomicExch(p.sched, 0u);
-      atomicExch(p.sched + 1, 0u);
+    if (atomicAdd(pp.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(pp.sched, 0u);
+      atomicExch(pp.sched + 1, 0u);
     }
   }
 }

@@ -75,8 +75,6 @@ struct PrefillParams {
   float* part_o;
   float* part_lse;
   float v_scale;             // E4M3 inputs: V dequantisation scale
-  uint32_t* sched;           // persistent form: {next item, CTAs finished}, zero at launch
-  int total_items;           // persistent form: work items of this launch
   int max_pages;
   int num_pages;
   int head_coord;            // paged: tensor-map dimension (1..3) of the kv head
