@@ -21,6 +21,7 @@ __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
     "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
     "append_kv", "prefill_paged", "prefill_fp8", "decode_paged_fp8", "cascade_decode", "cascade_workspace_bytes",
+    "prefill_last_schedule",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -40,11 +41,12 @@ EXPORTED_SYMBOLS = [
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
     "fa_decode_paged_fp8", "fa_decode_plan_kv", "fa_decode_plan_ex", "fa_cascade_workspace_bytes",
-    "fa_cascade_decode", "fa_prefill_fp8",
+    "fa_cascade_decode", "fa_prefill_fp8", "fa_prefill_last_schedule",
 ]
 
 FA_KV_BF16, FA_KV_E4M3 = 0, 1
 FA_DECODE_AUTO, FA_DECODE_CUDA_CORES, FA_DECODE_TENSOR_CORES = 0, 1, 2
+FA_SCHEDULE_GRID, FA_SCHEDULE_PERSISTENT = 0, 1
 _KV_DTYPES = {"bf16": FA_KV_BF16, "e4m3": FA_KV_E4M3}
 _KERNELS = {"auto": FA_DECODE_AUTO, "cuda_cores": FA_DECODE_CUDA_CORES,
             "tensor_cores": FA_DECODE_TENSOR_CORES}
@@ -140,6 +142,8 @@ def library() -> ctypes.CDLL:
     L.fa_decode_paged_fp8.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, f32, f32, f32, vp,
                                       vp, vp, ctypes.c_size_t, vp]
     L.fa_decode_paged_fp8.restype = i32
+    L.fa_prefill_last_schedule.argtypes = []
+    L.fa_prefill_last_schedule.restype = i32
     _lib = L
     return L
 
@@ -213,6 +217,13 @@ def prefill(q, k, v, cu_seqlens, *, causal: bool = True, scale: float | None = N
                               _stream_ptr(stream))
     _check(st, "fa_prefill")
     return out, lse
+
+
+def prefill_last_schedule() -> str | None:
+    """"persistent" or "grid": the schedule the calling thread's last prefill /
+    prefill_fp8 launched (None if that call failed or there was none)."""
+    return {FA_SCHEDULE_GRID: "grid", FA_SCHEDULE_PERSISTENT: "persistent"}.get(
+        library().fa_prefill_last_schedule())
 
 
 def prefill_fp8(q, k, v, cu_seqlens, *, q_scale: float, k_scale: float, v_scale: float,
@@ -581,7 +592,3 @@ def selftest_wait_timeout(limit_us: int = 20000, stream=None) -> int:
 
 def version() -> int:
     return library().fa_version()
-
-
-def default_scale(head_dim: int) -> float:
-    return 1.0 / math.sqrt(head_dim)

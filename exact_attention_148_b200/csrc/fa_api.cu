@@ -172,12 +172,14 @@ int launch_prefill_persistent(fa::PrefillParams& prm, const std::vector<std::pai
   return FA_OK;
 }
 
-// FA_PREFILL_SCHEDULE=persistent selects the persistent prefill; anything
-// else (or unset) the grid form.
+// The packed prefill runs the persistent form unless FA_PREFILL_SCHEDULE=grid.
 bool prefill_persistent_requested() {
   const char* s = std::getenv("FA_PREFILL_SCHEDULE");
-  return s != nullptr && std::strcmp(s, "persistent") == 0;
+  return s == nullptr || std::strcmp(s, "grid") != 0;
 }
+
+// Schedule of the calling thread's last fa_prefill / fa_prefill_fp8 launch.
+thread_local int t_last_prefill_schedule = -1;
 
 // The persistent prefill's counter pair for a launch on `stream`: one pair per
 // (device, stream), so launches that can overlap (other streams) never share
@@ -407,18 +409,24 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* cu_
   prm.scale_log2 = scale * kLog2e * q_scale * k_scale;
   prm.v_scale = v_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  t_last_prefill_schedule = -1;
+  int st = FA_OK;
   if (prefill_persistent_requested()) {
     uint32_t* sched = prefill_sched_slot(s);
     int sms = 0;
     if (sched != nullptr && sm_count(&sms) == FA_OK) {
-      if (f8) return launch_prefill_persistent<128, true>(prm, groups, s, sched, sms);
-      return head_dim == 128 ? launch_prefill_persistent<128, false>(prm, groups, s, sched, sms)
-                             : launch_prefill_persistent<64, false>(prm, groups, s, sched, sms);
+      if (f8) st = launch_prefill_persistent<128, true>(prm, groups, s, sched, sms);
+      else if (head_dim == 128) st = launch_prefill_persistent<128, false>(prm, groups, s, sched, sms);
+      else st = launch_prefill_persistent<64, false>(prm, groups, s, sched, sms);
+      if (st == FA_OK) t_last_prefill_schedule = FA_SCHEDULE_PERSISTENT;
+      return st;
     }
   }
-  if (f8) return launch_prefill<128, false, true>(prm, groups, s);
-  return head_dim == 128 ? launch_prefill<128, false>(prm, groups, s)
-                         : launch_prefill<64, false>(prm, groups, s);
+  if (f8) st = launch_prefill<128, false, true>(prm, groups, s);
+  else if (head_dim == 128) st = launch_prefill<128, false>(prm, groups, s);
+  else st = launch_prefill<64, false>(prm, groups, s);
+  if (st == FA_OK) t_last_prefill_schedule = FA_SCHEDULE_GRID;
+  return st;
 }
 
 }  // namespace
@@ -429,6 +437,8 @@ FA_API int fa_prefill(const void* q, const void* k, const void* v, const int32_t
   return prefill_impl(q, k, v, cu_seqlens_dev, cu_seqlens_host, batch, num_q_heads, num_kv_heads,
                       head_dim, causal, scale, false, 1.0f, 1.0f, 1.0f, out, lse, stream);
 }
+
+FA_API int fa_prefill_last_schedule(void) { return t_last_prefill_schedule; }
 
 FA_API int fa_prefill_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
                           const int32_t* cu_seqlens_host, int batch, int num_q_heads,

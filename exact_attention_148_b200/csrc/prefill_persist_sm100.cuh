@@ -34,7 +34,7 @@
 namespace fa {
 
 constexpr int kPersistQueue = 4;     // item ids in flight between the producer and the others
-constexpr int kSchedSlots = 64;      // counter pairs: one per stream that launches this kernel
+constexpr int kSchedSlots = 256;     // counter pairs: one per stream that launches this kernel
 
 template <int D, bool F8 = false>
 struct PrefillPersistCfg {

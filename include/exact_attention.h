@@ -107,11 +107,36 @@ typedef struct {
  *   out  [T, Hq, d] bf16 (written); lse [T, Hq] fp32 natural-log LSE, or NULL.
  * Supported: d in {64, 128}; Hq % Hkv == 0; each sequence length >= 1;
  * T < 2^31 / (Hq*d).  Output rows of different sequences never mix.
+ *
+ * Schedule (plan-stage load balancing: wsisp.com "FIA / FlashAttention",
+ * section 二).  The work is cut into items of two 128-row query tiles that read
+ * the same K/V tiles, ordered heaviest first.  By default one CTA per SM takes
+ * items from a device counter and keeps its pipelines running from one item to
+ * the next (the persistent form).  The counter is one of 256 pairs in the
+ * library's device memory, one per (device, stream) that launches the kernel,
+ * reset to zero by the last CTA of each launch.  The grid form (one CTA per
+ * item) runs instead when the environment variable FA_PREFILL_SCHEDULE is
+ * "grid", while `stream` is being captured into a graph (a graph's replays
+ * could overlap other launches on the same counter), and once 256 streams of a
+ * device have taken a counter (a stream keeps its counter for the life of the
+ * process).  Both forms compute bit-identical results;
+ * fa_prefill_last_schedule() tells which one the calling thread's last call
+ * launched.
  */
 int fa_prefill(const void* q, const void* k, const void* v,
                const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host, int batch,
                int num_q_heads, int num_kv_heads, int head_dim, int causal, float scale,
                void* out, float* lse, void* stream);
+
+/* Schedule of a prefill launch (see fa_prefill). */
+typedef enum { FA_SCHEDULE_GRID = 0, FA_SCHEDULE_PERSISTENT = 1 } fa_prefill_schedule;
+
+/*
+ * fa_prefill_last_schedule — the fa_prefill_schedule that the calling thread's
+ * last fa_prefill or fa_prefill_fp8 call launched, or -1 if that call failed or
+ * there was none.  Host only; never fails.
+ */
+int fa_prefill_last_schedule(void);
 
 /*
  * fa_prefill_fp8 — fa_prefill over E4M3 inputs (FP8 inference kernels:
@@ -326,7 +351,9 @@ int fa_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages,
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     stream capture.  The cached address is not looked up again, so after a
+ *     cudaDeviceReset on that device this entry point must not be used again
+ *     in the same process.
  *   - All calls on a device share the one array, which keeps whatever the last
  *     call left in it.  Nothing in it needs to start at zero: every partial the
  *     merge reads is written earlier in the same call.  Calls that overlap on
