@@ -2,7 +2,6 @@
 
 #include <algorithm>
 #include <functional>
-#include <queue>
 #include <vector>
 
 #include "../../include/exact_attention.h"
@@ -53,44 +52,104 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
   const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
   const double cta_bytes_per_us = cm.bytes_per_us;
   const double overhead_bytes = cm.overhead_us * cta_bytes_per_us;
-  std::priority_queue<double, std::vector<double>, std::greater<double>> running;
-  double v = 0.0, t = 0.0;
+  const double full = static_cast<double>(chunk) * bytes_per_token + overhead_bytes;
+  // Running CTAs' finish points (bytes done by every running CTA).  Full-chunk
+  // CTAs start in non-decreasing order and all have the same size, so their
+  // finish points come in order: a FIFO ring holds them.  The other CTAs
+  // (each request's last split) go to a min-heap.  The next event is the
+  // smaller of the two fronts, so events come in the same order as from one
+  // heap of all running CTAs.
+  std::vector<double> ring(static_cast<size_t>(std::max(slots, 1)));
+  size_t head = 0, count = 0;
+  std::vector<double> heap;
+  heap.reserve(static_cast<size_t>(slots));
+  const auto later = std::greater<double>();
+  auto start_cta = [&](double finish, bool full_chunk) {
+    if (full_chunk) {
+      size_t at = head + count;
+      if (at >= ring.size()) at -= ring.size();
+      ring[at] = finish;
+      ++count;
+    } else {
+      heap.push_back(finish);
+      std::push_heap(heap.begin(), heap.end(), later);
+    }
+  };
+  // CTAs in grid order: request b's n splits (every one a full chunk but the
+  // last), repeated for each of the units, then request b + 1.
   size_t b = 0;
-  int64_t u = 0, sidx = 0;
-  int max_splits = 1;
-  // next CTA in grid order, or a negative value when none is left
-  auto next_cta = [&]() -> double {
-    while (b < lens.size()) {
-      const int64_t L = lens[b];
-      const int64_t n = std::max<int64_t>(1, ceil_div(L, chunk));
-      max_splits = std::max<int>(max_splits, static_cast<int>(n));
-      if (sidx < n) {
-        const int64_t tok = std::max<int64_t>(0, std::min<int64_t>(chunk, L - sidx * chunk));
-        ++sidx;
-        return tok * bytes_per_token + overhead_bytes;
-      }
+  int64_t u = 0, sidx = 0, n = 1;
+  double last = 0.0;
+  int64_t max_splits = 1;
+  auto load = [&]() {
+    const int64_t L = lens[b];
+    n = std::max<int64_t>(1, ceil_div(L, chunk));
+    last = static_cast<double>(std::max<int64_t>(0, L - (n - 1) * chunk)) * bytes_per_token + overhead_bytes;
+    max_splits = std::max(max_splits, n);
+  };
+  if (!lens.empty()) load();
+  // start the next CTA at v, if any is left
+  auto next_cta = [&](double v) -> bool {
+    if (b >= lens.size()) return false;
+    const bool is_full = sidx != n - 1;
+    start_cta(v + (is_full ? full : last), is_full);
+    if (++sidx == n) {
       sidx = 0;
       if (++u == units) {
         u = 0;
-        ++b;
+        if (++b < lens.size()) load();
       }
     }
-    return -1.0;
+    return true;
   };
-  for (int i = 0; i < slots; ++i) {
-    const double c = next_cta();
-    if (c < 0) break;
-    running.push(v + c);
-  }
-  while (!running.empty()) {
-    const double rate = std::min(cta_bytes_per_us, hbm / static_cast<double>(running.size()));
-    const double nxt = running.top();
-    running.pop();
+  for (int i = 0; i < slots; ++i)
+    if (!next_cta(0.0)) break;
+  double v = 0.0, t = 0.0;
+  size_t rate_for = 0;   // running count the rate below was computed for
+  double rate = 0.0;
+  while (count + heap.size() > 0) {
+    if (count + heap.size() != rate_for) {
+      rate_for = count + heap.size();
+      rate = std::min(cta_bytes_per_us, hbm / static_cast<double>(rate_for));
+    }
+    double nxt;
+    if (count > 0 && (heap.empty() || ring[head] <= heap.front())) {
+      nxt = ring[head];
+      if (++head == ring.size()) head = 0;
+      --count;
+    } else {
+      nxt = heap.front();
+      std::pop_heap(heap.begin(), heap.end(), later);
+      heap.pop_back();
+    }
     t += (nxt - v) / rate;
     v = nxt;
-    const double c = next_cta();
-    if (c >= 0) running.push(v + c);
+    next_cta(v);
   }
+  return t + (max_splits > 1 ? kMergeLaunchUs : 0.0);
+}
+
+// A lower bound of estimate_decode_us for the same arguments, in O(batch):
+// the running CTAs never move more than the HBM bandwidth in total, nor more
+// than their slots' ceilings, and no CTA finishes faster than its own ceiling.
+double lower_bound_decode_us(const std::vector<int32_t>& lens, int64_t units, int64_t chunk,
+                             int slots, int head_dim, int kv_elem_bytes, const CtaModel& cm,
+                             int num_sms) {
+  const double bytes_per_token = 2.0 * head_dim * kv_elem_bytes;
+  const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
+  const double overhead_bytes = cm.overhead_us * cm.bytes_per_us;
+  double total = 0.0, largest = 0.0;
+  int64_t max_splits = 1;
+  for (const int32_t L : lens) {
+    const int64_t n = std::max<int64_t>(1, ceil_div(L, chunk));
+    max_splits = std::max(max_splits, n);
+    total += static_cast<double>(units) * (static_cast<double>(L) * bytes_per_token +
+                                           static_cast<double>(n) * overhead_bytes);
+    largest = std::max(largest, static_cast<double>(std::min<int64_t>(chunk, L)) * bytes_per_token +
+                                    overhead_bytes);
+  }
+  const double t = std::max({total / hbm, total / (static_cast<double>(slots) * cm.bytes_per_us),
+                             largest / cm.bytes_per_us});
   return t + (max_splits > 1 ? kMergeLaunchUs : 0.0);
 }
 }  // namespace
@@ -175,11 +234,22 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
       cands.push_back(round_up(ceil_div(max_len, s), page_size));
     const int64_t target = ceil_div(total * units, static_cast<int64_t>(slots) * kItemsPerSlot);
     cands.push_back(round_up(target, page_size));
-    double best_t = 0.0;
-    chunk = 0;
+    // Simulate the candidates in increasing order of their lower bound and
+    // skip any whose bound already exceeds the best estimate: the choice is
+    // the exhaustive search's, at a fraction of the simulations (the many-CTA
+    // candidates, the costly ones to simulate, have the highest bounds).
+    std::vector<std::pair<double, int64_t>> order;
     for (int64_t c : cands) {
       c = std::max<int64_t>(c, kMinChunkTokens);
       if (ceil_div(max_len, c) > kMaxSplits) continue;
+      order.emplace_back(lower_bound_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes,
+                                               cm, num_sms), c);
+    }
+    std::sort(order.begin(), order.end());
+    double best_t = 0.0;
+    chunk = 0;
+    for (const auto& [lb, c] : order) {
+      if (chunk != 0 && lb > best_t * (1.0 + 1e-9)) break;
       const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes, cm,
                                           num_sms);
       if (chunk == 0 || t < best_t * (1.0 - 1e-9) || (t <= best_t * (1.0 + 1e-9) && c > chunk)) {
