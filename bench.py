@@ -8,7 +8,11 @@ One step = one pass of the whole hot path over one batch of synthetic input:
      32 q / 8 kv heads, d=128, shuffled 64-token pages) through fa_decode_plan's
      plan and fa_decode_paged (split kernel + merge kernel).
 The line's ``value`` is the prefill throughput in TFLOP/s (causal algorithmic
-FLOPs); the decode half reports HBM GB/s under ``decode``.  ``--workload``
+FLOPs); the decode half reports HBM GB/s under ``decode``.  At one GPU the
+default run then times the other configurations alone, each under ``legs``
+with its own time, roofline and clock record: the 32K GQA causal prefill, the
+long split decode (4 x 131072, the planner's split count plus a sweep of fixed
+counts) and the ragged split decode (1 x 131072 + 63 x 2048).  ``--workload``
 selects a single configuration instead (one line for that configuration);
 ``chunked_prefill_batch`` times a chunked-prefill step (fa_append_kv of the
 chunk's K/V into the paged cache, then fa_prefill_paged over the whole cache).
@@ -159,6 +163,9 @@ class PrefillCase:
         else:
             fa.prefill(self.q, self.k, self.v, self.cu, causal=i.causal, scale=i.scale,
                        out=self.out, lse=self.lse, cu_seqlens_host=i.cu_seqlens)
+        # the schedule the library actually launched (it uses the grid form while
+        # a stream is being captured, or when it has no counter left)
+        self.schedule = fa.prefill_last_schedule()
 
     def run_e2e(self):
         """Host buffers in, host buffers out: H2D copies, the C-ABI call, D2H copies."""
@@ -191,7 +198,7 @@ class PrefillCase:
                 "num_q_heads": i.num_q_heads, "num_kv_heads": i.num_kv_heads,
                 "head_dim": i.head_dim, "causal": bool(i.causal),
                 "inputs": "e4m3 q/k/v, per-tensor scales" if self.fp8 else "bf16",
-                "schedule": os.environ.get("FA_PREFILL_SCHEDULE") == "persistent" and "persistent" or "grid",
+                "schedule": getattr(self, "schedule", None),
                 "algorithmic_tflop": round(self.flops / 1e12, 4)}
 
 
@@ -227,6 +234,21 @@ class DecodeCase:
         self.h_lens = torch.from_numpy(inp.cache_seqlens).pin_memory()
         self.h_out = torch.empty(self.q.shape, dtype=torch.int16).pin_memory()
         self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def replan(self, num_splits=0, kernel="auto"):
+        """A new plan (and workspace) over the same device-resident inputs."""
+        import torch
+        import exact_attention_148_b200 as fa
+        inp = self.inp
+        t0 = time.perf_counter()
+        self.plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=inp.num_q_heads,
+                                   num_kv_heads=inp.num_kv_heads, head_dim=inp.head_dim,
+                                   page_size=inp.page_size, max_pages_per_seq=inp.block_table.shape[1],
+                                   num_splits=num_splits, kv_dtype="e4m3" if self.fp8 else "bf16",
+                                   kernel=kernel, q_len=inp.q_len)
+        self.plan_ms = (time.perf_counter() - t0) * 1e3
+        self.ws = torch.empty(max(self.plan.workspace_bytes, 256), dtype=torch.uint8, device=self.q.device)
+        self.launches = 1 + (1 if self.plan.info.max_splits > 1 else 0)
 
     def run(self):
         import exact_attention_148_b200 as fa
@@ -520,23 +542,27 @@ def time_e2e_overlapped(case, steps, warmup, dist_ctx):
             out_done[b].record(s_out)
         used[b] = True
 
-    for i in range(warmup):
-        one(i)
-    torch.cuda.synchronize()
-    if dist_ctx is not None:
-        dist_ctx.barrier()
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(comp)
-    s_in.wait_event(start)
-    s_out.wait_event(start)
-    for i in range(steps):
-        one(warmup + i)
-    comp.wait_event(out_done[(warmup + steps - 1) % 2])
-    end.record(comp)
-    torch.cuda.synchronize()
-    for dev_attr in slots[0]:
-        setattr(case, dev_attr, slots[0][dev_attr])
+    try:
+        for i in range(warmup):
+            one(i)
+        torch.cuda.synchronize()
+        if dist_ctx is not None:
+            dist_ctx.barrier()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        for i in range(steps):
+            one(warmup + i)
+        comp.wait_event(out_done[(warmup + steps - 1) % 2])
+        end.record(comp)
+        torch.cuda.synchronize()
+    finally:
+        # the case keeps its own buffers even when a call raised part way
+        torch.cuda.synchronize()
+        for dev_attr in slots[0]:
+            setattr(case, dev_attr, slots[0][dev_attr])
     ms = start.elapsed_time(end) / steps
     if dist_ctx is not None:
         ms = dist_ctx.max_over_ranks([ms])[0]
@@ -816,6 +842,69 @@ def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=No
             "peak_source": f"{peak_src} HBM copy", "frac_of_spec": round(achieved / SPEC_PEAKS["hbm_gbs"], 4)}
 
 
+# The other configurations of the benchmark, timed in the default run after the
+# headline step: (workload, split counts swept besides the planner's choice).
+LEGS = [("long_gqa_prefill", ()), ("long_split_decode", (1, 2, 4, 8, 16, 32, 64)),
+        ("ragged_split_decode", ())]
+
+
+def case_roofline(c, ms, peaks, peak_src):
+    """Roofline entry of one case's kernel(s) at `ms` per call."""
+    if isinstance(c, PrefillCase):
+        pers = getattr(c, "schedule", None) == "persistent"
+        e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
+                           measured_traffic("prefill_persist" if pers else "prefill", c.inp.name),
+                           fp8_qk=c.fp8)
+        e["kernel"] = "%s<%d%s>" % ("fa_prefill_persist_kernel" if pers else "fa_prefill_pp_kernel",
+                                    c.inp.head_dim, ", e4m3" if c.fp8 else "")
+        return e
+    e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
+                       measured_traffic("decode_tc" if c.plan.info.tensor_cores else "decode",
+                                        c.inp.name, c))
+    e["kernel"] = ("fa_decode_tc_kernel" if c.plan.info.tensor_cores else "fa_decode_split_kernel") + \
+        ("<e4m3>" if c.fp8 else "") + " + fa_merge_kernel (one decode call)"
+    return e
+
+
+def run_legs(args, device, flush, peaks, peak_src):
+    """Time every other configuration once on this GPU (rank 0's replica):
+    value, ms, roofline and clocks per leg; the long split decode also over a
+    sweep of split counts.  Each leg's inputs are freed before the next."""
+    import torch
+    legs = []
+    steps = max(3, min(args.steps, 10))
+    for workload, sweep in LEGS:
+        c = build_cases(workload, device, 0)[0]
+        sampler = ClockSampler(device.index if device.index is not None else 0)
+        sampler.start()
+        ms = time_cases([c], steps, 3, flush, None)[0] / steps
+        rows = []
+        for ns in sweep:
+            c.replan(ns)
+            t = time_cases([c], steps, 2, flush, None)[0] / steps
+            rows.append({"num_splits": ns, "max_splits": c.plan.info.max_splits, "ms": round(t, 4),
+                         "gbs": round(c.bytes / (t * 1e-3) / 1e9, 1)})
+        clocks = sampler.stop()
+        if sweep:
+            c.replan(0)                      # describe the planner's own choice
+        prefill = isinstance(c, PrefillCase)
+        leg = {"workload": workload,
+               "value": round(c.flops / (ms * 1e-3) / 1e12, 3) if prefill else round(c.bytes / (ms * 1e-3) / 1e9, 1),
+               "unit": "TFLOP/s" if prefill else "GB/s", "ms": round(ms, 4), "steps": steps,
+               "launches_per_call": c.launches,
+               "roofline": case_roofline(c, ms, peaks, peak_src), "clocks": clocks,
+               "config": c.describe()}
+        if sweep:
+            auto = {"num_splits": "auto", "max_splits": c.plan.info.max_splits, "ms": round(ms, 4),
+                    "gbs": leg["value"]}
+            leg["splits_sweep"] = rows + [auto]
+        legs.append(leg)
+        del c
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return legs
+
+
 def run_ours(args):
     import torch
     import exact_attention_148_b200 as fa  # noqa: F401  (fails loudly if the library is missing)
@@ -854,12 +943,7 @@ def run_ours(args):
     rooflines = []
     for c, ms in zip(cases, ms_case):
         if isinstance(c, PrefillCase):
-            pers = os.environ.get("FA_PREFILL_SCHEDULE") == "persistent"
-            e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
-                               measured_traffic("prefill_persist" if pers else "prefill", c.inp.name),
-                               fp8_qk=c.fp8)
-            e["kernel"] = "%s<%d%s>" % ("fa_prefill_persist_kernel" if pers else "fa_prefill_pp_kernel",
-                                        c.inp.head_dim, ", e4m3" if c.fp8 else "")
+            e = case_roofline(c, ms, peaks, peak_src)
         elif isinstance(c, ChunkedAttnCase):
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
                                measured_traffic("prefill", c.inp.name))
@@ -872,11 +956,7 @@ def run_ours(args):
                                measured_traffic("append", c.inp.name))
             e["kernel"] = "fa_append_kv_kernel<%d>" % c.inp.head_dim
         else:
-            e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
-                               measured_traffic("decode_tc" if c.plan.info.tensor_cores else "decode",
-                                                c.inp.name, c))
-            e["kernel"] = ("fa_decode_tc_kernel" if c.plan.info.tensor_cores else "fa_decode_split_kernel") + \
-                ("<e4m3>" if c.fp8 else "") + " + fa_merge_kernel (one decode call)"
+            e = case_roofline(c, ms, peaks, peak_src)
         e["workload"] = c.inp.name
         e["ms_per_launch"] = round(ms / c.launches, 4)
         rooflines.append(e)
@@ -949,6 +1029,12 @@ def run_ours(args):
                        "steps": ("overlapped: step s+1 copies in and step s-1 copies out while step s "
                                  "computes (double-buffered device inputs and outputs)" if overlapped
                                  else "serial: copy in, compute, copy out, one step after another")}
+    if args.workload == "default" and N == 1 and not args.no_legs:
+        line["legs"] = run_legs(args, device, flush, peaks, peak_src)
+        line["legs_device_status"] = fa.device_status(clear=True)
+        line["legs_note"] = ("the benchmark's other configurations, each timed alone after the "
+                             "headline step (CUDA events, L2 flushed before every step); not part of "
+                             "value, ms_per_step or gpu_launches")
     line["gpu_launches"] = int(launches)
     line["clocks"] = clocks
     line["device_status"] = status
@@ -1037,13 +1123,15 @@ def main():
     ap.add_argument("--decode-kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"])
     ap.add_argument("--decode-heads", default=None, help="HQ:HKV override for a decode workload")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="default workload: skip the other configurations' legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
     ap.add_argument("--e2e-overlap", action="store_true",
                     help="end-to-end leg with consecutive steps' copies and compute overlapped")
     ap.add_argument("--prefill-schedule", default=None, choices=["grid", "persistent"],
                     help="packed prefill: one CTA per work item (grid) or one per SM (persistent); "
-                         "default: the library's (FA_PREFILL_SCHEDULE, else grid)")
+                         "default: the library's (FA_PREFILL_SCHEDULE, else persistent)")
     args = ap.parse_args()
     if args.prefill_schedule is not None:
         os.environ["FA_PREFILL_SCHEDULE"] = args.prefill_schedule

@@ -244,13 +244,17 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
       const int mine = (i0 + lane < num_pg) ? bt_row[i0 + lane] : 0;
       const int cnt = min(32, num_pg - i0);
       for (int ii = 0; ii < cnt; ++ii) {
-        const int phys = __shfl_sync(0xffffffffu, mine, ii);
+        int phys = __shfl_sync(0xffffffffu, mine, ii);
         if (lane == 0) {
           const int i = i0 + ii;
           const int st = i % C::STAGES;
           if (mbar_wait(bar_empty(st), ((i / C::STAGES) & 1) ^ 1, abort_flag)) {
-            if (phys < 0 || phys >= p.num_pages) record_status(FA_ERR_BAD_PAGE);
-            // An out-of-range page id reads as zeros (TMA bounds), never faults.
+            // A page id outside the pool is recorded and replaced by num_pages,
+            // one past the tensor map's last page, which TMA reads as zeros.
+            if (phys < 0 || phys >= p.num_pages) {
+              record_status(FA_ERR_BAD_PAGE);
+              phys = p.num_pages;
+            }
             int c1 = 0, c2 = 0, c3 = 0;
             c1 = (p.head_coord == 1) ? kv_head : (p.page_coord == 1 ? phys : 0);
             c2 = (p.head_coord == 2) ? kv_head : (p.page_coord == 2 ? phys : 0);

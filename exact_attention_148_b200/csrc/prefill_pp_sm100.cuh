@@ -30,7 +30,7 @@
 // masking, are computed on the FMA and ALU pipes instead, as
 // 2^x = 2^n * p(f), n = round(x), f = x - n in [-1/2, 1/2] (Cody & Waite
 // argument reduction), with a degree-3 minimax polynomial p fitted by the Remez
-// exchange algorithm (relative error 7.5e-5, see tools/fit_exp2_poly.py), far
+// exchange algorithm (relative error 7.5e-5; tests/test_exp2_poly.py re-derives it), far
 // below the 2^-9 rounding P gets when it is stored as bf16.  The rounding uses
 // the float adder (adding 1.5*2^23 leaves round(x) in the low mantissa bits)
 // and 2^n is added straight into the exponent field, so no instruction of this

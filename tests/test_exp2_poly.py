@@ -1,6 +1,12 @@
 """The prefill kernel's FMA-pipe exp2 (Cody-Waite reduction + degree-3 Remez
 polynomial), emulated in float32 on the CPU with the constants read from the
-kernel source, against numpy's exp2 and the fit's stated error bound."""
+kernel source, against numpy's exp2 and the fit's stated error bound.
+
+The constants themselves are re-derived here: 2^x = 2^n * 2^f with
+n = round(x), f = x - n in [-1/2, 1/2] (Cody & Waite, "Software Manual for the
+Elementary Functions", 1980), and p(f) the degree-3 polynomial of least
+maximum relative error on that interval, found by the Remez exchange
+algorithm."""
 import os
 import re
 
@@ -57,8 +63,37 @@ def test_exp2_poly_is_far_below_bf16_rounding():
     assert rel.max() < 2.0 ** -9 / 10
 
 
-def test_fit_script_reproduces_kernel_coefficients():
-    from exact_attention_148_b200.tools.fit_exp2_poly import remez_rel
+def remez_rel(deg=3, iters=40, a=-0.5, b=0.5):
+    """Minimax-relative-error polynomial for 2^f on [a, b] (Remez exchange).
+    Returns (coefficients c0..c_deg, max relative error)."""
+    n = deg + 2
+    xs = 0.5 * (a + b) - 0.5 * (b - a) * np.cos(np.pi * np.arange(n) / (n - 1))
+    grid = np.linspace(a, b, 200001)
+    target = np.exp2(grid)
+    for _ in range(iters):
+        # solve p(x_i) + (-1)^i E 2^{x_i} = 2^{x_i} on the reference points
+        A = np.zeros((n, n))
+        for i, x in enumerate(xs):
+            A[i, :deg + 1] = x ** np.arange(deg + 1)
+            A[i, deg + 1] = (-1) ** i * np.exp2(x)
+        c = np.linalg.solve(A, np.exp2(xs))[:deg + 1]
+        err = (np.polyval(c[::-1], grid) - target) / target
+        # new reference: the largest error of each sign run, n of them alternating
+        s = np.sign(err)
+        idx, start = [], 0
+        for k in range(1, len(grid) + 1):
+            if k == len(grid) or s[k] != s[start]:
+                seg = np.arange(start, k)
+                idx.append(seg[np.argmax(np.abs(err[seg]))])
+                start = k
+        if len(idx) >= n:
+            while len(idx) > n:
+                idx.pop(0 if abs(err[idx[0]]) < abs(err[idx[-1]]) else len(idx) - 1)
+            xs = grid[idx]
+    return c, np.max(np.abs(err))
+
+
+def test_kernel_coefficients_are_the_remez_fit():
     c, err = remez_rel()
     assert err < 8e-5
     for a, b in zip(c, kernel_coefficients()):

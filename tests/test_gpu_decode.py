@@ -27,17 +27,6 @@ def check_all_rows(inp, num_splits=0, what="", kernel="auto"):
     return out, lse, plan
 
 
-def check_sampled(inp, rows, num_splits=0, what="", dev=None):
-    out, lse, plan = decode_on_gpu(inp, num_splits, dev=dev)
-    o_ref, l_ref = oracle_rows(inp, rows)
-    bi = np.array([r[0] for r in rows])
-    hi = np.array([r[1] for r in rows])
-    o = out.float().cpu().numpy()[bi, hi].astype(np.float64)
-    l = lse.cpu().numpy()[bi, hi]
-    compare(o, l, o_ref, l_ref, what)
-    return plan
-
-
 SMALL_LENS = [1, 63, 64, 65, 1000, 4097]
 
 
@@ -122,18 +111,35 @@ def test_deterministic():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_bad_page_id_is_reported_not_faulted():
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+@pytest.mark.parametrize("bad_id", ["past_end", "negative"])
+def test_bad_page_id_is_reported_not_faulted(kernel, bad_id):
+    """A block_table entry outside the pool is recorded and read as a page of
+    zeros (the kernels replace it by one past the last page, which the tensor
+    map's bounds turn into a zero fill); the other pages are unaffected."""
     import exact_attention_148_b200 as fa
     inp = W.make_decode([200], 4, 4, 128, seed=1100)
     fa.device_status(clear=True)
     bt = inp.block_table.copy()
-    bt[0, 1] = inp.num_pages + 3          # outside the pool: reads as zeros
+    bt[0, 1] = inp.num_pages + 3 if bad_id == "past_end" else -5
     bad = W.DecodeInputs(inp.name, inp.q_bits, inp.k_pages_bits, inp.v_pages_bits, bt,
                          inp.cache_seqlens, inp.scale, inp.layout, inp.page_size)
-    out, lse, _ = decode_on_gpu(bad, 1)
+    out, lse, _ = decode_on_gpu(bad, 1, kernel=kernel)
     assert fa.device_status(clear=True) == fa.FA_ERR_BAD_PAGE
     assert np.isfinite(out.float().cpu().numpy()).all()
-    decode_on_gpu(inp, 1)
+    # the oracle on the same cache with that page's keys and values set to zero
+    k = inp.k_pages_bits.copy()
+    v = inp.v_pages_bits.copy()
+    zero_page = inp.num_pages                # an extra all-zero page for the oracle only
+    k = np.concatenate([k, np.zeros_like(k[:1])], axis=0)
+    v = np.concatenate([v, np.zeros_like(v[:1])], axis=0)
+    bt_ref = inp.block_table.copy()
+    bt_ref[0, 1] = zero_page
+    rows = [(0, h) for h in range(4)]
+    o_ref, l_ref = oracle.paged_decode_rows_ref(inp.q_bits, k, v, bt_ref, inp.cache_seqlens, inp.scale,
+                                                rows, inp.page_size, inp.layout, to_f64=W.as_f64)
+    compare(bf16_to_f64(out[0]), lse[0].cpu().numpy(), o_ref, l_ref, f"bad page ({kernel}, {bad_id})")
+    decode_on_gpu(inp, 1, kernel=kernel)
     assert fa.device_status(clear=True) == 0
 
 
@@ -147,31 +153,50 @@ def test_longer_cache_than_planned_is_reported():
     assert fa.device_status(clear=True) == fa.FA_ERR_PLAN_MISMATCH
 
 
-def _sample(inp, n, seed):
-    g = np.random.default_rng(seed)
-    rows = {(int(np.argmax(inp.cache_seqlens)), 0), (int(np.argmin(inp.cache_seqlens)), inp.num_q_heads - 1)}
-    while len(rows) < n:
-        rows.add((int(g.integers(inp.batch)), int(g.integers(inp.num_q_heads))))
-    return sorted(rows)
+_FULL_ORACLE = {}
 
 
-def test_paged_decode_batch_config_sampled():
-    inp = W.paged_decode_batch()
-    check_sampled(inp, _sample(inp, 96, 3), 0, "paged decode batch (64 req, 32q/8kv)")
+def oracle_every_row(inp):
+    """The oracle on every (request, head) row of a workload, kept for the
+    workload last asked for (its inputs are seeded, so one result serves every
+    split count and kernel)."""
+    if inp.name not in _FULL_ORACLE:
+        _FULL_ORACLE.clear()
+        rows = [(b, h) for b in range(inp.batch) for h in range(inp.num_q_heads)]
+        _FULL_ORACLE[inp.name] = oracle_rows(inp, rows)
+    return _FULL_ORACLE[inp.name]
 
 
-def test_long_split_decode_config_sampled():
-    inp = W.long_split_decode()
+def check_every_row(inp, settings, what):
+    """Every output row of the full-size workload against the oracle, for each
+    (num_splits, kernel) in settings, in the launch configuration bench.py times."""
+    import exact_attention_148_b200 as fa
+    o_ref, l_ref = oracle_every_row(inp)
     dev = decode_device_inputs(inp)
-    rows = _sample(inp, 24, 4)
-    for s in (0, 1, 8, 64):
-        check_sampled(inp, rows, s, f"long split decode splits={s}", dev=dev)
+    fa.device_status(clear=True)
+    for s, kernel in settings:
+        out, lse, plan = decode_on_gpu(inp, s, dev=dev, kernel=kernel)
+        compare(bf16_to_f64(out).reshape(-1, inp.head_dim), lse.cpu().numpy().reshape(-1), o_ref, l_ref,
+                f"{what} splits={s or 'auto'} ({plan.info.max_splits}) kernel={kernel}")
+        assert fa.device_status(clear=True) == 0, what
 
 
-def test_ragged_split_decode_config_sampled():
+def test_paged_decode_batch_config_every_row():
+    inp = W.paged_decode_batch()
+    check_every_row(inp, [(0, "auto"), (0, "cuda_cores"), (16, "auto")],
+                    "paged decode batch (64 req, 32q/8kv)")
+
+
+def test_long_split_decode_config_every_row():
+    inp = W.long_split_decode()
+    check_every_row(inp, [(0, "auto"), (1, "auto"), (8, "auto"), (64, "auto"), (0, "tensor_cores")],
+                    "long split decode (4 x 131072)")
+
+
+def test_ragged_split_decode_config_every_row():
     inp = W.ragged_split_decode()
-    rows = [(0, h) for h in (0, 7, 31)] + _sample(inp, 24, 5)
-    check_sampled(inp, sorted(set(rows)), 0, "ragged split decode")
+    check_every_row(inp, [(0, "auto"), (64, "auto"), (0, "tensor_cores")],
+                    "ragged split decode (1 x 131072 + 63 x 2048)")
 
 
 @pytest.mark.parametrize("kernel", ["tensor_cores", "cuda_cores"])

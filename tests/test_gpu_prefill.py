@@ -56,7 +56,7 @@ RAGGED = [1, 127, 128, 129, 300, 513]
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 1), (8, 2)])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 1), (8, 2), (16, 2), (8, 1), (6, 2), (3, 1)])
 @pytest.mark.parametrize("causal", [True, False])
 def test_small_varlen(d, hq, hkv, causal):
     inp = W.make_prefill(RAGGED, hq, hkv, d, causal=causal, seed=100 + d + hq + hkv)
@@ -83,6 +83,52 @@ def test_varlen_config_sampled():
 def test_long_gqa_config_sampled():
     inp = W.long_gqa_prefill()
     check_sampled(inp, 512, 2, "32K GQA causal prefill")
+
+
+def check_whole_heads(inp, heads, what):
+    """Every row of the chosen query heads of a full-size workload against the
+    oracle run on those heads and their kv heads alone (heads are independent,
+    and head h reads kv head h // (Hq / Hkv))."""
+    out, lse = prefill_on_gpu(inp)
+    G = inp.num_q_heads // inp.num_kv_heads
+    # one chosen q head per kv head, ordered by kv head, so that q head j of the
+    # sub-problem maps onto its kv head j
+    heads = sorted(heads)
+    kv = [h // G for h in heads]
+    assert len(set(kv)) == len(kv), "one q head per kv head"
+    o_ref, l_ref = oracle.attention_ref(W.as_f64(inp.q_bits[:, heads]), W.as_f64(inp.k_bits[:, kv]),
+                                        W.as_f64(inp.v_bits[:, kv]), inp.cu_seqlens, inp.causal,
+                                        inp.scale)
+    o = bf16_to_f64(out[:, heads])
+    l = lse.cpu().numpy()[:, heads]
+    return compare(o, l, o_ref, l_ref, what)
+
+
+def test_varlen_config_whole_heads():
+    """Four whole heads (every one of the 20,730 packed rows) of the varlen config."""
+    inp = W.varlen_causal_prefill()
+    check_whole_heads(inp, [0, 9, 22, 31], "varlen causal prefill, heads 0/9/22/31")
+
+
+def test_long_gqa_config_dense_rows():
+    """The 32K GQA config: every 32nd row of two heads on different kv heads,
+    plus every row of the first and last 128-row q tiles of both."""
+    inp = W.long_gqa_prefill()
+    out, lse = prefill_on_gpu(inp)
+    T = int(inp.cu_seqlens[-1])
+    heads = (0, 31)
+    tok = sorted(set(range(0, T, 32)) | set(range(128)) | set(range(T - 128, T)))
+    G = inp.num_q_heads // inp.num_kv_heads
+    q = W.bf16_bits_to_f32(inp.q_bits[:, list(heads)])
+    k = W.bf16_bits_to_f32(inp.k_bits[:, [h // G for h in heads]]).astype(np.float64)
+    v = W.bf16_bits_to_f32(inp.v_bits[:, [h // G for h in heads]]).astype(np.float64)
+    rows = [(t, j) for j in range(len(heads)) for t in tok]
+    o_ref, l_ref = oracle.attention_rows_ref(q, k, v, inp.cu_seqlens, inp.causal, inp.scale, rows)
+    ti = np.array([r[0] for r in rows])
+    hi = np.array([heads[r[1]] for r in rows])
+    o = out.float().cpu().numpy()[ti, hi].astype(np.float64)
+    l = lse.cpu().numpy()[ti, hi]
+    compare(o, l, o_ref, l_ref, "32K GQA causal prefill, dense rows of heads 0 and 31")
 
 
 def test_sequences_are_isolated():

@@ -7,16 +7,19 @@ device), processes with a device-memory budget fixed at start-up.  For them
 the library offers a decode entry point with no workspace argument: the split
 partials go to one static 16 MiB device array inside the library.
 
-These tests call that entry point through the C ABI and check its output
-against the workspace entry point (fa_decode_paged) on two calls in a row with
+These tests call that entry point through the C ABI on two calls in a row with
 different inputs, so whatever the first call left in the shared array cannot
-leak into the second.  This file is collected last on purpose.
+leak into the second.  The static and workspace entry points run the same
+kernels with the same plan, so their results must agree bit for bit; the
+static result is also checked against the fp64 oracle.  This file is collected
+last on purpose.
 """
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle
 import workloads as W
 from tests.gpu_util import bf16_to_f64, compare, decode_device_inputs
 
@@ -35,7 +38,8 @@ def _static_call(lib, dev, inp, plan, out, lse):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-def test_static_scratch_decode_matches_workspace_decode():
+@pytest.mark.parametrize("kernel", ["auto", "cuda_cores"])
+def test_static_scratch_decode_matches_workspace_decode(kernel):
     import torch
     import exact_attention_148_b200 as fa
     lib = fa.library()
@@ -44,7 +48,8 @@ def test_static_scratch_decode_matches_workspace_decode():
         inp = W.make_decode(lens, hq, hkv, 128, seed=seed)
         dev = decode_device_inputs(inp)
         plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
-                              max_pages_per_seq=inp.block_table.shape[1], num_splits=4)
+                              max_pages_per_seq=inp.block_table.shape[1], num_splits=4,
+                              kernel=kernel)
         assert 0 < plan.workspace_bytes <= fa.STATIC_SCRATCH_BYTES
         ref_out, ref_lse = fa.decode_paged(dev["q"], dev["k"], dev["v"], dev["bt"], dev["lens"], plan)
         out = torch.full_like(ref_out, float("nan"))
@@ -52,8 +57,14 @@ def test_static_scratch_decode_matches_workspace_decode():
         status = _static_call(lib, dev, inp, plan, out, lse)
         assert status == fa.FA_OK, fa.strerror(status)
         torch.cuda.synchronize()
-        compare(bf16_to_f64(out), lse.cpu().numpy(), bf16_to_f64(ref_out), ref_lse.cpu().numpy(),
-                f"static-scratch decode, call {call + 1}")
+        what = f"static-scratch decode ({kernel}), call {call + 1}"
+        assert torch.equal(out, ref_out), f"{what}: O differs from the workspace entry point"
+        assert torch.equal(lse, ref_lse), f"{what}: LSE differs from the workspace entry point"
+        o_ref, l_ref = oracle.paged_decode_ref(inp.q_bits, inp.k_pages_bits, inp.v_pages_bits,
+                                               inp.block_table, inp.cache_seqlens, inp.scale,
+                                               inp.page_size, inp.layout, to_f64=W.as_f64)
+        compare(bf16_to_f64(out), lse.cpu().numpy(), o_ref, l_ref, what + " vs oracle")
+        assert fa.device_status(clear=True) == 0
 
 
 def test_static_scratch_rejects_plans_larger_than_the_array():
@@ -67,3 +78,23 @@ def test_static_scratch_rejects_plans_larger_than_the_array():
     status = lib.fa_decode_paged_static(A, A, A, 100, 64 * 8 * 128, 8 * 128, 128, A, A, plan.handle,
                                         float("nan"), A, None, None)
     assert status == fa.FA_ERR_WORKSPACE
+
+
+def test_static_scratch_rejects_an_e4m3_plan_before_any_launch():
+    """The static entry point reads a bf16 cache; a plan made for an E4M3 cache
+    is refused with FA_ERR_PLAN_MISMATCH and nothing is written."""
+    import torch
+    import exact_attention_148_b200 as fa
+    lib = fa.library()
+    inp = W.make_decode([300, 900], 8, 2, 128, seed=13)
+    dev = decode_device_inputs(inp)
+    plan = fa.decode_plan(inp.cache_seqlens, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                          max_pages_per_seq=inp.block_table.shape[1], num_splits=2, kv_dtype="e4m3")
+    assert plan.workspace_bytes <= fa.STATIC_SCRATCH_BYTES
+    out = torch.full((inp.batch, 8, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((inp.batch, 8), 7.0, dtype=torch.float32, device="cuda")
+    status = _static_call(lib, dev, inp, plan, out, lse)
+    assert status == fa.FA_ERR_PLAN_MISMATCH, fa.strerror(status)
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0) and torch.all(lse == 7.0)
+    assert fa.device_status(clear=True) == 0
