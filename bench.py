@@ -924,7 +924,7 @@ def run_ours(args):
     status = fa.device_status(clear=True)
 
     e2e_case = None
-    overlapped = args.e2e_overlap and all(hasattr(c, "e2e_fields") for c in cases)
+    overlapped = not args.e2e_serial and all(hasattr(c, "e2e_fields") for c in cases)
     if not args.no_e2e:
         if overlapped:
             e2e_steps = max(2, min(args.steps, 8))
@@ -1127,8 +1127,9 @@ def main():
                     help="default workload: skip the other configurations' legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
-    ap.add_argument("--e2e-overlap", action="store_true",
-                    help="end-to-end leg with consecutive steps' copies and compute overlapped")
+    ap.add_argument("--e2e-serial", action="store_true",
+                    help="end-to-end leg without overlap: copy in, compute, copy out, one step after "
+                         "another (default: consecutive steps' copies overlap the compute)")
     ap.add_argument("--prefill-schedule", default=None, choices=["grid", "persistent"],
                     help="packed prefill: one CTA per work item (grid) or one per SM (persistent); "
                          "default: the library's (FA_PREFILL_SCHEDULE, else persistent)")
