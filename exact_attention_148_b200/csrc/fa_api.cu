@@ -403,6 +403,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* cu_
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_dev;
+  prm.total_q = static_cast<int>(T);
   prm.num_q_heads = num_q_heads;
   prm.group = group;
   prm.causal = causal ? 1 : 0;
@@ -511,6 +512,7 @@ FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_q_dev;
+  prm.total_q = static_cast<int>(T);
   prm.block_table = block_table;
   prm.cache_seqlens = cache_seqlens_dev;
   prm.max_pages = max_pages_per_seq;

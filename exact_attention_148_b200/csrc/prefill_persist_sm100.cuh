@@ -20,11 +20,13 @@
 //   * the softmax warps write O(i) and only then read S(i+1, 0) and arrive for
 //     PV(i+1, 0), which overwrites O, so the O columns need no new barrier.
 //
-// Item ids pass from the producer warp (which takes them from the counter)
-// to the other roles through a small shared-memory queue guarded by
-// item_full / item_empty mbarriers.  Every role takes every item, so all
-// per-role counters (ring entries, Q loads, tiles per slot, f16 V tiles)
-// advance identically.  The counter pair {next item, CTAs finished} is reset
+// Items pass from the producer warp (which takes their ids from the counter
+// and decodes them) to the other roles, decoded, through a small
+// shared-memory queue guarded by item_full / item_empty mbarriers, so no role
+// but the producer reads global memory between items.  Every role takes every
+// item, so all per-role counters (ring entries, Q loads, tiles per slot, f16
+// V tiles) advance identically.  While an item runs, the producer has already
+// claimed the next one and asked L2 for its Q tiles and first K/V tiles.  The counter pair {next item, CTAs finished} is reset
 // by the last CTA to finish, ready for the next launch on the same stream;
 // the host gives each stream its own pair.
 #pragma once
@@ -36,13 +38,27 @@ namespace fa {
 constexpr int kPersistQueue = 4;     // item ids in flight between the producer and the others
 constexpr int kSchedSlots = 256;     // counter pairs: one per stream that launches this kernel
 
+// One work item: two 128-row query slots of one sequence that read the same
+// K/V tiles (two heads of a kv head at one q tile when the GQA group is even,
+// else two consecutive q tiles of one head).  Same numbering as the grid
+// form's CTA index: groups in launch order, heaviest q tiles first in a group.
+struct PrefillItem {
+  int id;          // item number, or -1: no more work
+  int s0;          // first token of the sequence
+  int L;           // its length (queries = keys)
+  int kv_head;
+  int qtile[2];
+  int head[2];
+  int n_kv[2];     // key tiles of each slot (0: slot unused)
+};
+
 template <int D, bool F8 = false>
 struct PrefillPersistCfg {
   using B = PrefillPPCfg<D, F8>;
   // B's barriers, then q_empty[2], item_full[kPersistQueue], item_empty[kPersistQueue]
   static constexpr int NUM_BARS = B::NUM_BARS + 2 + 2 * kPersistQueue;
-  static constexpr int QUEUE_OFF = B::BAR_OFF + NUM_BARS * 8;
-  static constexpr int MISC_OFF = QUEUE_OFF + 4 * kPersistQueue;
+  static constexpr int QUEUE_OFF = (B::BAR_OFF + NUM_BARS * 8 + 15) & ~15;
+  static constexpr int MISC_OFF = QUEUE_OFF + static_cast<int>(sizeof(PrefillItem)) * kPersistQueue;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr int THREADS = B::THREADS;
   // roles that take each item from the queue: the MMA thread, 8 softmax warps,
@@ -59,19 +75,10 @@ struct PrefillPersistParams {
   int total_items;     // work items of this launch
 };
 
-// One work item: two 128-row query slots of one sequence that read the same
-// K/V tiles (two heads of a kv head at one q tile when the GQA group is even,
-// else two consecutive q tiles of one head).  Same numbering as the grid
-// form's CTA index: groups in launch order, heaviest q tiles first in a group.
-struct PrefillItem {
-  int s0;          // first token of the sequence
-  int L;           // its length (queries = keys)
-  int kv_head;
-  int qtile[2];
-  int head[2];
-  int n_kv[2];     // key tiles of each slot (0: slot unused)
-};
-
+// Decode item idx.  The sequence bounds come from the device cu_seqlens; a
+// sequence that leaves the T packed rows, or whose tile count differs from
+// what the host planned for its group (cu_seqlens_dev != cu_seqlens_host), is
+// recorded as FA_ERR_PLAN_MISMATCH and becomes an empty item.
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int idx, int BM, int BN) {
   int lo = 0, hi = p.num_groups - 1;
   while (lo < hi) {
@@ -79,14 +86,27 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     if (p.group_start[mid] <= idx) lo = mid; else hi = mid - 1;
   }
   PrefillItem w;
+  w.id = idx;
   const int seq = static_cast<int>(p.group_id[lo] >> 16);
   w.kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
   const int rank = idx - p.group_start[lo];
   w.s0 = p.cu_seqlens[seq];
   w.L = p.cu_seqlens[seq + 1] - w.s0;
-  const int n_qtiles = (w.L + BM - 1) / BM;
-  const int n_ktiles = (w.L + BN - 1) / BN;
+  const bool in_rows = w.s0 >= 0 && w.L >= 1 && w.s0 <= p.total_q - w.L;
+  const int n_qtiles = in_rows ? (w.L + BM - 1) / BM : 0;
+  const int n_ktiles = in_rows ? (w.L + BN - 1) / BN : 0;
   const int G = p.group;
+  const int planned = p.group_start[lo + 1] - p.group_start[lo];
+  const int derived = ((G & 1) == 0) ? n_qtiles * (G >> 1) : ((n_qtiles + 1) >> 1) * G;
+  if (!in_rows || derived != planned) {
+    if (rank == 0) record_status(FA_ERR_PLAN_MISMATCH);
+    w.s0 = 0;
+    w.L = 0;
+    w.qtile[0] = w.qtile[1] = -1;
+    w.head[0] = w.head[1] = 0;
+    w.n_kv[0] = w.n_kv[1] = 0;
+    return w;
+  }
   if ((G & 1) == 0) {
     const int half = G >> 1;
     const int t = n_qtiles - 1 - rank / half;
@@ -140,7 +160,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
   auto bar_q_empty = [&](int k) { return bars + 8 * (B::NUM_BARS + k); };
   auto bar_item_full = [&](int i) { return bars + 8 * (B::NUM_BARS + 2 + i); };
   auto bar_item_empty = [&](int i) { return bars + 8 * (B::NUM_BARS + 2 + QD + i); };
-  volatile int* queue = reinterpret_cast<volatile int*>(smem + C::QUEUE_OFF);
+  PrefillItem* queue = reinterpret_cast<PrefillItem*>(smem + C::QUEUE_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -181,15 +201,19 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-  // A consumer warp's next item id (-1: no more work; -2: aborted).  All
-  // lanes wait; lane 0 releases the queue entry once the id is in registers.
-  auto take_item_warp = [&](int n) -> int {
+  // A consumer warp's next item (id -1: no more work; -2: aborted).  All
+  // lanes wait; lane 0 releases the queue entry once the item is in registers.
+  auto take_item_warp = [&](int n) -> PrefillItem {
     const int qi = n % QD;
-    if (!__all_sync(0xffffffffu, mbar_wait(bar_item_full(qi), (n / QD) & 1, abort_flag))) return -2;
-    const int it = queue[qi];
+    PrefillItem w;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_item_full(qi), (n / QD) & 1, abort_flag))) {
+      w.id = -2;
+      return w;
+    }
+    w = queue[qi];
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_item_empty(qi));
-    return it;
+    return w;
   };
 
   if (warp == 8) {
@@ -204,19 +228,43 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         for (int c = 0; c < B::CHUNKS; ++c)
           tma_load_3d(q_s + k * B::TILE_BYTES + c * B::CHUNK_BYTES, &p.tm_q, bar, c * 64, h, row0);
       };
+      // Claim an item, decode it and ask L2 for its Q tiles and first K/V
+      // tiles, which the TMA loads of the next item then find there.
+      auto claim = [&]() -> PrefillItem {
+        const int id = static_cast<int>(atomicAdd(pp.sched, 1u));
+        PrefillItem w;
+        if (id >= pp.total_items) {
+          w.id = -1;
+          return w;
+        }
+        w = prefill_item(p, id, B::BM, B::BN);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          if (w.n_kv[k] > 0)
+#pragma unroll
+            for (int c = 0; c < B::CHUNKS; ++c)
+              tma_prefetch_l2_3d(&p.tm_q, c * 64, w.head[k], w.s0 + w.qtile[k] * B::BM);
+        const int pre = min(max(w.n_kv[0], w.n_kv[1]), 2);
+        for (int j = 0; j < pre; ++j)
+#pragma unroll
+          for (int c = 0; c < B::CHUNKS; ++c) {
+            tma_prefetch_l2_3d(&p.tm_k, c * 64, w.kv_head, w.s0 + j * B::BN);
+            tma_prefetch_l2_3d(&p.tm_v, c * 64, w.kv_head, w.s0 + j * B::BN);
+          }
+        return w;
+      };
       uint32_t issued = 0;          // ring entries issued
       int qc0 = 0, qc1 = 0;         // Q loads of each slot
-      int next = static_cast<int>(atomicAdd(pp.sched, 1u));
+      PrefillItem next = claim();
       bool ok = true;
       for (int n = 0; ok; ++n) {
-        const int it = next < pp.total_items ? next : -1;
+        const PrefillItem w = next;
         const int qi = n % QD;
         if (!mbar_wait(bar_item_empty(qi), ((n / QD) & 1) ^ 1, abort_flag)) break;
-        queue[qi] = it;
+        queue[qi] = w;
         mbar_arrive(bar_item_full(qi));
-        if (it < 0) break;
-        next = static_cast<int>(atomicAdd(pp.sched, 1u));   // claimed now, started after this item
-        const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+        if (w.id < 0) break;
+        next = claim();   // claimed and prefetched now, started after this item
         const int n_max = max(w.n_kv[0], w.n_kv[1]);
         // ring entries K_0, V_0, K_1, V_1, ...; both Q tiles right after K_0
         for (int e = 0; e < 2 * n_max; ++e) {
@@ -293,12 +341,12 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
       for (int n = 0; ok; ++n) {
         const int qi = n % QD;
         if (!mbar_wait(bar_item_full(qi), (n / QD) & 1, abort_flag)) break;
-        const int it = queue[qi];
+        const PrefillItem w = queue[qi];
         mbar_arrive(bar_item_empty(qi));
-        if (it < 0) break;
-        const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+        if (w.id < 0) break;
         const int nk0 = w.n_kv[0], nk1 = w.n_kv[1];
         const int n_max = max(nk0, nk1);
+        if (n_max == 0) continue;   // nothing loaded for an empty item
         // first scores of both slots (K_0 is entry `ring`)
         if (!mbar_wait(bar_kv_full(ring), (ring / NS) & 1, abort_flag)) break;
         if (nk0 > 0) {
@@ -367,9 +415,8 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
     uint32_t ring = 0;
     int vcount = 0;
     for (int n = 0;; ++n) {
-      const int it = take_item_warp(n);
-      if (it < 0) break;
-      const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+      const PrefillItem w = take_item_warp(n);
+      if (w.id < 0) break;
       const int n_max = max(w.n_kv[0], w.n_kv[1]);
       bool ok = true;
       for (int j = 0; j < n_max; ++j, ++vcount) {
@@ -416,9 +463,8 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
     const uint32_t oc = tmem + lane_base + 256u + (k ? D : 0);
     int tiles = 0;                                 // key tiles of this slot before the item
     for (int n = 0;; ++n) {
-      const int it = take_item_warp(n);
-      if (it < 0) break;
-      const PrefillItem w = prefill_item(p, it, B::BM, B::BN);
+      const PrefillItem w = take_item_warp(n);
+      if (w.id < 0) break;
       const int nk = k ? w.n_kv[1] : w.n_kv[0];   // (k is not a compile-time index)
       if (nk == 0) continue;
       const int my_qtile = k ? w.qtile[1] : w.qtile[0];
@@ -432,84 +478,13 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         const int g = tiles + j;
         if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(k), g & 1, abort_flag))) { ok = false; break; }
         tc_fence_after_sync();
-        uint32_t s[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_x32(sc + c * 32, s[c]);
-        tmem_ld_wait(s[0]);
-        reg_dep(s[1]);
-        reg_dep(s[2]);
-        reg_dep(s[3]);
-
+        // key tiles reaching past tile_last need the mask
         const bool masked = j * B::BN + B::BN - 1 > tile_last;
-        if (masked) {
-          const int lim = row_last - j * B::BN;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c * 32 + i > lim) s[c][i] = __float_as_uint(-INFINITY);
-        }
-        float mx[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          mx[c] = fmax3(__uint_as_float(s[c][0]), __uint_as_float(s[c][1]), __uint_as_float(s[c][2]));
-#pragma unroll
-          for (int i = 3; i < 31; i += 2)
-            mx[c] = fmax3(mx[c], __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
-          mx[c] = fmaxf(mx[c], __uint_as_float(s[c][31]));
-        }
-        const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        const float m_tile = rmax * p.scale_log2;
-        float alpha = 1.0f;
-        bool rescale = false;
-        if (j == 0) {
-          m_ref = (m_tile == -INFINITY) ? 0.0f : m_tile;
-        } else {
-          const bool need = m_tile > m_ref + kRescaleThreshold;
-          rescale = __any_sync(0xffffffffu, need);
-          if (need) {
-            alpha = ex2_approx(m_ref - m_tile);
-            m_ref = m_tile;
-          }
-        }
-        const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
-        const float2 neg_m2 = make_float2(-m_ref, -m_ref);
-        float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 x = __ffma2_rn(
-                make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), scale2, neg_m2);
-            const float p0 = ex2_approx(x.x);
-            const float p1 = ex2_approx(x.y);
-            ps[i & 3].x += p0;
-            ps[i & 3].y += p1;
-            pk[i] = F8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-          }
-          tmem_st_x16(sc + c * 16, pk);
-        }
-        l_sum = l_sum * alpha + (((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
-                                 ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y)));
-        if (rescale) {
-          // O holds P V of tiles < j against the old reference maximum: once
-          // PV(j - 1) has landed, scale it by alpha
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (g - 1) & 1, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld_x32(oc + c * 32, o);
-            tmem_ld_wait(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_x32(oc + c * 32, o);
-          }
+        if (!prefill_softmax_tile<D, F8, B::POLY_MASK>(sc, oc, j == 0, masked, row_last - j * B::BN,
+                                                       p.scale_log2, m_ref, l_sum, bar_o_done(k),
+                                                       (g - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
         }
         tmem_st_wait();
         tc_fence_before_sync();
@@ -522,15 +497,19 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
       const float inv_l = F8 ? p.v_scale / l_sum : 1.0f / l_sum;
       const bool valid = q_row < w.L;
       __nv_bfloat16* orow = p.out + (static_cast<size_t>(w.s0 + q_row) * p.num_q_heads + my_head) * D;
+      // all of O's columns in flight at once, one wait
+      uint32_t o[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld_x32(oc + c * 32, o[c]);
+      tmem_ld_wait(o[0]);
+#pragma unroll
+      for (int c = 1; c < D / 32; ++c) reg_dep(o[c]);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_x32(oc + c * 32, o);
-        tmem_ld_wait(o);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          pk[i] = pack_bf16x2(__uint_as_float(o[c][2 * i]) * inv_l, __uint_as_float(o[c][2 * i + 1]) * inv_l);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll

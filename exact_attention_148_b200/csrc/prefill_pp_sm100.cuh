@@ -25,16 +25,19 @@
 // exceeds it by more than 8 (a factor 256), which keeps O / l exact while
 // skipping most O rescales.
 //
-// Exponentials go to the MUFU unit (ex2.approx).  Optionally (compile-time
-// FA_PREFILL_POLY_MASK) some 32-column chunks of every 128, on tiles without
-// masking, are computed on the FMA and ALU pipes instead, as
+// Exponentials go to the MUFU unit (ex2.approx), whose 16 results per clock
+// per SM take as long for a 128 x 128 tile as its two MMAs.  Optionally
+// (compile-time FA_PREFILL_POLY_MASK) some 32-column chunks of every 128, on
+// tiles without masking, are computed on the FMA and ALU pipes instead, as
 // 2^x = 2^n * p(f), n = round(x), f = x - n in [-1/2, 1/2] (Cody & Waite
 // argument reduction), with a degree-3 minimax polynomial p fitted by the Remez
 // exchange algorithm (relative error 7.5e-5; tests/test_exp2_poly.py re-derives it), far
 // below the 2^-9 rounding P gets when it is stored as bf16.  The rounding uses
 // the float adder (adding 1.5*2^23 leaves round(x) in the low mantissa bits)
 // and 2^n is added straight into the exponent field, so no instruction of this
-// path runs on the MUFU/conversion (XU) pipe that ex2.approx uses.
+// path runs on the MUFU (XU) pipe that ex2.approx uses; pairs of elements go
+// through packed f32x2 adds and FMAs.
+
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -96,11 +99,6 @@ constexpr int kPrefillPPThreads = 320;
 #ifndef FA_PREFILL_POLY_MASK
 #define FA_PREFILL_POLY_MASK 0x0
 #endif
-// Bit c set: 32-column chunk c uses the packed half-precision MUFU ex2.
-#ifndef FA_PREFILL_F16EX2_MASK
-#define FA_PREFILL_F16EX2_MASK 0x0
-#endif
-
 // F8: Q, K and V are E4M3 bytes (one scale per tensor).  S = Q K^T runs as a
 // kind::f8f6f4 MMA on them as stored (exact products, half the tensor time of
 // bf16); P is kept as f16 and V is widened to f16 in shared memory by two
@@ -133,34 +131,22 @@ struct PrefillPPCfg {
   static constexpr int POLY_MASK = FA_PREFILL_POLY_MASK;
 };
 
-// 2^x on the FMA/ALU pipes (see the file comment).  Valid for x <= 8; inputs
-// below -125 are clamped (the result is then < 2^-124, negligible next to the
-// row maximum's term 2^0).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = __fadd_rn(x, 12582912.0f);     // 1.5 * 2^23 + round(x)
-  const float n = __fadd_rn(t, -12582912.0f);    // round(x)
-  const float f = __fadd_rn(x, -n);               // in [-1/2, 1/2]
-  float p = fmaf(0.0551716691f, f, 0.242611122f);
-  p = fmaf(p, f, 0.693260985f);
-  p = fmaf(p, f, 0.999928074f);
+// 2^x for a pair on the FMA and ALU pipes (see the file comment).  Valid for
+// x <= 8; inputs below -125 are clamped (the result is then < 2^-124,
+// negligible next to the row maximum's term 2^0).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));     // 1.5 * 2^23 + round(x)
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));   // round(x)
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);               // x - n, in [-1/2, 1/2]
+  float2 p = __ffma2_rn(make_float2(0.0551716691f, 0.0551716691f), f, make_float2(0.242611122f, 0.242611122f));
+  p = __ffma2_rn(p, f, make_float2(0.693260985f, 0.693260985f));
+  p = __ffma2_rn(p, f, make_float2(0.999928074f, 0.999928074f));
   // The low mantissa bits of t are round(x) in two's complement; shifted by 23
   // they add round(x) to p's exponent (mod 2^32, so negative n works too).
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Two exponentials with one MUFU instruction: the pair is rounded to f16
-// (11-bit significand) and put through ex2.approx.f16x2.  The argument rounding
-// costs a relative error of at most |x| * 2^-11 * ln 2 in 2^x (2.7e-3 at |x|=16,
-// where 2^x < 2^-16 already), comparable to the 2^-9 rounding P gets as bf16.
-__device__ __forceinline__ float2 ex2_pair_f16(float2 x) {
-  uint32_t h, e;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-  float lo, hi;
-  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-      : "=f"(lo), "=f"(hi) : "r"(e));
-  return make_float2(lo, hi);
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // Three-input maximum (sm_100 max.f32 with three sources).
@@ -216,6 +202,101 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
 
 constexpr int kPrefillPage = 64;
 
+// Online softmax of one 128 x 128 score tile for a slot's 128 rows (thread =
+// row = TMEM lane of its warpgroup): read S (fp32, columns sc .. sc+127),
+// write P (bf16, or f16 with E4M3 inputs) over S's first 64 columns, and
+// update the row's reference maximum m_ref (base 2, scale folded in) and
+// normaliser l_sum.  masked (the same for the whole tile): some row of the
+// tile has keys past its last visible one, lim: this row's last visible
+// column.  first: the row's first tile.  The reference maximum is raised only
+// when the tile's maximum exceeds it by more than kRescaleThreshold; then O
+// (columns oc ..) is rescaled once the previous P V has landed (o_done,
+// parity o_parity).  Returns false when a wait gave up.
+template <int D, bool F8, int POLY_MASK>
+__device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, bool first, bool masked,
+                                                     int lim, float scale_log2, float& m_ref,
+                                                     float& l_sum, uint32_t bar_o_done,
+                                                     uint32_t o_parity, volatile int* abort_flag) {
+  uint32_t s[4][32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_x32(sc + c * 32, s[c]);
+  tmem_ld_wait(s[0]);
+  reg_dep(s[1]);
+  reg_dep(s[2]);
+  reg_dep(s[3]);
+  if (masked) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c * 32 + i > lim) s[c][i] = __float_as_uint(-INFINITY);
+  }
+  // row maximum: eight independent 3-input-max chains of 16 columns, then a tree
+  float mx[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const uint32_t* v = &s[h >> 1][(h & 1) * 16];
+    float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+    for (int i = 3; i < 15; i += 2) m = fmax3(m, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+    mx[h] = fmaxf(m, __uint_as_float(v[15]));
+  }
+  const float rmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+  const float m_tile = rmax * scale_log2;
+  float alpha = 1.0f;
+  bool rescale = false;
+  if (first) {
+    m_ref = (m_tile == -INFINITY) ? 0.0f : m_tile;
+  } else {
+    const bool need = m_tile > m_ref + kRescaleThreshold;
+    rescale = __any_sync(0xffffffffu, need);
+    if (need) {
+      alpha = ex2_approx(m_ref - m_tile);
+      m_ref = m_tile;
+    }
+  }
+  // x = s * scale * log2(e) - m on the packed f32x2 FMA pipe; P chunk c (16
+  // packed columns) lands on S columns already in registers
+  const float2 scale2 = make_float2(scale_log2, scale_log2);
+  const float2 neg_m2 = make_float2(-m_ref, -m_ref);
+  float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                  make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+    const bool poly = ((POLY_MASK >> c) & 1) && !masked;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 x = __ffma2_rn(
+          make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), scale2, neg_m2);
+      const float2 e = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      ps[i & 3].x += e.x;   // (packed f32x2 adds here cost registers: spills)
+      ps[i & 3].y += e.y;
+      pk[i] = F8 ? pack_f16x2(e.x, e.y) : pack_bf16x2(e.x, e.y);
+    }
+    tmem_st_x16(sc + c * 16, pk);
+  }
+  l_sum = l_sum * alpha + (((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
+                           ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y)));
+  if (rescale) {
+    // O still holds the P V of earlier tiles against the old reference: once
+    // the previous P V has landed, scale it by alpha (1 on rows that kept
+    // their maximum).  This tile's P is in TMEM; its P V waits for p_full.
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, o_parity, abort_flag))) return false;
+    tc_fence_after_sync();
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld_x32(oc + c * 32, o);
+      tmem_ld_wait(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st_x32(oc + c * 32, o);
+    }
+  }
+  return true;
+}
+
 template <int D, bool PAGED, bool F8 = false>
 __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
     fa_prefill_pp_kernel(const __grid_constant__ PrefillParams p) {
@@ -241,7 +322,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
   int rank = bid - p.group_start[lo];
   const int s0 = p.cu_seqlens != nullptr ? p.cu_seqlens[seq] : 0;
   const int L = p.cu_seqlens != nullptr ? p.cu_seqlens[seq + 1] - s0 : p.uniform_q_len;   // queries
-  const int n_qtiles = (L + C::BM - 1) / C::BM;
+  const int n_qtiles = (L >= 1 && L <= p.total_q) ? (L + C::BM - 1) / C::BM : 0;
   int Lk = L;                                   // keys
   if constexpr (PAGED) {
     Lk = p.cache_seqlens != nullptr ? p.cache_seqlens[seq] : p.uniform_k_len;
@@ -253,9 +334,21 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
       Lk = min(max(Lk, p.causal ? L : 0), cap);
     }
   }
+  const int G = p.group;
+  {
+    // The device offsets must describe what the host planned: rows inside the
+    // T packed ones, and this group's CTA count (cu_seqlens_dev must equal
+    // cu_seqlens_host).  Otherwise record it and leave (uniform in the CTA).
+    const bool in_rows = s0 >= 0 && L >= 1 && s0 <= p.total_q - L;
+    const int nq = in_rows ? n_qtiles : 0;
+    const int derived = (((G & 1) == 0) ? nq * (G >> 1) : ((nq + 1) >> 1) * G) * max(p.kv_splits, 1);
+    if (!in_rows || derived != p.group_start[lo + 1] - p.group_start[lo]) {
+      if (rank == 0 && threadIdx.x == 0) record_status(FA_ERR_PLAN_MISMATCH);
+      return;
+    }
+  }
   const int off = p.causal ? Lk - L : 0;        // query i sits at key position i + off
   const int n_ktiles_all = (Lk + C::BN - 1) / C::BN;
-  const int G = p.group;
   // Key-range split: a group holds kv_splits copies of its q-tile CTAs, one
   // per range of kv_split_tiles key tiles (tiles [kt0, n_ktiles)).
   int kt0 = 0, n_ktiles = n_ktiles_all, split = 0;
@@ -625,97 +718,13 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
     for (int j = 0; j < nk; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(k), j & 1, abort_flag))) { ok = false; break; }
       tc_fence_after_sync();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_x32(sc + c * 32, s[c]);
-      tmem_ld_wait(s[0]);
-      reg_dep(s[1]);
-      reg_dep(s[2]);
-      reg_dep(s[3]);
-
+      // key tiles reaching past tile_last need the mask
       const bool masked = (kt0 + j) * C::BN + C::BN - 1 > tile_last;
-      if (masked) {
-        const int lim = row_last - (kt0 + j) * C::BN;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i > lim) s[c][i] = __float_as_uint(-INFINITY);
-      }
-      // row maximum: one 3-input-max chain per 32-column chunk, then a tree
-      float mx[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        mx[c] = fmax3(__uint_as_float(s[c][0]), __uint_as_float(s[c][1]), __uint_as_float(s[c][2]));
-#pragma unroll
-        for (int i = 3; i < 31; i += 2)
-          mx[c] = fmax3(mx[c], __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
-        mx[c] = fmaxf(mx[c], __uint_as_float(s[c][31]));
-      }
-      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      const float m_tile = rmax * p.scale_log2;
-      float alpha = 1.0f;
-      bool rescale = false;
-      if (j == 0) {
-        m_ref = (m_tile == -INFINITY) ? 0.0f : m_tile;
-      } else {
-        const bool need = m_tile > m_ref + kRescaleThreshold;
-        rescale = __any_sync(0xffffffffu, need);
-        if (need) {
-          alpha = ex2_approx(m_ref - m_tile);
-          m_ref = m_tile;
-        }
-      }
-      // x = s * scale * log2(e) - m on the packed f32x2 FMA pipe
-      const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
-      const float2 neg_m2 = make_float2(-m_ref, -m_ref);
-      float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                      make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-        const bool poly = ((C::POLY_MASK >> c) & 1) && !masked;
-        const bool half2 = (FA_PREFILL_F16EX2_MASK >> c) & 1;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 x = __ffma2_rn(
-              make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), scale2, neg_m2);
-          float p0, p1;
-          if (half2) {
-            const float2 e = ex2_pair_f16(x);
-            p0 = e.x;
-            p1 = e.y;
-          } else {
-            p0 = poly ? exp2_poly(x.x) : ex2_approx(x.x);
-            p1 = poly ? exp2_poly(x.y) : ex2_approx(x.y);
-          }
-          ps[i & 3].x += p0;
-          ps[i & 3].y += p1;
-          pk[i] = F8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-        }
-        // P chunk c (16 packed columns) lands on S columns already in registers.
-        tmem_st_x16(sc + c * 16, pk);
-      }
-      l_sum = l_sum * alpha + (((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
-                               ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y)));
-      if (rescale) {
-        // O still holds sum_{i<j} P_i V_i against the old reference maximum:
-        // once PV_{j-1} has landed, scale it by alpha (1 on rows that kept
-        // their maximum).  P_j is already in TMEM; PV_j waits for p_full.
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (j - 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_x32(oc + c * 32, o);
-          tmem_ld_wait(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st_x32(oc + c * 32, o);
-        }
+      if (!prefill_softmax_tile<D, F8, C::POLY_MASK>(sc, oc, j == 0, masked, row_last - (kt0 + j) * C::BN,
+                                                     p.scale_log2, m_ref, l_sum, bar_o_done(k),
+                                                     (j - 1) & 1, abort_flag)) {
+        ok = false;
+        break;
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -746,15 +755,19 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
         }
         if (valid) p.part_lse[prow] = (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
       } else {
+      // all of O's columns in flight at once, one wait
+      uint32_t o[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld_x32(oc + c * 32, o[c]);
+      tmem_ld_wait(o[0]);
+#pragma unroll
+      for (int c = 1; c < D / 32; ++c) reg_dep(o[c]);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_x32(oc + c * 32, o);
-        tmem_ld_wait(o);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          pk[i] = pack_bf16x2(__uint_as_float(o[c][2 * i]) * inv_l, __uint_as_float(o[c][2 * i + 1]) * inv_l);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll

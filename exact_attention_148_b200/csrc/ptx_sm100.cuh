@@ -136,6 +136,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Ask for a tile to be brought into L2 (no shared-memory destination, no
+// completion to wait for); out-of-range boxes are ignored like in a load.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
 // ----------------------------------------------------------------------------

@@ -17,11 +17,14 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 
 def kernel_coefficients():
-    body = open(SRC).read().split("float exp2_poly(float x)")[1].split("\n}")[0]
+    body = open(SRC).read().split("float2 exp2_poly2(float2 x)")[1].split("\n}")[0]
     nums = [float(x) for x in re.findall(r"([0-9]+\.[0-9]+)f", body)]
-    # clamp, +magic, -magic, then fmaf(c3, f, c2); fmaf(p, f, c1); fmaf(p, f, c0)
-    assert nums[:3] == [125.0, 12582912.0, 12582912.0], nums
-    c3, c2, c1, c0 = nums[3:7]
+    # clamp (x2), +magic (x2), -magic (x2), -1 (x2), then the packed
+    # fma(c3, f, c2); fma(p, f, c1); fma(p, f, c0), each constant twice
+    assert nums[:8] == [125.0, 125.0, 12582912.0, 12582912.0, 12582912.0, 12582912.0, 1.0, 1.0], nums
+    c = nums[8:16]
+    assert c[0::2] == c[1::2], c
+    c3, c2, c1, c0 = c[0::2]
     return c0, c1, c2, c3
 
 

@@ -169,3 +169,38 @@ def test_device_status_clean_after_prefill():
     inp = W.make_prefill([129], 2, 2, 64, causal=True, seed=51)
     prefill_on_gpu(inp)
     assert fa.device_status() == 0
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+def test_device_offsets_disagreeing_with_host_are_reported(schedule, monkeypatch):
+    """cu_seqlens_dev must equal cu_seqlens_host.  A device sequence that
+    leaves the T packed rows, or whose tile count differs from the host's, is
+    recorded as FA_ERR_PLAN_MISMATCH by the kernel and skipped; the other
+    sequences are computed as usual."""
+    import torch
+    import exact_attention_148_b200 as fa
+    monkeypatch.setenv("FA_PREFILL_SCHEDULE", schedule)
+    inp = W.make_prefill([200, 400, 300], 4, 2, 128, causal=True, seed=61)
+    q, k, v = (to_dev_bf16(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    want, want_lse = prefill_on_gpu(inp)
+    fa.device_status(clear=True)
+    # sequence 1 runs past T on the device (the host says it ends at 600)
+    bad = inp.cu_seqlens.copy()
+    bad[2] = bad[3] + 100
+    out = torch.zeros_like(want)
+    lse = torch.zeros_like(want_lse)
+    fa.prefill(q, k, v, to_dev_i32(bad), causal=True, scale=inp.scale, out=out, lse=lse,
+               cu_seqlens_host=inp.cu_seqlens)
+    assert fa.device_status(clear=True) == fa.FA_ERR_PLAN_MISMATCH
+    s0, s1 = int(inp.cu_seqlens[0]), int(inp.cu_seqlens[1])
+    assert torch.equal(out[s0:s1], want[s0:s1]) and torch.equal(lse[s0:s1], want_lse[s0:s1])
+    # sequence 0 one tile longer on the device than on the host
+    bad = inp.cu_seqlens.copy()
+    bad[1] = 260
+    fa.prefill(q, k, v, to_dev_i32(bad), causal=True, scale=inp.scale, out=out, lse=lse,
+               cu_seqlens_host=inp.cu_seqlens)
+    assert fa.device_status(clear=True) == fa.FA_ERR_PLAN_MISMATCH
+    # the consistent call afterwards is clean and unchanged
+    again, again_lse = prefill_on_gpu(inp)
+    assert fa.device_status(clear=True) == 0
+    assert torch.equal(again, want) and torch.equal(again_lse, want_lse)
