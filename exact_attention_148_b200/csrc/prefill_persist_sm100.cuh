@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         tc_fence_after_sync();
         // key tiles reaching past tile_last need the mask
         const bool masked = j * B::BN + B::BN - 1 > tile_last;
-        if (!prefill_softmax_tile<D, F8, B::POLY_MASK>(sc, oc, j == 0, masked, row_last - j * B::BN,
+        if (!prefill_softmax_tile<D, F8>(sc, oc, j == 0, masked, row_last - j * B::BN,
                                                        p.scale_log2, m_ref, l_sum, bar_o_done(k),
                                                        (g - 1) & 1, abort_flag)) {
           ok = false;

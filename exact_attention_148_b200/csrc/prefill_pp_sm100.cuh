@@ -26,17 +26,9 @@
 // skipping most O rescales.
 //
 // Exponentials go to the MUFU unit (ex2.approx), whose 16 results per clock
-// per SM take as long for a 128 x 128 tile as its two MMAs.  Optionally
-// (compile-time FA_PREFILL_POLY_MASK) some 32-column chunks of every 128, on
-// tiles without masking, are computed on the FMA and ALU pipes instead, as
-// 2^x = 2^n * p(f), n = round(x), f = x - n in [-1/2, 1/2] (Cody & Waite
-// argument reduction), with a degree-3 minimax polynomial p fitted by the Remez
-// exchange algorithm (relative error 7.5e-5; tests/test_exp2_poly.py re-derives it), far
-// below the 2^-9 rounding P gets when it is stored as bf16.  The rounding uses
-// the float adder (adding 1.5*2^23 leaves round(x) in the low mantissa bits)
-// and 2^n is added straight into the exponent field, so no instruction of this
-// path runs on the MUFU (XU) pipe that ex2.approx uses; pairs of elements go
-// through packed f32x2 adds and FMAs.
+// per SM take as long for a 128 x 128 tile as its two MMAs.  (Moving a share
+// of them to a polynomial on the FMA pipes, or deferring the row maximum,
+// measured slower on B200 in every form tried.)
 
 #pragma once
 
@@ -93,12 +85,6 @@ struct PrefillParams {
 
 constexpr int kPrefillPPThreads = 320;
 
-// Measured on B200 at d=128: any polynomial share slows the kernel (the
-// extra FMA/ALU instructions cost more issue slots than the MUFU time they
-// save), so by default every exponential uses ex2.approx.
-#ifndef FA_PREFILL_POLY_MASK
-#define FA_PREFILL_POLY_MASK 0x0
-#endif
 // F8: Q, K and V are E4M3 bytes (one scale per tensor).  S = Q K^T runs as a
 // kind::f8f6f4 MMA on them as stored (exact products, half the tensor time of
 // bf16); P is kept as f16 and V is widened to f16 in shared memory by two
@@ -127,27 +113,7 @@ struct PrefillPPCfg {
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  // Bit c set: the exponentials of 32-column chunk c use the FMA-pipe polynomial.
-  static constexpr int POLY_MASK = FA_PREFILL_POLY_MASK;
 };
-
-// 2^x for a pair on the FMA and ALU pipes (see the file comment).  Valid for
-// x <= 8; inputs below -125 are clamped (the result is then < 2^-124,
-// negligible next to the row maximum's term 2^0).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));     // 1.5 * 2^23 + round(x)
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));   // round(x)
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);               // x - n, in [-1/2, 1/2]
-  float2 p = __ffma2_rn(make_float2(0.0551716691f, 0.0551716691f), f, make_float2(0.242611122f, 0.242611122f));
-  p = __ffma2_rn(p, f, make_float2(0.693260985f, 0.693260985f));
-  p = __ffma2_rn(p, f, make_float2(0.999928074f, 0.999928074f));
-  // The low mantissa bits of t are round(x) in two's complement; shifted by 23
-  // they add round(x) to p's exponent (mod 2^32, so negative n works too).
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
 
 // Three-input maximum (sm_100 max.f32 with three sources).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -212,7 +178,7 @@ constexpr int kPrefillPage = 64;
 // when the tile's maximum exceeds it by more than kRescaleThreshold; then O
 // (columns oc ..) is rescaled once the previous P V has landed (o_done,
 // parity o_parity).  Returns false when a wait gave up.
-template <int D, bool F8, int POLY_MASK>
+template <int D, bool F8>
 __device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, bool first, bool masked,
                                                      int lim, float scale_log2, float& m_ref,
                                                      float& l_sum, uint32_t bar_o_done,
@@ -264,12 +230,11 @@ __device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, b
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint32_t pk[16];
-    const bool poly = ((POLY_MASK >> c) & 1) && !masked;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 x = __ffma2_rn(
           make_float2(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), scale2, neg_m2);
-      const float2 e = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       ps[i & 3].x += e.x;   // (packed f32x2 adds here cost registers: spills)
       ps[i & 3].y += e.y;
       pk[i] = F8 ? pack_f16x2(e.x, e.y) : pack_bf16x2(e.x, e.y);
@@ -720,7 +685,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
       tc_fence_after_sync();
       // key tiles reaching past tile_last need the mask
       const bool masked = (kt0 + j) * C::BN + C::BN - 1 > tile_last;
-      if (!prefill_softmax_tile<D, F8, C::POLY_MASK>(sc, oc, j == 0, masked, row_last - (kt0 + j) * C::BN,
+      if (!prefill_softmax_tile<D, F8>(sc, oc, j == 0, masked, row_last - (kt0 + j) * C::BN,
                                                      p.scale_log2, m_ref, l_sum, bar_o_done(k),
                                                      (j - 1) & 1, abort_flag)) {
         ok = false;
