@@ -7,6 +7,11 @@ library's CUDA kernels.  PyTorch provides device memory and streams.
 
 There is no CPU fallback: if the shared library is missing, or a tensor is not
 a CUDA tensor, the call raises.
+
+``FA_LIBRARY=debug`` in the environment (or ``select_library("debug")``) loads
+the bounds-checked build ``libexact_attention_debug.so`` instead: the same
+kernels with every computed global index checked against its buffer, a
+failure recorded as FA_ERR_DEBUG_INDEX in the device status word.
 """
 from __future__ import annotations
 
@@ -21,11 +26,13 @@ __all__ = [
     "FAError", "library", "lib_path", "prefill", "decode_plan", "DecodePlan", "decode_paged",
     "decode_paged_static", "merge_states", "device_status", "strerror", "EXPORTED_SYMBOLS",
     "append_kv", "prefill_paged", "prefill_fp8", "decode_paged_fp8", "cascade_decode", "cascade_workspace_bytes",
-    "prefill_last_schedule",
+    "prefill_last_schedule", "select_library", "debug_selftest_index",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_PKG_DIR, "libexact_attention.so")
+release_lib_path = os.path.join(_PKG_DIR, "libexact_attention.so")
+debug_lib_path = os.path.join(_PKG_DIR, "libexact_attention_debug.so")
+lib_path = debug_lib_path if os.environ.get("FA_LIBRARY") == "debug" else release_lib_path
 
 FA_OK = 0
 FA_ERR_INVALID_ARG = -1
@@ -35,13 +42,14 @@ FA_ERR_CUDA = -4
 FA_ERR_TIMEOUT = -5
 FA_ERR_PLAN_MISMATCH = -6
 FA_ERR_BAD_PAGE = -7
+FA_ERR_DEBUG_INDEX = -8
 
 EXPORTED_SYMBOLS = [
     "fa_prefill", "fa_decode_plan", "fa_plan_get_info", "fa_plan_free", "fa_decode_paged",
     "fa_merge_states", "fa_strerror", "fa_last_cuda_error", "fa_get_device_status", "fa_version",
     "fa_decode_paged_static", "fa_selftest_wait_timeout", "fa_append_kv", "fa_prefill_paged",
     "fa_decode_paged_fp8", "fa_decode_plan_kv", "fa_decode_plan_ex", "fa_cascade_workspace_bytes",
-    "fa_cascade_decode", "fa_prefill_fp8", "fa_prefill_last_schedule",
+    "fa_cascade_decode", "fa_prefill_fp8", "fa_prefill_last_schedule", "fa_debug_selftest_index",
 ]
 
 FA_KV_BF16, FA_KV_E4M3 = 0, 1
@@ -144,8 +152,30 @@ def library() -> ctypes.CDLL:
     L.fa_decode_paged_fp8.restype = i32
     L.fa_prefill_last_schedule.argtypes = []
     L.fa_prefill_last_schedule.restype = i32
+    L.fa_debug_selftest_index.argtypes = [vp, i32, vp]
+    L.fa_debug_selftest_index.restype = i32
     _lib = L
     return L
+
+
+def select_library(variant: str) -> None:
+    """"release" or "debug" (bounds-checked): the build later calls load.
+    Plans made with one build must not be passed to the other."""
+    global lib_path, _lib
+    lib_path = {"release": release_lib_path, "debug": debug_lib_path}[variant]
+    _lib = None
+
+
+def debug_selftest_index(buf, stream=None) -> int:
+    """Bounds-checked build only: a kernel writes buf[0] and then tries an
+    index past half of buf, which its check must refuse (the refused index is
+    still inside buf).  Returns the call's status (FA_ERR_UNSUPPORTED on the
+    release build, which launches nothing)."""
+    torch = _torch()
+    _require_cuda(buf)
+    if buf.dtype != torch.int32 or buf.numel() < 4:
+        raise ValueError("buf must be an int32 CUDA tensor of at least 4 elements")
+    return library().fa_debug_selftest_index(_ptr(buf), int(buf.numel()), _stream_ptr(stream))
 
 
 def strerror(status: int) -> str:

@@ -30,6 +30,7 @@ struct AppendParams {
   __nv_bfloat16* k_pages;
   __nv_bfloat16* v_pages;
   int64_t page_stride, token_stride, head_stride;   // elements
+  int64_t pool_elems;           // elements from the pool's base to one past its last one
   int total_new;
   int batch;
   int num_kv_heads;
@@ -59,6 +60,7 @@ __global__ void __launch_bounds__(kAppendThreads) fa_append_kv_kernel(const Appe
       continue;
     }
     const int pos = len - n + (t - first);
+    if (!FA_DBG_OK(pos >= 0 && pos / kAppendPage < p.max_pages)) continue;
     const int phys = p.block_table[static_cast<size_t>(b) * p.max_pages + pos / kAppendPage];
     if (phys < 0 || phys >= p.num_pages) {
       if (lane == 0) record_status(FA_ERR_BAD_PAGE);
@@ -85,6 +87,7 @@ __global__ void __launch_bounds__(kAppendThreads) fa_append_kv_kernel(const Appe
         const int e = e0 + 32 * u;
         if (e < pieces) {
           const int64_t dst = dst_row + (e / VEC) * p.head_stride + (e % VEC) * 8;   // elements
+          if (!FA_DBG_OK(dst >= 0 && dst + 8 <= p.pool_elems)) continue;
           *reinterpret_cast<uint4*>(p.k_pages + dst) = kv[u];
           *reinterpret_cast<uint4*>(p.v_pages + dst) = vv[u];
         }

@@ -241,7 +241,8 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
     int issued = 0;
     bool ok = true;
     for (int i0 = 0; ok && i0 < num_pg; i0 += 32) {
-      const int mine = (i0 + lane < num_pg) ? bt_row[i0 + lane] : 0;
+      const int mine = (i0 + lane < num_pg && FA_DBG_OK(page_begin + i0 + lane < p.max_pages))
+                           ? bt_row[i0 + lane] : 0;
       const int cnt = min(32, num_pg - i0);
       for (int ii = 0; ii < cnt; ++ii) {
         int phys = __shfl_sync(0xffffffffu, mine, ii);
@@ -286,8 +287,9 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
     float2 qr[GC][COLS / 2];
 #pragma unroll
     for (int gi = 0; gi < GC; ++gi) {
+      const size_t qrow = static_cast<size_t>(b) * p.num_q_heads + qh0 + gi;
       const uint8_t* src = reinterpret_cast<const uint8_t*>(
-          p.q + (static_cast<size_t>(b) * p.num_q_heads + qh0 + gi) * D + c0);
+          p.q + (FA_DBG_OK(qrow < static_cast<size_t>(p.batch) * p.num_q_heads) ? qrow : 0) * D + c0);
       load_bf16_row<COLS>(src, qr[gi]);
 #pragma unroll
       for (int c = 0; c < COLS / 2; ++c) {
@@ -453,13 +455,18 @@ __global__ void __launch_bounds__(kDecodeThreads, GC == 8 ? 1 : 2)
       const float lse_v = (M == -INFINITY) ? -INFINITY
                                            : (M + log2f(lsum) - (KV8 ? 60.0f : 0.0f)) * 0.69314718055994530942f;
       const size_t row = static_cast<size_t>(b) * p.num_q_heads + qh0 + gi;
+      const size_t rows = static_cast<size_t>(p.batch) * p.num_q_heads;
       if (direct) {
-        p.out[row * D + c] = __float2bfloat16_rn(o);
-        if (c == 0 && p.lse != nullptr) p.lse[row] = lse_v;
+        if (FA_DBG_OK(row < rows)) {
+          p.out[row * D + c] = __float2bfloat16_rn(o);
+          if (c == 0 && p.lse != nullptr) p.lse[row] = lse_v;
+        }
       } else {
-        const size_t srow = static_cast<size_t>(split) * p.batch * p.num_q_heads + row;
-        p.ws_o[srow * D + c] = o;
-        if (c == 0) p.ws_lse[srow] = lse_v;
+        const size_t srow = static_cast<size_t>(split) * rows + row;
+        if (FA_DBG_OK(srow < static_cast<size_t>(p.max_splits) * rows)) {
+          p.ws_o[srow * D + c] = o;
+          if (c == 0) p.ws_lse[srow] = lse_v;
+        }
       }
     }
   }
@@ -494,12 +501,14 @@ __global__ void __launch_bounds__(128) fa_merge_kernel(const MergeParams p) {
   const int r = rh / p.num_heads;
   int ns = p.num_states;
   if (p.cache_seqlens != nullptr) {
+    if (!FA_DBG_OK(r / p.q_len < (p.rows + p.q_len - 1) / p.q_len)) return;
     int seqlen = p.cache_seqlens[r / p.q_len];
     seqlen = max(0, min(seqlen, p.max_pages * kDecodePage));
     ns = min(p.num_states, (seqlen + p.chunk_tokens - 1) / p.chunk_tokens);
     if (ns <= 1) return;
   }
   const size_t stride = static_cast<size_t>(p.rows) * p.num_heads;
+  if (!FA_DBG_OK(ns <= p.num_states)) return;
   float M = -INFINITY;
   for (int i = lane; i < ns; i += 32) M = fmaxf(M, p.lse_parts[i * stride + rh]);
 #pragma unroll
@@ -566,6 +575,7 @@ __global__ void __launch_bounds__(128) fa_cascade_merge_kernel(const CascadeMerg
   const int rh = blockIdx.x * 4 + warp;
   if (rh >= p.rows * p.num_heads) return;
   const size_t stride = static_cast<size_t>(p.rows) * p.num_heads;
+  if (!FA_DBG_OK(p.num_prefix >= 0)) return;
   const float ls = p.suffix_lse[rh];
   float M = ls;
   for (int i = lane; i < p.num_prefix; i += 32) M = fmaxf(M, p.prefix_lse[i * stride + rh]);

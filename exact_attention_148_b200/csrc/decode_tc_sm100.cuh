@@ -245,6 +245,7 @@ __global__ void __launch_bounds__(kDecodeTcThreads, NPAD == 8 ? 2 : 1)
     for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
       const int rr = e / D;
       const size_t row = (static_cast<size_t>(b) * QL + rr / G) * p.num_q_heads + qh0 + rr % G;
+      if (!FA_DBG_OK(row < static_cast<size_t>(p.batch) * QL * p.num_q_heads)) continue;
       p.out[row * D + e % D] = __float2bfloat16_rn(0.0f);
       if (e % D == 0 && p.lse != nullptr) p.lse[row] = -INFINITY;
     }
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kDecodeTcThreads, NPAD == 8 ? 2 : 1)
         pg_base = lp0 & ~31;
         const int lp = pg_base + lane;
         int id = p.num_pages;                       // past the split: zero fill
-        if (lp < num_pg) {
+        if (lp < num_pg && FA_DBG_OK(page_begin + lp < p.max_pages)) {
           id = bt_row[lp];
           if (id < 0 || id >= p.num_pages) {
             record_status(FA_ERR_BAD_PAGE);
@@ -467,9 +468,9 @@ __global__ void __launch_bounds__(kDecodeTcThreads, NPAD == 8 ? 2 : 1)
       for (int h = quad; h < NPAD; h += 4) {      // h = operand row t * G + head
         uint32_t hi = 0, lo = 0;
         float sq = 1.0f;
-        if (h < R) {
-          const uint2 u = *reinterpret_cast<const uint2*>(
-              p.q + ((static_cast<size_t>(b) * QL + h / G) * p.num_q_heads + qh0 + h % G) * D + 4 * lane);
+        const size_t qrow = (static_cast<size_t>(b) * QL + h / G) * p.num_q_heads + qh0 + h % G;
+        if (h < R && FA_DBG_OK(qrow < static_cast<size_t>(p.batch) * QL * p.num_q_heads)) {
+          const uint2 u = *reinterpret_cast<const uint2*>(p.q + qrow * D + 4 * lane);
           const float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
                               __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
           float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
@@ -623,13 +624,18 @@ __global__ void __launch_bounds__(kDecodeTcThreads, NPAD == 8 ? 2 : 1)
         ov = lsum > 0.0f ? ov / lsum : 0.0f;
         const float lse_v = (lsum > 0.0f) ? (m[h] + log2f(lsum)) * 0.69314718055994530942f : -INFINITY;
         const size_t row = (static_cast<size_t>(b) * QL + h / G) * p.num_q_heads + qh0 + h % G;
+        const size_t rows = static_cast<size_t>(p.batch) * QL * p.num_q_heads;
         if (direct) {
-          p.out[row * D + r] = __float2bfloat16_rn(ov);
-          if (r == 0 && p.lse != nullptr) p.lse[row] = lse_v;
+          if (FA_DBG_OK(row < rows)) {
+            p.out[row * D + r] = __float2bfloat16_rn(ov);
+            if (r == 0 && p.lse != nullptr) p.lse[row] = lse_v;
+          }
         } else {
-          const size_t srow = static_cast<size_t>(split) * p.batch * QL * p.num_q_heads + row;
-          p.ws_o[srow * D + r] = ov;
-          if (r == 0) p.ws_lse[srow] = lse_v;
+          const size_t srow = static_cast<size_t>(split) * rows + row;
+          if (FA_DBG_OK(srow < static_cast<size_t>(p.max_splits) * rows)) {
+            p.ws_o[srow * D + r] = ov;
+            if (r == 0) p.ws_lse[srow] = lse_v;
+          }
         }
       }
     }

@@ -200,20 +200,17 @@ uint32_t* prefill_sched_slot(cudaStream_t stream) {
     cudaGetLastError();
     return nullptr;
   }
+  // The counters' address is looked up on every call (cheap once the module
+  // is loaded), so it stays right after a cudaDeviceReset reloads the module.
+  void* base = nullptr;
+  if (cudaGetSymbolAddress(&base, g_prefill_sched) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
   static std::mutex mu;
   static std::map<std::pair<int, unsigned long long>, int> slot_of;
   static std::map<int, int> taken;
-  static std::map<int, uint32_t*> base_of;
   std::lock_guard<std::mutex> lock(mu);
-  auto b = base_of.find(dev);
-  if (b == base_of.end()) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_prefill_sched) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    b = base_of.emplace(dev, static_cast<uint32_t*>(ptr)).first;
-  }
   const auto key = std::make_pair(dev, id);
   auto it = slot_of.find(key);
   if (it == slot_of.end()) {
@@ -221,7 +218,7 @@ uint32_t* prefill_sched_slot(cudaStream_t stream) {
     if (t >= fa::kSchedSlots) return nullptr;
     it = slot_of.emplace(key, t++).first;
   }
-  return b->second + 2 * it->second;
+  return static_cast<uint32_t*>(base) + 2 * it->second;
 }
 
 // Launch order of the prefill CTAs: sequences heaviest first (most query-key
@@ -404,6 +401,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* cu_
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_dev;
   prm.total_q = static_cast<int>(T);
+  prm.batch = batch;
   prm.num_q_heads = num_q_heads;
   prm.group = group;
   prm.causal = causal ? 1 : 0;
@@ -513,6 +511,7 @@ FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_q_dev;
   prm.total_q = static_cast<int>(T);
+  prm.batch = batch;
   prm.block_table = block_table;
   prm.cache_seqlens = cache_seqlens_dev;
   prm.max_pages = max_pages_per_seq;
@@ -558,6 +557,8 @@ FA_API int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_
   ap.page_stride = page_stride;
   ap.token_stride = token_stride;
   ap.head_stride = head_stride;
+  ap.pool_elems = (num_pages - 1) * page_stride + (page_size - 1) * token_stride +
+                  (num_kv_heads - 1) * head_stride + head_dim;
   ap.total_new = total_new;
   ap.batch = batch;
   ap.num_kv_heads = num_kv_heads;
@@ -815,6 +816,7 @@ FA_API const char* fa_strerror(int status) {
     case FA_ERR_TIMEOUT: return "device wait timed out";
     case FA_ERR_PLAN_MISMATCH: return "plan does not cover the call";
     case FA_ERR_BAD_PAGE: return "block_table entry outside the page pool";
+    case FA_ERR_DEBUG_INDEX: return "index outside its buffer (bounds-checked build)";
   }
   return "unknown status";
 }
@@ -844,6 +846,29 @@ FA_API int fa_selftest_wait_timeout(int64_t limit_us, void* stream) {
 }
 
 FA_API int fa_version(void) { return 100; }
+
+#ifdef FA_DEBUG
+namespace fa {
+// buf[0] = 1, then a store at n/2 + 1 checked against a logical extent of n/2.
+__global__ void fa_debug_selftest_index_kernel(int32_t* buf, int n) {
+  const int half = n / 2;
+  if (FA_DBG_OK(0 < half)) buf[0] = 1;
+  if (FA_DBG_OK(half + 1 < half)) buf[half + 1] = 1;
+}
+}  // namespace fa
+#endif
+
+FA_API int fa_debug_selftest_index(int32_t* buf, int n, void* stream) {
+  if (buf == nullptr || n < 4 || !aligned(buf, 4)) return FA_ERR_INVALID_ARG;
+#ifdef FA_DEBUG
+  fa::fa_debug_selftest_index_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(buf, n);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+#else
+  (void)stream;
+  return FA_ERR_UNSUPPORTED;
+#endif
+}
 
 // ============================================================================
 // Scratch-free decode (fa_decode_paged_static): the split partials go to a
@@ -990,6 +1015,7 @@ FA_API int fa_cascade_decode(const void* q, const void* k_pages, const void* v_p
                             &prm.head_coord, &prm.page_coord);
   if (st != FA_OK) return st;
   prm.cu_seqlens = nullptr;
+  prm.batch = 1;                     // one sequence: the batch's queries over the prefix
   prm.uniform_q_len = pl.batch;
   prm.cache_seqlens = nullptr;
   prm.uniform_k_len = prefix_len;

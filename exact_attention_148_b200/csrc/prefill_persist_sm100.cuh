@@ -90,8 +90,9 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   const int seq = static_cast<int>(p.group_id[lo] >> 16);
   w.kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
   const int rank = idx - p.group_start[lo];
-  w.s0 = p.cu_seqlens[seq];
-  w.L = p.cu_seqlens[seq + 1] - w.s0;
+  const bool seq_ok = FA_DBG_OK(seq < p.batch);
+  w.s0 = seq_ok ? p.cu_seqlens[seq] : -1;
+  w.L = seq_ok ? p.cu_seqlens[seq + 1] - w.s0 : 0;
   const bool in_rows = w.s0 >= 0 && w.L >= 1 && w.s0 <= p.total_q - w.L;
   const int n_qtiles = in_rows ? (w.L + BM - 1) / BM : 0;
   const int n_ktiles = in_rows ? (w.L + BN - 1) / BN : 0;
@@ -495,7 +496,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (tiles + nk - 1) & 1, abort_flag))) break;
       tc_fence_after_sync();
       const float inv_l = F8 ? p.v_scale / l_sum : 1.0f / l_sum;
-      const bool valid = q_row < w.L;
+      const bool valid = q_row < w.L && FA_DBG_OK(w.s0 + q_row < p.total_q && my_head < p.num_q_heads);
       __nv_bfloat16* orow = p.out + (static_cast<size_t>(w.s0 + q_row) * p.num_q_heads + my_head) * D;
       // all of O's columns in flight at once, one wait
       uint32_t o[D / 32][32];

@@ -75,6 +75,7 @@ struct PrefillParams {
   int head_coord;            // paged: tensor-map dimension (1..3) of the kv head
   int page_coord;            // paged: tensor-map dimension (1..3) of the page id
   int num_q_heads;
+  int batch;                 // sequences (rows of cu_seqlens - 1, of block_table)
   int group;                 // Hq / Hkv
   int causal;
   float scale_log2;          // scale * log2(e)
@@ -284,6 +285,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
   }
   const int seq = static_cast<int>(p.group_id[lo] >> 16);
   const int kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
+  if (!FA_DBG_OK(seq < p.batch)) return;   // uniform in the CTA; nothing allocated yet
   int rank = bid - p.group_start[lo];
   const int s0 = p.cu_seqlens != nullptr ? p.cu_seqlens[seq] : 0;
   const int L = p.cu_seqlens != nullptr ? p.cu_seqlens[seq + 1] - s0 : p.uniform_q_len;   // queries
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
         pg_base = lp0 & ~31;
         const int lp = pg_base + lane;
         int id = p.num_pages;
-        if (lp * kPrefillPage < Lk) {
+        if (lp * kPrefillPage < Lk && FA_DBG_OK(lp < p.max_pages)) {
           id = bt_row[lp];
           if (id < 0 || id >= p.num_pages) {
             record_status(FA_ERR_BAD_PAGE);
@@ -699,18 +701,19 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
     if (nk > 0 && ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done(k), (nk - 1) & 1, abort_flag))) {
       tc_fence_after_sync();
       const float inv_l = F8 ? p.v_scale / l_sum : 1.0f / l_sum;
-      const bool valid = q_row < L;
+      const bool valid = q_row < L && FA_DBG_OK(s0 + q_row < p.total_q && my_head < p.num_q_heads);
       __nv_bfloat16* orow =
           p.out + (static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head) * D;
       if (p.part_o != nullptr) {
         // key-range split: normalised fp32 O and LSE of this range
         const size_t prow = (static_cast<size_t>(split) * p.total_q + s0 + q_row) * p.num_q_heads + my_head;
+        const bool pvalid = valid && FA_DBG_OK(split < max(p.kv_splits, 1));
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld_x32(oc + c * 32, o);
           tmem_ld_wait(o);
-          if (valid) {
+          if (pvalid) {
             float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + c * 32);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
@@ -718,7 +721,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
                                    __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
           }
         }
-        if (valid) p.part_lse[prow] = (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
+        if (pvalid) p.part_lse[prow] = (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
       } else {
       // all of O's columns in flight at once, one wait
       uint32_t o[D / 32][32];

@@ -20,6 +20,21 @@ __device__ int g_device_status;
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
 
+// Bounds-checked builds (FA_DEBUG): every global index a kernel computes is
+// checked against its buffer's extent before the access; a failed check
+// records FA_ERR_DEBUG_INDEX and the access is skipped, so a bad index shows
+// up in the status word instead of touching memory.  Release builds compile
+// the checks away.
+#ifdef FA_DEBUG
+__device__ __forceinline__ bool debug_index_ok(bool ok) {
+  if (!ok) record_status(FA_ERR_DEBUG_INDEX);
+  return ok;
+}
+#define FA_DBG_OK(cond) ::fa::debug_index_ok(cond)
+#else
+#define FA_DBG_OK(cond) true
+#endif
+
 // Upper bound on any single wait; far above any legitimate wait in these
 // kernels (microseconds), low enough to hand the GPU back quickly.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;

@@ -29,6 +29,10 @@
  *     cache length beyond what its plan covers) or a wait that exceeds its
  *     bound records a code in a per-device status word; read it with
  *     fa_get_device_status().  Kernels never trap.
+ *   - The same library built with FA_DEBUG (libexact_attention_debug.so) also
+ *     checks every global index a kernel computes against its buffer before
+ *     the access; a failed check records FA_ERR_DEBUG_INDEX and skips the
+ *     access.  Its results are bit-identical to the release build's.
  */
 #ifndef EXACT_ATTENTION_H_
 #define EXACT_ATTENTION_H_
@@ -49,7 +53,9 @@ typedef enum {
   FA_ERR_TIMEOUT = -5,       /* (device status) a bounded wait gave up */
   FA_ERR_PLAN_MISMATCH = -6, /* plan does not match the call's shapes, or a
                                 device cache length exceeds what it covers */
-  FA_ERR_BAD_PAGE = -7       /* (device status) block_table entry outside the pool */
+  FA_ERR_BAD_PAGE = -7,      /* (device status) block_table entry outside the pool */
+  FA_ERR_DEBUG_INDEX = -8    /* (device status, FA_DEBUG builds only) a computed index failed
+                                its bounds check; the access was skipped */
 } fa_status;
 
 /* Opaque host-side decode plan, created by fa_decode_plan, freed by fa_plan_free. */
@@ -434,6 +440,19 @@ int fa_selftest_wait_timeout(int64_t limit_us, void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int fa_version(void);
+
+/*
+ * fa_debug_selftest_index — check of the bounds-checked build's index checks
+ * (libexact_attention_debug.so, compiled with FA_DEBUG).  No page counterpart:
+ * it tests this library's failure detection.  On `stream`, one kernel sets
+ * buf[0] = 1 and then tries buf[n/2 + 1], an index it checks against n/2 and
+ * must refuse: the check records FA_ERR_DEBUG_INDEX in the device status
+ * word and skips the store (the index lies inside buf, so even a check that
+ * failed to refuse would write nothing outside it).
+ *   buf: device int32 [n], n >= 4.
+ * The release build launches nothing and returns FA_ERR_UNSUPPORTED.
+ */
+int fa_debug_selftest_index(int32_t* buf, int n, void* stream);
 
 #ifdef __cplusplus
 }

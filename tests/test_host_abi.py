@@ -51,6 +51,22 @@ def test_only_api_symbols_are_exported(lib):
     assert fa_names == set(header_functions())
 
 
+def test_bounds_checked_build_exports_the_same_symbols():
+    import subprocess
+    path = _build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    names = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {n for n in names if n.startswith("fa_")} == set(header_functions())
+
+
+def test_release_build_refuses_the_index_selftest(lib):
+    # no CUDA call is made: the release build returns before any launch
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.fa_debug_selftest_index(fake, 16, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_debug_selftest_index(fake, 2, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.strerror(fa.FA_ERR_DEBUG_INDEX).startswith("index outside")
+
+
 def test_version_and_strerror(lib):
     assert fa.version() == 100
     assert fa.strerror(0) == "ok"
