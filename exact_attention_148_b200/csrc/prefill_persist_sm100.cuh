@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
   const uint32_t bar_q1 = bars + 8 * (9 + 2 * NS);
   auto bar_vh_full = [&](int sl) { return bars + 8 * (10 + 2 * NS + sl); };
   auto bar_vh_empty = [&](int sl) { return bars + 8 * (12 + 2 * NS + sl); };
+  auto bar_p_half = [&](int k) { return bars + 8 * (B::P_HALF_BAR + k); };
   auto bar_q_empty = [&](int k) { return bars + 8 * (B::NUM_BARS + k); };
   auto bar_item_full = [&](int i) { return bars + 8 * (B::NUM_BARS + 2 + i); };
   auto bar_item_empty = [&](int i) { return bars + 8 * (B::NUM_BARS + 2 + QD + i); };
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s_full(k), 1);
       mbar_init(bar_p_full(k), 4);
+      mbar_init(bar_p_half(k), 4);
       mbar_init(bar_o_done(k), 1);
       mbar_init(bar_q_empty(k), 1);
       if constexpr (F8) {
@@ -324,13 +326,14 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         }
       };
       // V operand: ring entry R (bf16) or f16 tile vslot (E4M3)
-      auto issue_pv = [&](int k, uint32_t R, int vslot, bool accumulate) {
+      // keys 64h .. 64h+63 (the P columns of half h)
+      auto issue_pv_half = [&](int k, uint32_t R, int vslot, bool accumulate, int h) {
         const uint32_t o_tmem = tmem + 256u + (k ? D : 0);
         const uint32_t p_tmem = tmem + (k ? 128u : 0u);
         const uint64_t vd = F8 ? v_desc0 + static_cast<uint64_t>((vslot * B::VH_TILE) >> 4)
                                : v_desc0 + ring_off(R);
 #pragma unroll
-        for (int kk = 0; kk < B::BN / 16; ++kk)
+        for (int kk = h * B::BN / 32; kk < (h + 1) * B::BN / 32; ++kk)
           mma_bf16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                       (accumulate || kk > 0) ? 1u : 0u);
       };
@@ -370,9 +373,13 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         // One slot's step at key tile j: O_k += P_k V_j, then S_k(j+1).
         auto slot_step = [&](int k, int nk, int tb, int j, uint32_t v_R, int vslot, uint32_t k_R) -> bool {
           if (j >= nk) return true;
+          // the first half of P V starts while the softmax finishes the second half
+          if (!mbar_wait(bar_p_half(k), (tb + j) & 1, abort_flag)) return false;
+          tc_fence_after_sync();
+          issue_pv_half(k, v_R, vslot, j > 0, 0);
           if (!mbar_wait(bar_p_full(k), (tb + j) & 1, abort_flag)) return false;
           tc_fence_after_sync();
-          issue_pv(k, v_R, vslot, j > 0);
+          issue_pv_half(k, v_R, vslot, true, 1);
           tc_commit(bar_o_done(k));
           if (j + 1 < nk) {
             issue_qk(k, k_R);
@@ -483,7 +490,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         const bool masked = j * B::BN + B::BN - 1 > tile_last;
         if (!prefill_softmax_tile<D, F8>(sc, oc, j == 0, masked, row_last - j * B::BN,
                                                        p.scale_log2, m_ref, l_sum, bar_o_done(k),
-                                                       (g - 1) & 1, abort_flag)) {
+                                                       (g - 1) & 1, bar_p_half(k), abort_flag)) {
           ok = false;
           break;
         }

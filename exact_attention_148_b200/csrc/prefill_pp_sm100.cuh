@@ -108,8 +108,9 @@ struct PrefillPPCfg {
   static constexpr int VH_TILE = 2 * CHUNK_BYTES;
   static constexpr int BAR_OFF = VH_OFF + (F8 ? 2 * VH_TILE : 0);
   // q_full (slot 0), kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], final, v_tail,
-  // q_full (slot 1), F8: vh_full[2], vh_empty[2]
-  static constexpr int NUM_BARS = 1 + 2 * NS + 9 + (F8 ? 4 : 0);
+  // q_full (slot 1), F8: vh_full[2], vh_empty[2]; then p_half[2]
+  static constexpr int P_HALF_BAR = 10 + 2 * NS + (F8 ? 4 : 0);
+  static constexpr int NUM_BARS = P_HALF_BAR + 2;
   static constexpr int THREADS = F8 ? 384 : 320;           // F8: + two converter warps
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
@@ -183,7 +184,8 @@ template <int D, bool F8>
 __device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, bool first, bool masked,
                                                      int lim, float scale_log2, float& m_ref,
                                                      float& l_sum, uint32_t bar_o_done,
-                                                     uint32_t o_parity, volatile int* abort_flag) {
+                                                     uint32_t o_parity, uint32_t bar_p_half,
+                                                     volatile int* abort_flag) {
   uint32_t s[4][32];
 #pragma unroll
   for (int c = 0; c < 4; ++c) tmem_ld_x32(sc + c * 32, s[c]);
@@ -223,7 +225,9 @@ __device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, b
     }
   }
   // x = s * scale * log2(e) - m on the packed f32x2 FMA pipe; P chunk c (16
-  // packed columns) lands on S columns already in registers
+  // packed columns) lands on S columns already in registers.  After the first
+  // two chunks (keys 0-63) the warp arrives on p_half, so the first half of
+  // P V can start while the second half is exponentiated.
   const float2 scale2 = make_float2(scale_log2, scale_log2);
   const float2 neg_m2 = make_float2(-m_ref, -m_ref);
   float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -241,25 +245,32 @@ __device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, b
       pk[i] = F8 ? pack_f16x2(e.x, e.y) : pack_bf16x2(e.x, e.y);
     }
     tmem_st_x16(sc + c * 16, pk);
+    if (c == 1) {
+      if (rescale) {
+        // O holds the P V of earlier tiles against the old reference: scale
+        // it by alpha (1 on rows that kept their maximum) before any of this
+        // tile's P V.  S(j) completing implies the previous P V did (one
+        // thread issues both, in order), so this wait ends at once.
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, o_parity, abort_flag))) return false;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int oc32 = 0; oc32 < D / 32; ++oc32) {
+          uint32_t o[32];
+          tmem_ld_x32(oc + oc32 * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_x32(oc + oc32 * 32, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bar_p_half);
+    }
   }
   l_sum = l_sum * alpha + (((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
                            ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y)));
-  if (rescale) {
-    // O still holds the P V of earlier tiles against the old reference: once
-    // the previous P V has landed, scale it by alpha (1 on rows that kept
-    // their maximum).  This tile's P is in TMEM; its P V waits for p_full.
-    if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, o_parity, abort_flag))) return false;
-    tc_fence_after_sync();
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      tmem_ld_x32(oc + c * 32, o);
-      tmem_ld_wait(o);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-      tmem_st_x32(oc + c * 32, o);
-    }
-  }
   return true;
 }
 
@@ -367,6 +378,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
   const uint32_t bar_q1 = bars + 8 * (9 + 2 * C::NS);   // slot 1's Q tile
   auto bar_vh_full = [&](int sl) { return bars + 8 * (10 + 2 * C::NS + sl); };
   auto bar_vh_empty = [&](int sl) { return bars + 8 * (12 + 2 * C::NS + sl); };
+  auto bar_p_half = [&](int k) { return bars + 8 * (C::P_HALF_BAR + k); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -381,6 +393,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s_full(k), 1);
       mbar_init(bar_p_full(k), 4);
+      mbar_init(bar_p_half(k), 4);
       mbar_init(bar_o_done(k), 1);
       if constexpr (F8) {
         mbar_init(bar_vh_full(k), 2);
@@ -570,14 +583,15 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
           else mma_bf16_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int k, int item, bool accumulate) {
+      // O_k += P_k V over keys 64h .. 64h+63 (the P columns of half h)
+      auto issue_pv_half = [&](int k, int item, bool accumulate, int h) {
         const uint32_t o_tmem = tmem + 256u + (k ? D : 0);
         const uint32_t p_tmem = tmem + (k ? 128u : 0u);
         // F8: the f16 copy of V_j in slot j & 1 (item = 2j + 1)
         const uint64_t vd = F8 ? v_desc0 + static_cast<uint64_t>((((item >> 1) & 1) * C::VH_TILE) >> 4)
                                : v_desc0 + ring_off(item);
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
+        for (int kk = h * C::BN / 32; kk < (h + 1) * C::BN / 32; ++kk)
           mma_bf16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                       (accumulate || kk > 0) ? 1u : 0u);
       };
@@ -604,9 +618,13 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
       // them was issued first and MMAs of one thread run in order.
       auto slot_step = [&](int k, int nk, int j, int v_item, int k_item) -> bool {
         if (j >= nk) return true;
+        // the first half of P V starts while the softmax finishes the second half
+        if (!mbar_wait(bar_p_half(k), j & 1, abort_flag)) return false;
+        tc_fence_after_sync();
+        issue_pv_half(k, v_item, j > 0, 0);
         if (!mbar_wait(bar_p_full(k), j & 1, abort_flag)) return false;
         tc_fence_after_sync();
-        issue_pv(k, v_item, j > 0);
+        issue_pv_half(k, v_item, true, 1);
         tc_commit(bar_o_done(k));
         if (j + 1 < nk) {
           issue_qk(k, k_item);
@@ -689,7 +707,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
       const bool masked = (kt0 + j) * C::BN + C::BN - 1 > tile_last;
       if (!prefill_softmax_tile<D, F8>(sc, oc, j == 0, masked, row_last - (kt0 + j) * C::BN,
                                                      p.scale_log2, m_ref, l_sum, bar_o_done(k),
-                                                     (j - 1) & 1, abort_flag)) {
+                                                     (j - 1) & 1, bar_p_half(k), abort_flag)) {
         ok = false;
         break;
       }

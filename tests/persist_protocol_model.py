@@ -213,7 +213,7 @@ def prefill_items(lens, num_q_heads, num_kv_heads, causal, BM=128, BN=128):
 
 
 MUTATIONS = ("no_q_empty_wait", "late_q_empty", "no_epilogue_wait", "consumers_short",
-             "no_vh_empty_wait", "v_release_before_pv")
+             "no_vh_empty_wait", "v_release_before_pv", "rescale_after_half")
 
 
 def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
@@ -229,6 +229,7 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
     for k in range(2):
         sim.bar(f"s_full{k}")
         sim.bar(f"p_full{k}", 4)
+        sim.bar(f"p_half{k}", 4)
         sim.bar(f"o_done{k}")
         sim.bar(f"q_empty{k}")
         if F8:
@@ -304,7 +305,7 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
                 if nk[k] > 0:
                     yield ("wait", f"q{k}", qc[k])
                     yield ("mma", [(f"qtile{k}", ("Q", it, k)), (f"ring{ring % NS}", ("KV", it, 0))],
-                           [(f"sp{k}", ("S", it, k, 0), None)])
+                           [(f"sp{k}a", ("S", it, k, 0), None), (f"sp{k}b", ("S", it, k, 0), None)])
                     yield ("commit", f"s_full{k}")
                     if nk[k] == 1:
                         yield ("commit", f"q_empty{k}")
@@ -314,7 +315,7 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
             def slot_step(k, j, v_R, vslot, k_R, it=it, nk=nk):
                 if j >= nk[k]:
                     return
-                yield ("wait", f"p_full{k}", tiles[k] + j)
+                yield ("wait", f"p_half{k}", tiles[k] + j)
                 v = (f"vh{vslot}", ("VH", it, j)) if F8 else (f"ring{v_R % NS}", ("KV", it, 2 * j + 1))
 
                 def check_o(k=k, j=j, it=it):
@@ -323,11 +324,18 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
                     if j > 0 and o_state[k] != (it, j):
                         sim.err(f"P V ({it}, {j}) accumulates onto {o_state[k]}")
                     o_state[k] = (it, j + 1)
-                yield ("mma", [(f"sp{k}", ("P", it, k, j)), v], [(f"o{k}", ("O", it, k, j + 1), check_o)])
+                # P V over the first 64 keys, then (p_full) the last 64
+                yield ("mma", [(f"sp{k}a", ("P", it, k, j)), v], [(f"o{k}", ("O half", it, k, j + 1), check_o)])
+                yield ("wait", f"p_full{k}", tiles[k] + j)
+                def check_half(k=k, j=j, it=it):
+                    cur = sim.content.get(f"o{k}")
+                    if cur is None or cur[0] != ("O half", it, k, j + 1):
+                        sim.err(f"second half of P V ({it}, {j}) accumulates onto {cur and cur[0]}")
+                yield ("mma", [(f"sp{k}b", ("P", it, k, j)), v], [(f"o{k}", ("O", it, k, j + 1), check_half)])
                 yield ("commit", f"o_done{k}")
                 if j + 1 < nk[k]:
                     yield ("mma", [(f"qtile{k}", ("Q", it, k)), (f"ring{k_R % NS}", ("KV", it, 2 * j + 2))],
-                           [(f"sp{k}", ("S", it, k, j + 1), None)])
+                           [(f"sp{k}a", ("S", it, k, j + 1), None), (f"sp{k}b", ("S", it, k, j + 1), None)])
                     yield ("commit", f"s_full{k}")
                     if j + (3 if mutation == "late_q_empty" else 2) == nk[k]:
                         yield ("commit", f"q_empty{k}")
@@ -395,16 +403,30 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
             for j in range(nk):
                 g = tiles + j
                 yield ("wait", f"s_full{k}", g)
-                if wq == 0:          # the warpgroup's S read and P store, modelled once
-                    yield ("read", f"sp{k}", ("S", it, k, j))
-                yield ("delay", rng.uniform(0.5, 2.0))
+                if wq == 0:          # the warpgroup's S read and P stores, modelled once
+                    yield ("read", f"sp{k}a", ("S", it, k, j))
+                    yield ("read", f"sp{k}b", ("S", it, k, j))
+                yield ("delay", rng.uniform(0.3, 1.0))
                 if wq == 0:
-                    yield ("write", f"sp{k}", ("P", it, k, j))
+                    yield ("write", f"sp{k}a", ("P", it, k, j))
                 if j > 0 and rescale[(it, k, j)]:
+                    # before any of this tile's P V: the previous P V has landed
+                    if mutation != "rescale_after_half":
+                        yield ("wait", f"o_done{k}", g - 1)
+                        yield ("delay", rng.uniform(0.1, 0.5))   # the O loads take time
+                        if wq == 0:
+                            yield ("read", f"o{k}", ("O", it, k, j))
+                            yield ("write", f"o{k}", ("O", it, k, j))
+                yield ("arrive", f"p_half{k}")
+                if j > 0 and rescale[(it, k, j)] and mutation == "rescale_after_half":
                     yield ("wait", f"o_done{k}", g - 1)
+                    yield ("delay", rng.uniform(0.1, 0.5))
                     if wq == 0:
                         yield ("read", f"o{k}", ("O", it, k, j))
                         yield ("write", f"o{k}", ("O", it, k, j))
+                yield ("delay", rng.uniform(0.3, 1.0))
+                if wq == 0:
+                    yield ("write", f"sp{k}b", ("P", it, k, j))
                 yield ("arrive", f"p_full{k}")
             if nk == 0:
                 continue
