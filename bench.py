@@ -788,15 +788,16 @@ def kernel_source_hash(kind):
 
 
 def measured_traffic(kind, workload, case=None):
-    """DRAM bytes per launch from profiles/dram_traffic.md, or None when no
-    capture matches the current kernel source.  The paged decode batch is too
-    large for a multi-pass capture, so its 16-request capture is scaled by KV
-    bytes (traffic tracks the KV read one-for-one)."""
+    """(DRAM bytes per launch, how it was obtained) from profiles/dram_traffic.md,
+    or (None, None) when no capture matches the current kernel source.  A decode
+    workload without its own row uses the 16-request capture of the same split
+    kernel scaled by K/V bytes (every decode capture reads its K/V bytes one for
+    one); the full-size workloads are too large for a multi-pass capture."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     try:
         lines = open(path).read().splitlines()
     except OSError:
-        return None
+        return None, None
     rows = {}
     for ln in lines:
         parts = [x.strip() for x in ln.strip().strip("|").split("|")]
@@ -805,14 +806,15 @@ def measured_traffic(kind, workload, case=None):
             rows[(parts[0], parts[1])] = (parts[2], int(parts[3]) + int(parts[4]))
     sha = kernel_source_hash(kind)
     if (kind, workload) in rows and rows[(kind, workload)][0] == sha:
-        return rows[(kind, workload)][1]
-    if kind in ("decode", "decode_tc") and workload == "paged_decode_batch" and \
+        return rows[(kind, workload)][1], "ncu capture of this workload"
+    if kind in ("decode", "decode_tc") and case is not None and not case.fp8 and \
             (kind, "paged_decode_batch16") in rows:
         h, t16 = rows[(kind, "paged_decode_batch16")]
-        if h == sha and case is not None:
+        if h == sha:
             kv16 = 2.0 * float(np.sum(W.paged_decode_batch16_lengths())) * 8 * 128 * 2
-            return int(t16 * case.inp.kv_bytes() / kv16)
-    return None
+            return int(t16 * case.inp.kv_bytes() / kv16), \
+                "16-request ncu capture of the same split kernel, scaled by K/V bytes"
+    return None, None
 
 
 def aggregate_throughput(work_per_replica: float, ms_max: float, n_replicas: int, scale: float) -> float:
@@ -821,7 +823,8 @@ def aggregate_throughput(work_per_replica: float, ms_max: float, n_replicas: int
     return n_replicas * work_per_replica / (ms_max * 1e-3) / scale
 
 
-def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=None, fp8_qk=False):
+def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=(None, None), fp8_qk=False):
+    traffic, traffic_src = traffic
     if kind == "tensor":
         achieved = algorithmic / (ms_per_launch * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
@@ -833,12 +836,12 @@ def roofline_entry(kind, algorithmic, ms_per_launch, peaks, peak_src, traffic=No
             peak, spec = round(peak * 4.0 / 3.0, 1), spec * 4.0 / 3.0
             src += " x 4/3 (Q K^T at the fp8 rate = 2 x bf16 nominal, P V at the f16 rate)"
         return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
-                "frac_of_spec": round(achieved / spec, 4)}
+                "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_source": traffic_src,
+                "peak_source": src, "frac_of_spec": round(achieved / spec, 4)}
     achieved = algorithmic / (ms_per_launch * 1e-3) / 1e9
     peak = peaks["hbm_gbs"]
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_source": traffic_src,
             "peak_source": f"{peak_src} HBM copy", "frac_of_spec": round(achieved / SPEC_PEAKS["hbm_gbs"], 4)}
 
 
@@ -949,7 +952,7 @@ def run_ours(args):
                                measured_traffic("prefill", c.inp.name))
             e["kernel"] = "fa_prefill_pp_kernel<%d, paged>" % c.inp.head_dim
         elif isinstance(c, CascadeCase):
-            e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src, None)
+            e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src)
             e["kernel"] = "fa_prefill_pp_kernel<paged, key ranges> + decode split + fa_cascade_merge_kernel"
         elif isinstance(c, AppendCase):
             e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src,
