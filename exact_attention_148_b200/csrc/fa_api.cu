@@ -398,6 +398,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* cu_
     if (st != FA_OK) return st;
   }
   prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.out_v8 = aligned(out, 32) ? 1 : 0;
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_dev;
   prm.total_q = static_cast<int>(T);
@@ -508,6 +509,7 @@ FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
                             &prm.head_coord, &prm.page_coord);
   if (st != FA_OK) return st;
   prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.out_v8 = aligned(out, 32) ? 1 : 0;
   prm.lse = lse;
   prm.cu_seqlens = cu_seqlens_q_dev;
   prm.total_q = static_cast<int>(T);

@@ -518,12 +518,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(__uint_as_float(o[c][2 * i]) * inv_l, __uint_as_float(o[c][2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
+        if (valid) store_o_chunk(orow + c * 32, pk, p.out_v8);
       }
       if (valid && p.lse != nullptr)
         p.lse[static_cast<size_t>(w.s0 + q_row) * p.num_q_heads + my_head] =

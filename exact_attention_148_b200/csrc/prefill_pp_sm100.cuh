@@ -75,6 +75,7 @@ struct PrefillParams {
   int head_coord;            // paged: tensor-map dimension (1..3) of the kv head
   int page_coord;            // paged: tensor-map dimension (1..3) of the page id
   int num_q_heads;
+  int out_v8;                // out is 32-byte aligned: O rows go out in 32-byte stores
   int batch;                 // sequences (rows of cu_seqlens - 1, of block_table)
   int group;                 // Hq / Hkv
   int causal;
@@ -180,6 +181,19 @@ constexpr int kPrefillPage = 64;
 // when the tile's maximum exceeds it by more than kRescaleThreshold; then O
 // (columns oc ..) is rescaled once the previous P V has landed (o_done,
 // parity o_parity).  Returns false when a wait gave up.
+// 32 bf16 columns of one O row (64 bytes): two 32-byte stores (whole L2
+// sectors) when the output is 32-byte aligned, else four 16-byte stores.
+__device__ __forceinline__ void store_o_chunk(__nv_bfloat16* dst, const uint32_t (&pk)[16], int v8) {
+  if (v8) {
+    st_global_v8(dst, pk);
+    st_global_v8(dst + 16, pk + 8);
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) d4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+  }
+}
+
 template <int D, bool F8>
 __device__ __forceinline__ bool prefill_softmax_tile(uint32_t sc, uint32_t oc, bool first, bool masked,
                                                      int lim, float scale_log2, float& m_ref,
@@ -754,12 +768,7 @@ __global__ void __launch_bounds__(PrefillPPCfg<D, F8>::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(__uint_as_float(o[c][2 * i]) * inv_l, __uint_as_float(o[c][2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
+        if (valid) store_o_chunk(orow + c * 32, pk, p.out_v8);
       }
       if (valid && p.lse != nullptr)
         p.lse[static_cast<size_t>(s0 + q_row) * p.num_q_heads + my_head] =

@@ -156,6 +156,22 @@ def test_deterministic():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+def test_output_only_16_byte_aligned(schedule, monkeypatch):
+    """An `out` that is 16- but not 32-byte aligned takes the 16-byte stores;
+    its bytes equal those of a 32-byte aligned `out`."""
+    import torch
+    monkeypatch.setenv("FA_PREFILL_SCHEDULE", schedule)
+    inp = W.make_prefill([300, 129], 4, 2, 128, causal=True, seed=43)
+    a, la = prefill_on_gpu(inp)
+    T, H, d = a.shape
+    buf = torch.empty(T * H * d + 8, dtype=torch.bfloat16, device=a.device)
+    out = buf[8:].view(T, H, d)   # 16 bytes past a 256-byte aligned allocation
+    assert out.data_ptr() % 32 == 16
+    b, lb = prefill_on_gpu(inp, out=out)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
 def test_without_lse_matches():
     import torch
     inp = W.make_prefill([257], 2, 2, 128, causal=True, seed=41)
