@@ -25,9 +25,10 @@
 // shared-memory queue guarded by item_full / item_empty mbarriers, so no role
 // but the producer reads global memory between items.  Every role takes every
 // item, so all per-role counters (ring entries, Q loads, tiles per slot, f16
-// V tiles) advance identically.  While an item runs, the producer has already
-// claimed the next one and asked L2 for its Q tiles and first K/V tiles.  The counter pair {next item, CTAs finished} is reset
-// by the last CTA to finish, ready for the next launch on the same stream;
+// V tiles) advance identically.  Once the last load of an item is issued, the
+// producer claims the next one and asks L2 for its Q tiles and first K/V
+// tiles.  The counter pair {next item, CTAs finished} is reset by the last CTA
+// to finish, ready for the next launch on the same stream;
 // the host gives each stream its own pair.
 #pragma once
 
@@ -267,7 +268,6 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
         queue[qi] = w;
         mbar_arrive(bar_item_full(qi));
         if (w.id < 0) break;
-        next = claim();   // claimed and prefetched now, started after this item
         const int n_max = max(w.n_kv[0], w.n_kv[1]);
         // ring entries K_0, V_0, K_1, V_1, ...; both Q tiles right after K_0
         for (int e = 0; e < 2 * n_max; ++e) {
@@ -294,6 +294,12 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
             }
           }
         }
+        // The next item is claimed (and its first tiles asked of L2) only once
+        // every load of this one is issued, about NS ring entries before this
+        // item's last MMA: a CTA holds at most one item it has not started, so
+        // near the end of the launch the last items go to the CTAs that free
+        // up first.
+        if (ok) next = claim();
       }
       if (*abort_flag) {
         // let the copies in flight land before the CTA's shared memory goes away
