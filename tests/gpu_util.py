@@ -107,3 +107,24 @@ def oracle_pool_after_append(inp: W.ChunkedPrefillInputs):
     return oracle.append_kv_ref(inp.k_pages_bits, inp.v_pages_bits, inp.k_new_bits, inp.v_new_bits,
                                 inp.cu_seqlens_q, inp.block_table, inp.cache_seqlens,
                                 inp.page_size, inp.layout)
+
+
+def jumping_keys(inp, factors, tile=128):
+    """inp with the key rows of key tile t of every sequence multiplied by
+    factors[t % len(factors)]: scores that jump far above (or below) the
+    earlier tiles' from one key tile to the next."""
+    import workloads as W
+    k = W.bf16_bits_to_f32(inp.k_bits).copy()
+    cu = inp.cu_seqlens
+    for b in range(len(cu) - 1):
+        for t0 in range(int(cu[b]), int(cu[b + 1]), tile):
+            k[t0:min(t0 + tile, int(cu[b + 1]))] *= factors[((t0 - int(cu[b])) // tile) % len(factors)]
+    inp.k_bits = W.f32_to_bf16_bits(k)
+    return inp
+
+
+# Per-tile key scales: x8 lifts a tile's scores ~30 (base 2) above the first
+# tile's (past the rescale threshold, under the bf16 overflow guard of 64),
+# x25 and x40 by 65-75 more (past the guard).  Scores stay near 120, where
+# fp32 scores still meet the LSE bound.
+JUMP_FACTORS = [1.0, 8.0, 1.0, 25.0, 3.0, 40.0, 0.5, 12.0]

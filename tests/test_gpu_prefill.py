@@ -4,7 +4,8 @@ import pytest
 
 import oracle
 import workloads as W
-from tests.gpu_util import bf16_to_f64, compare, prefill_on_gpu, to_dev_bf16, to_dev_i32
+from tests.gpu_util import (JUMP_FACTORS, bf16_to_f64, compare, jumping_keys, prefill_on_gpu, to_dev_bf16,
+                            to_dev_i32)
 
 pytestmark = pytest.mark.gpu
 
@@ -170,6 +171,18 @@ def test_output_only_16_byte_aligned(schedule, monkeypatch):
     assert out.data_ptr() % 32 == 16
     b, lb = prefill_on_gpu(inp, out=out)
     assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+def test_score_jumps_between_key_tiles(schedule, monkeypatch):
+    """Scores that jump by tens to hundreds (base 2) from one key tile to the
+    next: the reference maximum raised a tile late, and re-referenced at once
+    where a tile's P would otherwise overflow, against the oracle."""
+    monkeypatch.setenv("FA_PREFILL_SCHEDULE", schedule)
+    inp = jumping_keys(W.make_prefill([700, 300, 1000, 129], 4, 2, 128, causal=True, seed=47), JUMP_FACTORS)
+    check_full(inp, f"score jumps ({schedule})")
+    inp = jumping_keys(W.make_prefill([1000, 257], 2, 2, 64, causal=False, seed=48), [1.0, 6.0, 1.0, 16.0, 2.0])
+    check_full(inp, f"score jumps, d=64, full attention ({schedule})")
 
 
 def test_without_lse_matches():

@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 import workloads as W
-from tests.gpu_util import bf16_to_f64, compare, to_dev_i32
+from tests.gpu_util import JUMP_FACTORS, bf16_to_f64, compare, jumping_keys, to_dev_i32
 
 pytestmark = pytest.mark.gpu
 
@@ -74,6 +74,18 @@ def test_saturated_codes_and_unequal_scales():
     assert (inp.v_bits & 0x7F == 0x7E).mean() > 0.05          # many +-448 codes
     inp.q_scale, inp.k_scale, inp.v_scale = inp.q_scale * 2.0, inp.k_scale * 0.5, inp.v_scale * 3.0
     check_full(inp, "fp8 saturated, unequal scales")
+
+
+def test_score_jumps_between_key_tiles_fp8():
+    """Key tiles scaled by up to 200: with f16 P the overflow guard (2^15)
+    re-references most jumping tiles at once; K gets its own scale so the
+    large keys do not saturate."""
+    base = jumping_keys(W.make_prefill([700, 300, 1000], 4, 2, 128, causal=True, seed=49), JUMP_FACTORS)
+    inp = W.to_fp8_prefill(base)
+    kf = W.bf16_bits_to_f32(base.k_bits)
+    inp.k_scale = float(np.abs(kf).max()) / W.E4M3_MAX
+    inp.k_bits = W.quantize_e4m3(kf, inp.k_scale)
+    check_full(inp, "fp8 score jumps")
 
 
 def test_matches_bf16_kernel_on_exact_inputs():
