@@ -380,6 +380,8 @@ class ChunkedAttnCase:
         fa.prefill_paged(s.q, s.cu, s.kp, s.vp, s.bt, s.lens, causal=s.inp.causal, scale=s.inp.scale,
                          layout=s.inp.layout, out=s.out, lse=s.lse,
                          cu_seqlens_q_host=s.inp.cu_seqlens_q, cache_seqlens_host=s.inp.cache_seqlens)
+        # the schedule the library actually launched (see PrefillCase.run)
+        self.schedule = fa.prefill_last_schedule()
 
     def run_e2e(self):
         import torch
@@ -399,7 +401,7 @@ class ChunkedAttnCase:
         return {"workload": i.name, "batch": i.batch, "chunk_tokens_total": int(i.chunk_lens.sum()),
                 "prefix_tokens_total": int(i.prefix_lens.sum()), "num_q_heads": i.num_q_heads,
                 "num_kv_heads": i.num_kv_heads, "head_dim": i.head_dim, "page_size": i.page_size,
-                "layout": i.layout, "causal": bool(i.causal),
+                "layout": i.layout, "causal": bool(i.causal), "schedule": getattr(self, "schedule", None),
                 "algorithmic_tflop": round(self.flops / 1e12, 4)}
 
 
@@ -948,9 +950,11 @@ def run_ours(args):
         if isinstance(c, PrefillCase):
             e = case_roofline(c, ms, peaks, peak_src)
         elif isinstance(c, ChunkedAttnCase):
+            pers = getattr(c, "schedule", None) == "persistent"
             e = roofline_entry("tensor", c.flops, ms / c.launches, peaks, peak_src,
-                               measured_traffic("prefill", c.inp.name))
-            e["kernel"] = "fa_prefill_pp_kernel<%d, paged>" % c.inp.head_dim
+                               measured_traffic("prefill_persist" if pers else "prefill", c.inp.name))
+            e["kernel"] = "%s<%d, paged>" % ("fa_prefill_persist_kernel" if pers else "fa_prefill_pp_kernel",
+                                             c.inp.head_dim)
         elif isinstance(c, CascadeCase):
             e = roofline_entry("hbm", c.bytes, ms, peaks, peak_src)
             e["kernel"] = "fa_prefill_pp_kernel<paged, key ranges> + decode split + fa_cascade_merge_kernel"

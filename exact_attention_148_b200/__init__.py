@@ -250,8 +250,9 @@ def prefill(q, k, v, cu_seqlens, *, causal: bool = True, scale: float | None = N
 
 
 def prefill_last_schedule() -> str | None:
-    """"persistent" or "grid": the schedule the calling thread's last prefill /
-    prefill_fp8 launched (None if that call failed or there was none)."""
+    """"persistent" or "grid": the schedule the calling thread's last prefill,
+    prefill_fp8 or prefill_paged launched (None if that call failed or there
+    was none)."""
     return {FA_SCHEDULE_GRID: "grid", FA_SCHEDULE_PERSISTENT: "persistent"}.get(
         library().fa_prefill_last_schedule())
 

@@ -142,12 +142,12 @@ int launch_prefill(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t,
 }
 
 // Persistent prefill (packed Q/K/V): one CTA per SM, items from a counter.
-template <int D, bool F8>
+template <int D, bool F8, bool PAGED = false>
 int launch_prefill_persistent(fa::PrefillParams& prm, const std::vector<std::pair<uint32_t, int>>& groups,
                               cudaStream_t stream, uint32_t* sched, int num_sms) {
-  constexpr int kSmem = fa::PrefillPersistCfg<D, F8>::SMEM_BYTES;
-  constexpr int kThreads = fa::PrefillPersistCfg<D, F8>::THREADS;
-  auto kernel = fa::fa_prefill_persist_kernel<D, F8>;
+  constexpr int kSmem = fa::PrefillPersistCfg<D, F8, PAGED>::SMEM_BYTES;
+  constexpr int kThreads = fa::PrefillPersistCfg<D, F8, PAGED>::THREADS;
+  auto kernel = fa::fa_prefill_persist_kernel<D, F8, PAGED>;
   int st = ensure_smem(reinterpret_cast<const void*>(kernel), kSmem);
   if (st != FA_OK) return st;
   for (size_t off = 0; off < groups.size(); off += fa::kPrefillMaxGroups) {
@@ -523,8 +523,20 @@ FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return head_dim == 128 ? launch_prefill<128, true>(prm, groups, s)
-                         : launch_prefill<64, true>(prm, groups, s);
+  t_last_prefill_schedule = -1;
+  if (prefill_persistent_requested()) {
+    uint32_t* sched = prefill_sched_slot(s);
+    int sms = 0;
+    if (sched != nullptr && sm_count(&sms) == FA_OK) {
+      st = head_dim == 128 ? launch_prefill_persistent<128, false, true>(prm, groups, s, sched, sms)
+                           : launch_prefill_persistent<64, false, true>(prm, groups, s, sched, sms);
+      if (st == FA_OK) t_last_prefill_schedule = FA_SCHEDULE_PERSISTENT;
+      return st;
+    }
+  }
+  st = head_dim == 128 ? launch_prefill<128, true>(prm, groups, s) : launch_prefill<64, true>(prm, groups, s);
+  if (st == FA_OK) t_last_prefill_schedule = FA_SCHEDULE_GRID;
+  return st;
 }
 
 FA_API int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_seqlens_new_dev,

@@ -45,15 +45,17 @@ constexpr int kSchedSlots = 256;     // counter pairs: one per stream that launc
 // form's CTA index: groups in launch order, heaviest q tiles first in a group.
 struct PrefillItem {
   int id;          // item number, or -1: no more work
-  int s0;          // first token of the sequence
-  int L;           // its length (queries = keys)
+  int s0;          // first query of the sequence in the packed rows
+  int L;           // its queries
+  int Lk;          // its keys (= L for packed K/V; the cached length when paged)
+  int seq;         // sequence (row of the block table when paged)
   int kv_head;
   int qtile[2];
   int head[2];
   int n_kv[2];     // key tiles of each slot (0: slot unused)
 };
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool PAGED = false>
 struct PrefillPersistCfg {
   using B = PrefillPPCfg<D, F8>;
   // B's barriers, then q_empty[2], item_full[kPersistQueue], item_empty[kPersistQueue]
@@ -67,6 +69,7 @@ struct PrefillPersistCfg {
   static constexpr int CONSUMERS = 1 + 8 + (F8 ? 2 : 0);
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(!F8 || B::NS % 2 == 0, "E4M3: V tiles must stay on odd ring slots");
+  static_assert(!(F8 && PAGED), "E4M3 inputs: packed K/V only");
 };
 
 // Launch arguments: the grid form's, plus the work counter.
@@ -79,7 +82,11 @@ struct PrefillPersistParams {
 // Decode item idx.  The sequence bounds come from the device cu_seqlens; a
 // sequence that leaves the T packed rows, or whose tile count differs from
 // what the host planned for its group (cu_seqlens_dev != cu_seqlens_host), is
-// recorded as FA_ERR_PLAN_MISMATCH and becomes an empty item.
+// recorded as FA_ERR_PLAN_MISMATCH and becomes an empty item.  PAGED: the
+// keys are the sequence's cached length (cache_seqlens_dev); one below the
+// query count or above the block table's capacity is recorded the same way
+// and clamped, as in the grid form.
+template <bool PAGED = false>
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int idx, int BM, int BN) {
   int lo = 0, hi = p.num_groups - 1;
   while (lo < hi) {
@@ -92,11 +99,25 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   w.kv_head = static_cast<int>(p.group_id[lo] & 0xFFFFu);
   const int rank = idx - p.group_start[lo];
   const bool seq_ok = FA_DBG_OK(seq < p.batch);
+  w.seq = seq;
   w.s0 = seq_ok ? p.cu_seqlens[seq] : -1;
   w.L = seq_ok ? p.cu_seqlens[seq + 1] - w.s0 : 0;
+  w.Lk = w.L;
+  if constexpr (PAGED) {
+    if (seq_ok) {
+      int Lk = p.cache_seqlens[seq];
+      const int cap = p.max_pages * kPrefillPage;
+      if ((p.causal && Lk < w.L) || Lk > cap || Lk < 0) {
+        if (rank == 0) record_status(FA_ERR_PLAN_MISMATCH);
+        Lk = min(max(Lk, p.causal ? w.L : 0), cap);
+      }
+      w.Lk = Lk;
+    }
+  }
   const bool in_rows = w.s0 >= 0 && w.L >= 1 && w.s0 <= p.total_q - w.L;
   const int n_qtiles = in_rows ? (w.L + BM - 1) / BM : 0;
-  const int n_ktiles = in_rows ? (w.L + BN - 1) / BN : 0;
+  const int n_ktiles = in_rows ? (w.Lk + BN - 1) / BN : 0;
+  const int off = p.causal ? w.Lk - w.L : 0;   // query i sits at key position i + off
   const int G = p.group;
   const int planned = p.group_start[lo + 1] - p.group_start[lo];
   const int derived = ((G & 1) == 0) ? n_qtiles * (G >> 1) : ((n_qtiles + 1) >> 1) * G;
@@ -104,6 +125,7 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     if (rank == 0) record_status(FA_ERR_PLAN_MISMATCH);
     w.s0 = 0;
     w.L = 0;
+    w.Lk = 0;
     w.qtile[0] = w.qtile[1] = -1;
     w.head[0] = w.head[1] = 0;
     w.n_kv[0] = w.n_kv[1] = 0;
@@ -125,17 +147,17 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const bool active = w.qtile[k] >= 0 && w.qtile[k] < n_qtiles;
-    w.n_kv[k] = !active ? 0 : (p.causal ? min(n_ktiles, (w.qtile[k] * BM + BM - 1) / BN + 1) : n_ktiles);
+    w.n_kv[k] = !active ? 0 : (p.causal ? min(n_ktiles, (w.qtile[k] * BM + BM - 1 + off) / BN + 1) : n_ktiles);
   }
   return w;
 }
 
-template <int D, bool F8 = false>
-__global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
+template <int D, bool F8 = false, bool PAGED = false>
+__global__ void __launch_bounds__(PrefillPersistCfg<D, F8, PAGED>::THREADS, 1)
     fa_prefill_persist_kernel(const __grid_constant__ PrefillPersistParams pp) {
   const PrefillParams& p = pp.p;
   using B = PrefillPPCfg<D, F8>;
-  using C = PrefillPersistCfg<D, F8>;
+  using C = PrefillPersistCfg<D, F8, PAGED>;
   constexpr int NS = B::NS;
   constexpr int QD = kPersistQueue;
   extern __shared__ uint8_t smem_raw[];
@@ -156,6 +178,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
   auto bar_p_full = [&](int k) { return bars + 8 * (3 + 2 * NS + k); };
   auto bar_o_done = [&](int k) { return bars + 8 * (5 + 2 * NS + k); };
   const uint32_t bar_final = bars + 8 * (7 + 2 * NS);
+  const uint32_t bar_vtail = bars + 8 * (8 + 2 * NS);   // PAGED: a V tile whose last page ends early
   const uint32_t bar_q1 = bars + 8 * (9 + 2 * NS);
   auto bar_vh_full = [&](int sl) { return bars + 8 * (10 + 2 * NS + sl); };
   auto bar_vh_empty = [&](int sl) { return bars + 8 * (12 + 2 * NS + sl); };
@@ -193,6 +216,7 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
       mbar_init(bar_item_empty(i), C::CONSUMERS);
     }
     mbar_init(bar_final, 1);
+    mbar_init(bar_vtail, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -220,7 +244,167 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
     return w;
   };
 
-  if (warp == 8) {
+  if (PAGED && warp == 8) {
+    // ------------------------------------------ TMA producer + scheduler, paged K/V
+    // The packed producer's order, with the grid form's paged loads: key tile
+    // jt is logical pages 2jt and 2jt+1, whose physical ids the whole warp
+    // reads 32 at a time; a page past the cache end or outside the pool loads
+    // from page index num_pages (TMA zero fill, the bad id recorded).  The V
+    // tile holding the cache's last page, when that page ends early, lands on
+    // bar_vtail; once the item's loads are issued the warp zeroes the rows
+    // past the end (0 * NaN would otherwise reach O) and marks the tile full.
+    // Lane 0 claims the items and issues every copy and barrier operation.
+    auto load_q = [&](int k, int h, int row0, uint32_t bar) {
+      mbar_arrive_expect_tx(bar, B::TILE_BYTES);
+#pragma unroll
+      for (int c = 0; c < B::CHUNKS; ++c)
+        tma_load_3d(q_s + k * B::TILE_BYTES + c * B::CHUNK_BYTES, &p.tm_q, bar, c * 64, h, row0);
+    };
+    auto claim = [&]() -> PrefillItem {   // lane 0
+      const int id = static_cast<int>(atomicAdd(pp.sched, 1u));
+      PrefillItem w;
+      if (id >= pp.total_items) {
+        w.id = -1;
+        return w;
+      }
+      w = prefill_item<true>(p, id, B::BM, B::BN);
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (w.n_kv[k] > 0)
+#pragma unroll
+          for (int c = 0; c < B::CHUNKS; ++c)
+            tma_prefetch_l2_3d(&p.tm_q, c * 64, w.head[k], w.s0 + w.qtile[k] * B::BM);
+      return w;
+    };
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+    }
+    uint32_t issued = 0;          // ring entries issued
+    int qc0 = 0, qc1 = 0;         // Q loads of each slot
+    int tails = 0;                // tail V tiles zeroed (bar_vtail phases)
+    int tail_R = -1;              // ring entry of the tail V tile not yet marked full
+    PrefillItem next;
+    if (lane == 0) next = claim();
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      const int qi = n % QD;
+      if (lane == 0) {
+        ok = mbar_wait(bar_item_empty(qi), ((n / QD) & 1) ^ 1, abort_flag);
+        if (ok) {
+          queue[qi] = next;
+          mbar_arrive(bar_item_full(qi));
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      __syncwarp();
+      const PrefillItem w = queue[qi];   // rewritten only QD items later
+      if (w.id < 0) break;
+      const int n_max = max(w.n_kv[0], w.n_kv[1]);
+      const int32_t* bt_row = p.block_table + static_cast<size_t>(w.seq) * p.max_pages;
+      const int tail_tile = (w.Lk % kPrefillPage != 0) ? (w.Lk - 1) / B::BN : -1;
+      int pg_base = -1, pg_mine = 0;
+      // ring entries K_0, V_0, K_1, V_1, ...; both Q tiles right after K_0
+      for (int e = 0; e < 2 * n_max; ++e) {
+        const int jt = e >> 1;
+        const int lp0 = 2 * jt;
+        if ((lp0 & ~31) != pg_base) {
+          pg_base = lp0 & ~31;
+          const int lp = pg_base + lane;
+          int id = p.num_pages;
+          if (lp * kPrefillPage < w.Lk && FA_DBG_OK(lp < p.max_pages)) {
+            id = bt_row[lp];
+            if (id < 0 || id >= p.num_pages) {
+              record_status(FA_ERR_BAD_PAGE);
+              id = p.num_pages;
+            }
+          }
+          pg_mine = id;
+        }
+        const int ph0 = __shfl_sync(0xffffffffu, pg_mine, lp0 & 31);
+        const int ph1 = __shfl_sync(0xffffffffu, pg_mine, (lp0 + 1) & 31);
+        if (lane == 0) {
+          const uint32_t R = issued;
+          if (mbar_wait(bar_kv_empty(R), ((R / NS) & 1) ^ 1, abort_flag)) {
+            const bool vtail = (e & 1) && jt == tail_tile;
+            const uint32_t bar = vtail ? bar_vtail : bar_kv_full(R);
+            mbar_arrive_expect_tx(bar, B::TILE_BYTES);
+            const CUtensorMap* map = (e & 1) ? &p.tm_v : &p.tm_k;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int phys = h ? ph1 : ph0;
+              const int c1 = (p.head_coord == 1) ? w.kv_head : (p.page_coord == 1 ? phys : 0);
+              const int c2 = (p.head_coord == 2) ? w.kv_head : (p.page_coord == 2 ? phys : 0);
+              const int c3 = (p.head_coord == 3) ? w.kv_head : (p.page_coord == 3 ? phys : 0);
+#pragma unroll
+              for (int c = 0; c < B::CHUNKS; ++c)
+                tma_load_4d(kv_s(R) + c * B::CHUNK_BYTES + h * (B::CHUNK_BYTES / 2), map, bar, c * 64, c1, c2,
+                            c3);
+            }
+            ++issued;
+            if (vtail) tail_R = static_cast<int>(R);
+            if (e == 0) {
+              // a slot's Q tile is free once the last S MMA of its previous item completed
+              if (w.n_kv[0] > 0) {
+                ok = mbar_wait(bar_q_empty(0), (qc0 & 1) ^ 1, abort_flag);
+                if (ok) {
+                  load_q(0, w.head[0], w.s0 + w.qtile[0] * B::BM, bar_q);
+                  ++qc0;
+                }
+              }
+              if (ok && w.n_kv[1] > 0) {
+                ok = mbar_wait(bar_q_empty(1), (qc1 & 1) ^ 1, abort_flag);
+                if (ok) {
+                  load_q(1, w.head[1], w.s0 + w.qtile[1] * B::BM, bar_q1);
+                  ++qc1;
+                }
+              }
+            }
+          } else {
+            ok = false;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+      }
+      tail_R = __shfl_sync(0xffffffffu, tail_R, 0);
+      if (ok && tail_R >= 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_vtail, tails & 1, abort_flag));
+        if (ok) {
+          // rows [Lk, end of its page) of the tile, in every 64-column chunk
+          const int r0 = w.Lk - tail_tile * B::BN;
+          const int r1 = ((w.Lk + kPrefillPage - 1) / kPrefillPage) * kPrefillPage - tail_tile * B::BN;
+          uint4* tile = reinterpret_cast<uint4*>(smem + B::KV_OFF + (tail_R % NS) * B::TILE_BYTES);
+          const int per_chunk = (r1 - r0) * 8;   // 16-byte stores per chunk
+          for (int i = lane; i < B::CHUNKS * per_chunk; i += 32) {
+            const int c = i / per_chunk, u = i % per_chunk;
+            tile[(c * B::CHUNK_BYTES + r0 * 128) / 16 + u] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_kv_full(tail_R));
+          ++tails;
+          tail_R = -1;
+        }
+      }
+      // the next item is claimed once this one's loads are issued (see below)
+      if (ok && lane == 0) next = claim();
+    }
+    if (lane == 0) {
+      if (*abort_flag) {
+        // let the copies in flight land before the CTA's shared memory goes away
+        volatile int never = 0;
+        for (uint32_t i = (issued > static_cast<uint32_t>(NS) ? issued - NS : 0u); i < issued; ++i) {
+          if (static_cast<int>(i) == tail_R) mbar_wait(bar_vtail, tails & 1, &never);
+          else mbar_wait(bar_kv_full(i), (i / NS) & 1, &never);
+        }
+        if (qc0 > 0) mbar_wait(bar_q, (qc0 - 1) & 1, &never);
+        if (qc1 > 0) mbar_wait(bar_q1, (qc1 - 1) & 1, &never);
+      }
+      __threadfence();   // this thread's counter updates precede the CTA's finish count
+    }
+  } else if (warp == 8) {
     // ---------------------------------------------------------------- TMA producer + scheduler
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -484,8 +668,11 @@ __global__ void __launch_bounds__(PrefillPersistCfg<D, F8>::THREADS, 1)
       const int my_qtile = k ? w.qtile[1] : w.qtile[0];
       const int my_head = k ? w.head[1] : w.head[0];
       const int q_row = my_qtile * B::BM + r;
-      const int row_last = p.causal ? min(q_row, w.L - 1) : w.L - 1;
-      const int tile_last = p.causal ? min(my_qtile * B::BM, w.L - 1) : w.L - 1;
+      // query q_row sees keys up to q_row + off (bottom-right aligned when
+      // paged; off = 0 for packed K/V); key tiles past tile_last need the mask
+      const int off = p.causal ? w.Lk - w.L : 0;
+      const int row_last = p.causal ? min(q_row + off, w.Lk - 1) : w.Lk - 1;
+      const int tile_last = p.causal ? min(my_qtile * B::BM + off, w.Lk - 1) : w.Lk - 1;
       float m_ref = 0.0f, l_sum = 0.0f;
       bool ok = true;
       for (int j = 0; j < nk; ++j) {

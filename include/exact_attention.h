@@ -139,8 +139,8 @@ typedef enum { FA_SCHEDULE_GRID = 0, FA_SCHEDULE_PERSISTENT = 1 } fa_prefill_sch
 
 /*
  * fa_prefill_last_schedule — the fa_prefill_schedule that the calling thread's
- * last fa_prefill or fa_prefill_fp8 call launched, or -1 if that call failed or
- * there was none.  Host only; never fails.
+ * last fa_prefill, fa_prefill_fp8 or fa_prefill_paged call launched, or -1 if
+ * that call failed or there was none.  Host only; never fails.
  */
 int fa_prefill_last_schedule(void);
 
@@ -217,7 +217,9 @@ int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_seqlens
  * included): they are never used.  A block_table entry outside the pool reads
  * as zeros and records FA_ERR_BAD_PAGE; device lengths that disagree with the
  * host copies record FA_ERR_PLAN_MISMATCH.  The host and device copies of
- * cu_seqlens_q and cache_seqlens must hold the same values.
+ * cu_seqlens_q and cache_seqlens must hold the same values.  Schedule: as for
+ * fa_prefill (persistent by default, the grid form under FA_PREFILL_SCHEDULE=
+ * grid, during graph capture or past 256 streams; bit-identical results).
  */
 int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
                      const int32_t* cu_seqlens_q_host, const void* k_pages, const void* v_pages,

@@ -214,11 +214,17 @@ def prefill_items(lens, num_q_heads, num_kv_heads, causal, BM=128, BN=128):
 
 MUTATIONS = ("no_q_empty_wait", "late_q_empty", "no_epilogue_wait", "consumers_short",
              "no_vh_empty_wait", "v_release_before_pv", "rescale_after_half")
+# planted mistakes of the paged producer's tail hand-off
+PAGED_MUTATIONS = ("tail_full_before_zero", "tail_no_land_wait")
 
 
-def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
+def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None, tails=frozenset()):
     """One CTA taking the items `claimed` (indices into `items`, in claim
-    order).  Raises ProtocolError on any violation."""
+    order).  Raises ProtocolError on any violation.  tails (paged K/V, bf16
+    only): items whose last V tile holds the cache's last, partly filled page;
+    that tile lands on the vtail barrier, the producer zeroes its rows past the
+    end and only then arrives on its kv_full barrier."""
+    assert not (tails and F8)
     sim = _Sim(seed)
     rng = sim.rng
     sim.bar("q0")
@@ -245,6 +251,7 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
                 sim.err(f"queue entry {i} released after {queue_reads.get(i, 0)} of {consumers} reads")
         sim.on_complete[f"item_empty{i}"] = all_read
     sim.bar("final")
+    sim.bar("vtail")
     queue, queue_reads = {}, {}
     o_state = [None, None]      # per slot: (item, tiles accumulated) or "read out"
     epilogue_reads = {}
@@ -252,7 +259,7 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
     rescale = {}
 
     def producer():
-        issued, qc = 0, [0, 0]
+        issued, qc, tails_done = 0, [0, 0], 0
         for n, it in enumerate(list(claimed) + [-1]):
             qi = n % QD
             if n >= QD:
@@ -265,12 +272,19 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
             if it < 0:
                 return
             nkv = items[it]
+            tail_R = None
             for e in range(2 * max(nkv)):
                 R = issued
                 if R >= NS:
                     yield ("wait", f"kv_empty{R % NS}", R // NS - 1)
-                yield ("expect_tx", f"kv_full{R % NS}", 1)
-                yield ("tma", f"kv_full{R % NS}", 1, f"ring{R % NS}", ("KV", it, e))
+                if it in tails and e == 2 * max(nkv) - 1:
+                    # the tail V tile lands on vtail; it is marked full below
+                    yield ("expect_tx", "vtail", 1)
+                    yield ("tma", "vtail", 1, f"ring{R % NS}", ("KV raw", it, e))
+                    tail_R = (R, e)
+                else:
+                    yield ("expect_tx", f"kv_full{R % NS}", 1)
+                    yield ("tma", f"kv_full{R % NS}", 1, f"ring{R % NS}", ("KV", it, e))
                 issued += 1
                 if e == 0:
                     for k in range(2):
@@ -280,6 +294,18 @@ def simulate(items, claimed, NS, F8, seed=0, QD=4, mutation=None):
                             yield ("expect_tx", f"q{k}", 1)
                             yield ("tma", f"q{k}", 1, f"qtile{k}", ("Q", it, k))
                             qc[k] += 1
+            if tail_R is not None:
+                R, e = tail_R
+                if mutation == "tail_full_before_zero":
+                    yield ("arrive", f"kv_full{R % NS}")
+                if mutation != "tail_no_land_wait":
+                    yield ("wait", "vtail", tails_done)
+                    yield ("read", f"ring{R % NS}", ("KV raw", it, e))
+                yield ("delay", rng.uniform(0.1, 0.6))          # the warp zeroes the rows past the end
+                yield ("write", f"ring{R % NS}", ("KV", it, e))
+                if mutation != "tail_full_before_zero":
+                    yield ("arrive", f"kv_full{R % NS}")
+                tails_done += 1
             yield ("delay", rng.uniform(0.0, 0.2))
 
     def take(n):
@@ -466,3 +492,12 @@ def random_case(seed):
     items = prefill_items(lens, hkv * G, hkv, rng.random() < 0.7)
     claimed = sorted(rng.sample(range(len(items)), min(len(items), rng.randint(1, 12))))
     return items, claimed, NS, F8
+
+
+def random_paged_case(seed):
+    """random_case restricted to bf16, with a random set of items whose last
+    V tile is a partly filled page (paged K/V)."""
+    rng = random.Random(seed + 30011)
+    items, claimed, _, _ = random_case(seed)
+    tails = frozenset(i for i in claimed if rng.random() < 0.5)
+    return items, claimed, rng.choice([5, 8]), tails

@@ -54,6 +54,36 @@ def test_unused_slots_poisoned_with_nan():
     check_full(inp, "chunked poisoned")
 
 
+def _schedule_cases():
+    return {
+        "tiny causal": W.tiny_chunked_prefill(),
+        "tiny full d=64 HND": W.tiny_chunked_prefill(64, "HND", False),
+        "odd group, page tails": W.make_chunked_prefill([0, 333, 129, 1024, 5], [200, 77, 300, 128, 1], 6, 2,
+                                                        128, seed=730, extra_pages=2),
+        "poisoned": W.poison_chunked(W.tiny_chunked_prefill()),
+    }
+
+
+@pytest.mark.parametrize("case", list(_schedule_cases()))
+def test_persistent_and_grid_schedules_bit_identical(case, monkeypatch):
+    """The persistent paged prefill (the default) and the grid form read the
+    same tiles in the same order: bit-identical O and LSE, including NaN-filled
+    page tails, which both zero before P V."""
+    import torch
+    import exact_attention_148_b200 as fa
+    inp = _schedule_cases()[case]
+    dev = chunked_device_inputs(inp)
+    monkeypatch.setenv("FA_PREFILL_SCHEDULE", "grid")
+    a = chunked_on_gpu(inp, dev=dev)
+    assert fa.prefill_last_schedule() == "grid"
+    monkeypatch.delenv("FA_PREFILL_SCHEDULE", raising=False)
+    b = chunked_on_gpu(inp, dev=dev, append=False)
+    assert fa.prefill_last_schedule() == "persistent"
+    assert torch.equal(a[0], b[0]), f"{case}: O differs between the schedules"
+    assert torch.equal(a[1], b[1]), f"{case}: LSE differs between the schedules"
+    assert _device_status() == 0
+
+
 def test_empty_prefix_is_bit_identical_to_prefill():
     """With nothing cached the chunked kernel sees the same tiles and masks as
     the packed prefill: the results must agree bit for bit."""
