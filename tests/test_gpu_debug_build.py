@@ -71,6 +71,9 @@ def every_entry_point(monkeypatch):
             keep(prefill_on_gpu(W.make_prefill(lens, hq, hkv, d, causal=causal, seed=700 + d + hq)),
                  f"prefill {sched} d={d}")
         keep(fp8_prefill(W.to_fp8_prefill(W.make_prefill(lens, 4, 2, 128, seed=710))), f"fp8 prefill {sched}")
+        keep(chunked_on_gpu(W.tiny_chunked_prefill())[:2], f"append + chunked prefill {sched}")
+        keep(chunked_on_gpu(W.poison_chunked(W.tiny_chunked_prefill(64, "HND")))[:2],
+             f"chunked prefill, NaN page tails {sched}")
     monkeypatch.delenv("FA_PREFILL_SCHEDULE", raising=False)
     dec = W.make_decode([70, 1500, 129, 0, 4097], 8, 2, 128, seed=720, extra_pages=3)
     for kernel in ("tensor_cores", "cuda_cores"):
@@ -79,7 +82,6 @@ def every_entry_point(monkeypatch):
     keep(decode_on_gpu(W.make_decode([300, 65], 4, 4, 64, seed=721), 3)[:2], "decode d=64")
     keep(fp8_decode(W.to_fp8_cache(dec), 3), "fp8 decode")
     keep(mtp_run(W.make_decode([300, 1200, 64], 8, 2, 128, seed=722, q_len=2), 3), "multi-token decode")
-    keep(chunked_on_gpu(W.tiny_chunked_prefill())[:2], "append + chunked prefill")
     keep(cascade_run(W.make_cascade(777, [5, 300, 0, 129], 8, 2, 128, seed=723)), "cascade decode")
     g = torch.Generator(device="cuda").manual_seed(724)
     parts_o = torch.randn(3, 5, 4, 128, device="cuda", generator=g)
