@@ -2,6 +2,7 @@
 
 #include <algorithm>
 #include <functional>
+#include <limits>
 #include <vector>
 
 #include "../../include/exact_attention.h"
@@ -45,9 +46,12 @@ CtaModel cta_model(bool tensor_cores, int kv_elem_bytes, int heads_per_cta) {
 // group, then request) and every running CTA moves at min(one CTA's limit,
 // HBM bandwidth / running CTAs).  Event simulation over a min-heap of finish
 // points measured in "bytes done by every running CTA" (all running CTAs
-// advance at the same rate, so that scale is shared).
+// advance at the same rate, so that scale is shared).  The elapsed time only
+// grows as events are processed, so the simulation stops, returning a value
+// above `cutoff`, as soon as it passes `cutoff` (a candidate that cannot win).
 double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64_t chunk, int slots,
-                          int head_dim, int kv_elem_bytes, const CtaModel& cm, int num_sms) {
+                          int head_dim, int kv_elem_bytes, const CtaModel& cm, int num_sms,
+                          int max_len, double cutoff) {
   const double bytes_per_token = 2.0 * head_dim * kv_elem_bytes;   // K and V rows of one kv head
   const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
   const double cta_bytes_per_us = cm.bytes_per_us;
@@ -56,23 +60,59 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
   // Running CTAs' finish points (bytes done by every running CTA).  Full-chunk
   // CTAs start in non-decreasing order and all have the same size, so their
   // finish points come in order: a FIFO ring holds them.  The other CTAs
-  // (each request's last split) go to a min-heap.  The next event is the
-  // smaller of the two fronts, so events come in the same order as from one
-  // heap of all running CTAs.
+  // (each request's last split, one per unit) have the request's own size,
+  // so a request's finish in the order they start: each request's wait in a
+  // queue of their own (lastq, units entries per request) and a min-heap
+  // holds the first of every request with some running, a handful of requests
+  // rather than every running CTA.  (Past kMaxQueuedLast entries one heap of
+  // all running last splits is used instead.)  The next event is the smaller
+  // of the two fronts, so events come in the same order as from one heap of
+  // all running CTAs.
   std::vector<double> ring(static_cast<size_t>(std::max(slots, 1)));
   size_t head = 0, count = 0;
-  std::vector<double> heap;
-  heap.reserve(static_cast<size_t>(slots));
+  const bool queued = static_cast<int64_t>(lens.size()) * units <= kMaxQueuedLast;
+  std::vector<double> lastq(queued ? lens.size() * static_cast<size_t>(units) : 0);
+  std::vector<int32_t> qhead(queued ? lens.size() : 0), qtail(queued ? lens.size() : 0);
+  using Front = std::pair<double, int32_t>;   // (finish point, request)
+  std::vector<Front> fronts;                  // min-heap of each request's first
+  std::vector<double> heap;                   // min-heap of all (past kMaxQueuedLast)
+  size_t running_last = 0;
   const auto later = std::greater<double>();
-  auto start_cta = [&](double finish, bool full_chunk) {
+  const auto later_front = [](const Front& x, const Front& y) { return x.first > y.first; };
+  auto start_cta = [&](double finish, bool full_chunk, size_t req) {
     if (full_chunk) {
       size_t at = head + count;
       if (at >= ring.size()) at -= ring.size();
       ring[at] = finish;
       ++count;
+      return;
+    }
+    ++running_last;
+    if (queued) {
+      lastq[req * static_cast<size_t>(units) + static_cast<size_t>(qtail[req])] = finish;
+      if (qtail[req]++ == qhead[req]) {
+        fronts.emplace_back(finish, static_cast<int32_t>(req));
+        std::push_heap(fronts.begin(), fronts.end(), later_front);
+      }
     } else {
       heap.push_back(finish);
       std::push_heap(heap.begin(), heap.end(), later);
+    }
+  };
+  auto last_front = [&]() { return queued ? fronts.front().first : heap.front(); };
+  auto pop_last = [&]() {
+    --running_last;
+    if (queued) {
+      const int32_t r = fronts.front().second;
+      std::pop_heap(fronts.begin(), fronts.end(), later_front);
+      fronts.pop_back();
+      if (++qhead[r] < qtail[r]) {
+        fronts.emplace_back(lastq[static_cast<size_t>(r) * static_cast<size_t>(units) + static_cast<size_t>(qhead[r])], r);
+        std::push_heap(fronts.begin(), fronts.end(), later_front);
+      }
+    } else {
+      std::pop_heap(heap.begin(), heap.end(), later);
+      heap.pop_back();
     }
   };
   // CTAs in grid order: request b's n splits (every one a full chunk but the
@@ -80,19 +120,17 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
   size_t b = 0;
   int64_t u = 0, sidx = 0, n = 1;
   double last = 0.0;
-  int64_t max_splits = 1;
   auto load = [&]() {
     const int64_t L = lens[b];
     n = std::max<int64_t>(1, ceil_div(L, chunk));
     last = static_cast<double>(std::max<int64_t>(0, L - (n - 1) * chunk)) * bytes_per_token + overhead_bytes;
-    max_splits = std::max(max_splits, n);
   };
   if (!lens.empty()) load();
   // start the next CTA at v, if any is left
   auto next_cta = [&](double v) -> bool {
     if (b >= lens.size()) return false;
     const bool is_full = sidx != n - 1;
-    start_cta(v + (is_full ? full : last), is_full);
+    start_cta(v + (is_full ? full : last), is_full, b);
     if (++sidx == n) {
       sidx = 0;
       if (++u == units) {
@@ -104,29 +142,31 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
   };
   for (int i = 0; i < slots; ++i)
     if (!next_cta(0.0)) break;
+  const double merge = ceil_div(std::max(max_len, 1), chunk) > 1 ? kMergeLaunchUs : 0.0;
+  const double limit = cutoff - merge;
   double v = 0.0, t = 0.0;
   size_t rate_for = 0;   // running count the rate below was computed for
-  double rate = 0.0;
-  while (count + heap.size() > 0) {
-    if (count + heap.size() != rate_for) {
-      rate_for = count + heap.size();
-      rate = std::min(cta_bytes_per_us, hbm / static_cast<double>(rate_for));
+  double inv_rate = 0.0;
+  while (count + running_last > 0) {
+    if (count + running_last != rate_for) {
+      rate_for = count + running_last;
+      inv_rate = 1.0 / std::min(cta_bytes_per_us, hbm / static_cast<double>(rate_for));
     }
+    if (t > limit) return t + merge;
     double nxt;
-    if (count > 0 && (heap.empty() || ring[head] <= heap.front())) {
+    if (count > 0 && (running_last == 0 || ring[head] <= last_front())) {
       nxt = ring[head];
       if (++head == ring.size()) head = 0;
       --count;
     } else {
-      nxt = heap.front();
-      std::pop_heap(heap.begin(), heap.end(), later);
-      heap.pop_back();
+      nxt = last_front();
+      pop_last();
     }
-    t += (nxt - v) / rate;
+    t += (nxt - v) * inv_rate;
     v = nxt;
     next_cta(v);
   }
-  return t + (max_splits > 1 ? kMergeLaunchUs : 0.0);
+  return t + merge;
 }
 
 // A lower bound of estimate_decode_us for the same arguments, in O(batch):
@@ -246,12 +286,16 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
                                                cm, num_sms), c);
     }
     std::sort(order.begin(), order.end());
+    // Candidates in increasing order of their lower bound; none whose bound
+    // exceeds the best estimate can win (its estimate is at least its bound),
+    // and a simulation stops once it passes the best estimate.
     double best_t = 0.0;
     chunk = 0;
     for (const auto& [lb, c] : order) {
       if (chunk != 0 && lb > best_t * (1.0 + 1e-9)) break;
-      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes, cm,
-                                          num_sms);
+      const double cutoff = chunk == 0 ? std::numeric_limits<double>::infinity() : best_t * (1.0 + 1e-9);
+      const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes, cm, num_sms,
+                                          max_len, cutoff);
       if (chunk == 0 || t < best_t * (1.0 - 1e-9) || (t <= best_t * (1.0 + 1e-9) && c > chunk)) {
         best_t = t;
         chunk = c;

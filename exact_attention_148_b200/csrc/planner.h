@@ -15,6 +15,9 @@ constexpr uint32_t kPlanMagic = 0xFA148D0Cu;
 constexpr int kMaxSplits = 128;
 constexpr int kMinChunkTokens = 512;
 constexpr int kItemsPerSlot = 8;   // the many-small-items candidate: items per resident CTA slot
+// Decode-time simulation: last splits kept in per-request queues up to this
+// many (batch x units) entries, one heap of all running ones beyond.
+constexpr int64_t kMaxQueuedLast = int64_t{1} << 21;
 
 struct DecodePlan {
   uint32_t magic = kPlanMagic;
