@@ -396,3 +396,27 @@ def test_cascade_validation_before_any_cuda_call(lib):
     assert call(ws=A + 16) == fa.FA_ERR_INVALID_ARG
     p8 = _plan([100, 2000], hq=8, hkv=2, kv_dtype="e4m3")
     assert call(plan=p8.handle) == fa.FA_ERR_PLAN_MISMATCH
+
+
+def _batch64():
+    # the paged decode batch's lengths (workloads.paged_decode_batch and its variants)
+    return np.random.default_rng(3).integers(1024, 32768 + 1, size=64)
+
+
+@pytest.mark.parametrize("name,lens,hq,hkv,q_len,kv,chunk,splits,tensor_cores", [
+    ("paged_decode_batch", _batch64(), 32, 8, 1, "bf16", 3200, 10, 1),
+    ("ragged_split_decode", [131072] + [2048] * 63, 32, 32, 1, "bf16", 16384, 8, 0),
+    ("long_split_decode", [131072] * 4, 32, 32, 1, "bf16", 65536, 2, 0),
+    ("paged_decode_gqa8", _batch64(), 64, 8, 1, "bf16", 3200, 10, 1),
+    ("paged_decode_gqa16", _batch64(), 32, 2, 1, "bf16", 5376, 6, 1),
+    ("paged_decode_batch_fp8", _batch64(), 32, 8, 1, "e4m3", 4032, 8, 1),
+    ("speculative_decode_batch", _batch64(), 32, 8, 4, "bf16", 10688, 3, 1),
+])
+def test_planner_choices_for_the_benchmark_batches(name, lens, hq, hkv, q_len, kv, chunk, splits, tensor_cores):
+    """The automatic plans the measured decode numbers were taken with (148
+    SMs): a change to the planner's search or model that moves one of them
+    shows up here, to be measured again."""
+    lens = np.asarray(lens, dtype=np.int32)
+    p = fa.decode_plan(lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                       max_pages_per_seq=int(((lens + 63) // 64).max()), num_sms=148, kv_dtype=kv, q_len=q_len)
+    assert (p.info.chunk_tokens, p.info.max_splits, p.info.tensor_cores) == (chunk, splits, tensor_cores), name
