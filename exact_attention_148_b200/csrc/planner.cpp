@@ -278,9 +278,11 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     // skip any whose bound already exceeds the best estimate: the choice is
     // the exhaustive search's, at a fraction of the simulations (the many-CTA
     // candidates, the costly ones to simulate, have the highest bounds).
+    for (int64_t& c : cands) c = std::max<int64_t>(c, kMinChunkTokens);
+    std::sort(cands.begin(), cands.end());
+    cands.erase(std::unique(cands.begin(), cands.end()), cands.end());   // one simulation per chunk
     std::vector<std::pair<double, int64_t>> order;
-    for (int64_t c : cands) {
-      c = std::max<int64_t>(c, kMinChunkTokens);
+    for (const int64_t c : cands) {
       if (ceil_div(max_len, c) > kMaxSplits) continue;
       order.emplace_back(lower_bound_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes,
                                                cm, num_sms), c);
