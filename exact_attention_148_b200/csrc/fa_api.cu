@@ -474,7 +474,7 @@ FA_API int fa_prefill_paged(const void* q, const int32_t* cu_seqlens_q_dev,
   if (!(scale > 0.0f) || std::isinf(scale)) return FA_ERR_INVALID_ARG;
   if (cu_seqlens_q_host[0] != 0) return FA_ERR_INVALID_ARG;
   const int64_t capacity = static_cast<int64_t>(max_pages_per_seq) * page_size;
-  if (capacity > INT32_MAX) return FA_ERR_INVALID_ARG;
+  if (capacity > (int64_t{1} << 30)) return FA_ERR_INVALID_ARG;   // as for fa_decode_plan
   std::vector<int64_t> q_lens, k_lens;
   for (int b = 0; b < batch; ++b) {
     const int64_t lq = static_cast<int64_t>(cu_seqlens_q_host[b + 1]) - cu_seqlens_q_host[b];

@@ -206,7 +206,8 @@ int fa_append_kv(const void* k_new, const void* v_new, const int32_t* cu_seqlens
  *   k_pages, v_pages, num_pages, strides, block_table, max_pages_per_seq:
  *       the page pool and table, as for fa_decode_paged.
  *   cache_seqlens_dev / cache_seqlens_host [batch] int32: keys per request,
- *       k_len_b >= q_len_b, k_len_b <= max_pages_per_seq * page_size.
+ *       k_len_b >= q_len_b, k_len_b <= max_pages_per_seq * page_size, and
+ *       max_pages_per_seq * page_size <= 2^30 (else FA_ERR_INVALID_ARG).
  *   causal != 0: the chunk's queries are the last q_len_b positions of the
  *       request's sequence, so query i sees keys 0 .. k_len_b - q_len_b + i
  *       (with k_len_b == q_len_b this is fa_prefill's causal mask).

@@ -305,6 +305,7 @@ def test_prefill_paged_validation_before_any_cuda_call(lib):
     # cache shorter than the chunk, and a cache past the table's capacity
     assert call(lens=np.array([99, 200], dtype=np.int32)) == fa.FA_ERR_INVALID_ARG
     assert call(max_pages=3) == fa.FA_ERR_INVALID_ARG               # 200 > 3 * 64
+    assert call(max_pages=(1 << 24) + 1) == fa.FA_ERR_INVALID_ARG   # capacity past 2^30 keys
     assert call(cu=np.array([0, 0, 300], dtype=np.int32)) == fa.FA_ERR_INVALID_ARG
 
 
