@@ -2,7 +2,9 @@
 
 fa_prefill_persist_kernel runs four kinds of roles in one CTA (TMA producer,
 MMA thread, eight softmax warps, two E4M3 converter warps) that hand tiles to
-each other through mbarriers waited on by phase parity.  A mistake in that
+each other through mbarriers waited on by phase parity.  With paged K/V the
+producer also hands over the V tile of a request's last, partly filled page
+only after zeroing its rows past the cache end (`tails`).  A mistake in that
 protocol shows up on the GPU as a hang (bounded by the kernels' wait limits),
 a stale tile or a wrong output; this model finds such mistakes on the host.
 
