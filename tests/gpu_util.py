@@ -128,3 +128,28 @@ def jumping_keys(inp, factors, tile=128):
 # x25 and x40 by 65-75 more (past the guard).  Scores stay near 120, where
 # fp32 scores still meet the LSE bound.
 JUMP_FACTORS = [1.0, 8.0, 1.0, 25.0, 3.0, 40.0, 0.5, 12.0]
+
+
+def jumping_keys_paged(inp, factors, tile=128):
+    """A ChunkedPrefillInputs with the key at logical position t of every
+    request multiplied by factors[(t // tile) % len(factors)]: the cached
+    prefix in the page pool and the chunk's own new rows alike (NHD or HND)."""
+    import workloads as W
+    kp = W.bf16_bits_to_f32(inp.k_pages_bits).copy()
+    kn = W.bf16_bits_to_f32(inp.k_new_bits).copy()
+    ps = inp.page_size
+    prefix = inp.prefix_lens
+    for b in range(inp.batch):
+        for t in range(int(prefix[b])):
+            f = factors[(t // tile) % len(factors)]
+            page, slot = int(inp.block_table[b, t // ps]), t % ps
+            if inp.layout == "NHD":
+                kp[page, slot] *= f
+            else:
+                kp[page, :, slot] *= f
+        for i in range(int(inp.chunk_lens[b])):
+            t = int(prefix[b]) + i
+            kn[int(inp.cu_seqlens_q[b]) + i] *= factors[(t // tile) % len(factors)]
+    inp.k_pages_bits = W.f32_to_bf16_bits(kp)
+    inp.k_new_bits = W.f32_to_bf16_bits(kn)
+    return inp

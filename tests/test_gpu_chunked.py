@@ -5,8 +5,9 @@ import pytest
 
 import oracle
 import workloads as W
-from tests.gpu_util import (bf16_to_f64, chunked_device_inputs, chunked_on_gpu, compare,
-                            oracle_pool_after_append, prefill_on_gpu, to_dev_bf16, to_dev_i32)
+from tests.gpu_util import (JUMP_FACTORS, bf16_to_f64, chunked_device_inputs, chunked_on_gpu, compare,
+                            jumping_keys_paged, oracle_pool_after_append, prefill_on_gpu, to_dev_bf16,
+                            to_dev_i32)
 
 pytestmark = pytest.mark.gpu
 
@@ -82,6 +83,17 @@ def test_persistent_and_grid_schedules_bit_identical(case, monkeypatch):
     assert torch.equal(a[0], b[0]), f"{case}: O differs between the schedules"
     assert torch.equal(a[1], b[1]), f"{case}: LSE differs between the schedules"
     assert _device_status() == 0
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+def test_score_jumps_between_key_tiles(schedule, monkeypatch):
+    """Cached and new keys whose scores jump by tens to hundreds (base 2) from
+    one 128-key tile to the next, through the block table: the reference
+    maximum raised late or at once, against the oracle."""
+    monkeypatch.setenv("FA_PREFILL_SCHEDULE", schedule)
+    inp = jumping_keys_paged(W.make_chunked_prefill([0, 333, 700, 1024], [200, 77, 300, 129], 8, 2, 128,
+                                                    seed=740, extra_pages=2), JUMP_FACTORS)
+    check_full(inp, f"chunked score jumps ({schedule})")
 
 
 def test_empty_prefix_is_bit_identical_to_prefill():
