@@ -153,3 +153,23 @@ def jumping_keys_paged(inp, factors, tile=128):
     inp.k_pages_bits = W.f32_to_bf16_bits(kp)
     inp.k_new_bits = W.f32_to_bf16_bits(kn)
     return inp
+
+
+def jumping_keys_decode(inp, factors, tile=128):
+    """A DecodeInputs with the cached key at logical position t of every
+    request multiplied by factors[(t // tile) % len(factors)] (NHD or HND pool)."""
+    import workloads as W
+    kp = W.bf16_bits_to_f32(inp.k_pages_bits).copy()
+    ps = inp.page_size
+    for b in range(inp.batch):
+        L = int(inp.cache_seqlens[b])
+        for t0 in range(0, L, ps):
+            page = int(inp.block_table[b, t0 // ps])
+            for t in range(t0, min(t0 + ps, L)):
+                f = factors[(t // tile) % len(factors)]
+                if inp.layout == "NHD":
+                    kp[page, t - t0] *= f
+                else:
+                    kp[page, :, t - t0] *= f
+    inp.k_pages_bits = W.f32_to_bf16_bits(kp)
+    return inp

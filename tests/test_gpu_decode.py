@@ -4,7 +4,8 @@ import pytest
 
 import oracle
 import workloads as W
-from tests.gpu_util import (bf16_to_f64, compare, decode_device_inputs, decode_on_gpu, to_dev_i32)
+from tests.gpu_util import (JUMP_FACTORS, bf16_to_f64, compare, decode_device_inputs, decode_on_gpu,
+                            jumping_keys_decode, to_dev_i32)
 
 pytestmark = pytest.mark.gpu
 
@@ -216,3 +217,13 @@ def test_tensor_core_poisoned_and_permuted():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
     c = decode_on_gpu(W.relayout(inp, "HND"), 3, kernel="tensor_cores")
     assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
+
+
+@pytest.mark.parametrize("kernel", ["tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("num_splits", [0, 1, 5])
+def test_score_jumps_between_key_blocks(kernel, num_splits):
+    """Cached keys whose scores jump by tens to hundreds (base 2) from one
+    128-key block to the next: every split's online softmax and the log-sum-exp
+    merge across splits, against the oracle."""
+    inp = jumping_keys_decode(W.make_decode([1000, 129, 2500, 64, 700], 8, 2, 128, seed=750), JUMP_FACTORS)
+    check_all_rows(inp, num_splits, f"decode score jumps {kernel} splits={num_splits}", kernel=kernel)

@@ -5,7 +5,8 @@ import pytest
 
 import oracle
 import workloads as W
-from tests.gpu_util import (bf16_to_f64, compare, decode_device_inputs, to_dev_bf16, to_dev_i32)
+from tests.gpu_util import (JUMP_FACTORS, bf16_to_f64, compare, decode_device_inputs, jumping_keys_decode,
+                            to_dev_bf16, to_dev_i32)
 
 pytestmark = pytest.mark.gpu
 
@@ -161,3 +162,17 @@ def test_full_size_sampled_rows(kernel):
     hi = np.array([r[1] for r in rows])
     compare(out.float().cpu().numpy()[bi, hi].astype(np.float64), lse.cpu().numpy()[bi, hi],
             o_ref, l_ref, "fp8 full size")
+
+
+@pytest.mark.parametrize("kernel", ["tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("num_splits", [0, 1, 5])
+def test_score_jumps_between_key_blocks_fp8(kernel, num_splits):
+    """The bf16 decode's score-jump case on an E4M3 cache; K gets its own
+    scale so the large keys do not saturate."""
+    base = jumping_keys_decode(W.make_decode([1000, 129, 2500, 64, 700], 8, 2, 128, seed=751), JUMP_FACTORS)
+    inp = W.to_fp8_cache(base)
+    kf = W.bf16_bits_to_f32(base.k_pages_bits)
+    k_scale = float(np.abs(kf).max()) / W.E4M3_MAX
+    inp.k_pages_bits = W.quantize_e4m3(kf, k_scale)
+    inp.extra = dict(inp.extra, k_scale=k_scale)
+    check_all_rows(inp, num_splits, f"fp8 decode score jumps {kernel} splits={num_splits}", kernel=kernel)
