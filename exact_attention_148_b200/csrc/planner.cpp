@@ -49,9 +49,16 @@ CtaModel cta_model(bool tensor_cores, int kv_elem_bytes, int heads_per_cta) {
 // advance at the same rate, so that scale is shared).  The elapsed time only
 // grows as events are processed, so the simulation stops, returning a value
 // above `cutoff`, as soon as it passes `cutoff` (a candidate that cannot win).
+// Buffers of one simulation, kept across the candidates of a plan.
+struct SimScratch {
+  std::vector<double> ring, lastq, heap;
+  std::vector<int32_t> qhead, qtail;
+  std::vector<std::pair<double, int32_t>> fronts;
+};
+
 double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64_t chunk, int slots,
                           int head_dim, int kv_elem_bytes, const CtaModel& cm, int num_sms,
-                          int max_len, double cutoff) {
+                          int max_len, double cutoff, SimScratch& sc) {
   const double bytes_per_token = 2.0 * head_dim * kv_elem_bytes;   // K and V rows of one kv head
   const double hbm = kHbmBytesPerUs148 * num_sms / 148.0;
   const double cta_bytes_per_us = cm.bytes_per_us;
@@ -68,14 +75,23 @@ double estimate_decode_us(const std::vector<int32_t>& lens, int64_t units, int64
   // all running last splits is used instead.)  The next event is the smaller
   // of the two fronts, so events come in the same order as from one heap of
   // all running CTAs.
-  std::vector<double> ring(static_cast<size_t>(std::max(slots, 1)));
+  std::vector<double>& ring = sc.ring;
+  ring.resize(static_cast<size_t>(std::max(slots, 1)));
   size_t head = 0, count = 0;
   const bool queued = static_cast<int64_t>(lens.size()) * units <= kMaxQueuedLast;
-  std::vector<double> lastq(queued ? lens.size() * static_cast<size_t>(units) : 0);
-  std::vector<int32_t> qhead(queued ? lens.size() : 0), qtail(queued ? lens.size() : 0);
+  std::vector<double>& lastq = sc.lastq;
+  std::vector<int32_t>& qhead = sc.qhead;
+  std::vector<int32_t>& qtail = sc.qtail;
+  if (queued) {
+    lastq.resize(lens.size() * static_cast<size_t>(units));
+    qhead.assign(lens.size(), 0);
+    qtail.assign(lens.size(), 0);
+  }
   using Front = std::pair<double, int32_t>;   // (finish point, request)
-  std::vector<Front> fronts;                  // min-heap of each request's first
-  std::vector<double> heap;                   // min-heap of all (past kMaxQueuedLast)
+  std::vector<Front>& fronts = sc.fronts;     // min-heap of each request's first
+  std::vector<double>& heap = sc.heap;        // min-heap of all (past kMaxQueuedLast)
+  fronts.clear();
+  heap.clear();
   size_t running_last = 0;
   const auto later = std::greater<double>();
   const auto later_front = [](const Front& x, const Front& y) { return x.first > y.first; };
@@ -293,11 +309,12 @@ int make_decode_plan(const int32_t* cache_seqlens_host, int batch, int num_q_hea
     // and a simulation stops once it passes the best estimate.
     double best_t = 0.0;
     chunk = 0;
+    SimScratch scratch;
     for (const auto& [lb, c] : order) {
       if (chunk != 0 && lb > best_t * (1.0 + 1e-9)) break;
       const double cutoff = chunk == 0 ? std::numeric_limits<double>::infinity() : best_t * (1.0 + 1e-9);
       const double t = estimate_decode_us(pl.seqlens, units, c, slots, head_dim, kv_elem_bytes, cm, num_sms,
-                                          max_len, cutoff);
+                                          max_len, cutoff, scratch);
       if (chunk == 0 || t < best_t * (1.0 - 1e-9) || (t <= best_t * (1.0 + 1e-9) && c > chunk)) {
         best_t = t;
         chunk = c;
