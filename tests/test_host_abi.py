@@ -421,3 +421,67 @@ def test_planner_choices_for_the_benchmark_batches(name, lens, hq, hkv, q_len, k
     p = fa.decode_plan(lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
                        max_pages_per_seq=int(((lens + 63) // 64).max()), num_sms=148, kv_dtype=kv, q_len=q_len)
     assert (p.info.chunk_tokens, p.info.max_splits, p.info.tensor_cores) == (chunk, splits, tensor_cores), name
+
+
+def _random_lengths(rng):
+    kind = rng.integers(0, 4)
+    B = int(rng.integers(1, 257))
+    if kind == 0:      # uniform over a wide range
+        return rng.integers(0, 1 << 17, size=B)
+    if kind == 1:      # a few long requests among short ones
+        lens = rng.integers(1, 4096, size=B)
+        lens[rng.integers(0, B, size=max(1, B // 16))] = rng.integers(1 << 16, 1 << 20)
+        return lens
+    if kind == 2:      # page multiples and their neighbours
+        return np.clip(64 * rng.integers(0, 600, size=B) + rng.integers(-1, 2, size=B), 0, None)
+    return rng.integers(0, 600, size=B)   # all within the minimum chunk
+
+
+def test_plan_invariants_on_random_batches(lib):
+    """Seeded batch mixes (lengths 0 to 2^20, 1-256 requests, every head
+    group, both cache types, 1-4 query tokens, automatic and forced splits):
+    the plan tiles every request's keys in page-multiple chunks within the
+    split limit, sizes the workspace for its splits, and picks the kernel by
+    the documented rule."""
+    rng = np.random.default_rng(2024)
+    for case in range(300):
+        lens = _random_lengths(rng).astype(np.int32)
+        hkv = int(rng.choice([1, 2, 4, 8]))
+        G = int(rng.choice([1, 2, 3, 4, 8, 16]))
+        d = int(rng.choice([64, 128]))
+        kv = "e4m3" if rng.random() < 0.3 else "bf16"
+        q_len = int(rng.choice([1, 1, 2, 4])) if d == 128 and G <= 8 else 1
+        if q_len * G > 16:
+            q_len = 1
+        L = int(lens.max())
+        splits = 0 if rng.random() < 0.6 else int(rng.integers(1, 200))
+        max_pages = max(1, (L + 63) // 64)
+        if q_len > 1:
+            lens = np.maximum(lens, q_len).astype(np.int32)
+            L = int(lens.max())
+            max_pages = max(1, (L + 63) // 64)
+        p = fa.decode_plan(lens, num_q_heads=G * hkv, num_kv_heads=hkv, head_dim=d,
+                           max_pages_per_seq=max_pages, num_sms=148, num_splits=splits,
+                           kv_dtype=kv, q_len=q_len)
+        i = p.info
+        where = f"case {case}: B={len(lens)} max={L} G={G} d={d} {kv} q_len={q_len} splits={splits}"
+        chunk = i.chunk_tokens
+        assert chunk % 64 == 0 and chunk >= 64, where
+        assert 1 <= i.max_splits <= 128, where
+        assert i.max_splits == max(_splits(x, chunk) for x in lens), where
+        if splits:
+            assert i.max_splits <= splits, where
+        elif L > 512:
+            assert chunk >= min(512, L) or i.max_splits == 128, where
+        tc_ok = d == 128 and q_len * G <= 16
+        assert bool(i.tensor_cores) == (q_len > 1 or (tc_ok and (kv == "e4m3" or G >= 4))), where
+        hpc = G if i.tensor_cores else next(g for g in (8, 4, 2, 1) if G % g == 0)
+        assert i.heads_per_cta == hpc, where
+        units = hkv * (G // hpc)
+        assert i.num_work_items == units * sum(_splits(x, chunk) for x in lens), where
+        if i.max_splits == 1:
+            assert p.workspace_bytes == 0, where
+        else:
+            rows = len(lens) * q_len * G * hkv
+            need = i.max_splits * rows * (d * 4 + 4)
+            assert need <= p.workspace_bytes < need + 512 and p.workspace_bytes % 256 == 0, where
