@@ -1,5 +1,7 @@
-"""Host-side model of the tensor-core split-decode kernel's synchronisation
-protocol (fa_decode_tc_kernel, one CTA = one (request, kv head, split)).
+"""Host-side models of the split-decode kernels' synchronisation protocols:
+the tensor-core kernel (fa_decode_tc_kernel, `simulate`) and, at the end of
+this file, the CUDA-core kernel (fa_decode_split_kernel, `simulate_cc`); one
+CTA = one (request, kv head, split).
 
 The kernel runs a TMA producer (warp 0), an MMA thread (warp 1) and four
 softmax warps, one per TMEM lane quadrant.  They hand data to each other
@@ -226,3 +228,119 @@ def random_case(seed):
     tail = r.random() < 0.5
     grew = [False] + [r.random() < 0.4 for _ in range(n_tiles - 1)]
     return n_tiles, items, kv8, tail, grew
+
+
+# --------------------------------------------------------------------------
+# The CUDA-core split kernel (fa_decode_split_kernel): one TMA lane fills a
+# ring of STAGES page slots (K and V of one 64-token page each; full barrier
+# with a byte count, empty barrier with four arrivals); four consumer warps
+# each read their own 16 token rows of a page (scores from K, then P V from V)
+# and arrive on the page's empty barrier; after the last page the warps pass
+# the named barrier, write their (O, m, l) states into a combine scratch that
+# aliases the start of the K ring, pass the named barrier again and read every
+# warp's state.  Shared memory of the K ring is tracked in 256-byte chunks so
+# the aliasing is exact for every head size, group size and cache type.
+
+CC_MUTATIONS = (
+    "empty_three_arrivals",    # a page slot freed after three of the four warps
+    "release_before_pv",       # a warp frees the slot after its scores, before P V
+    "no_barrier_before_combine",
+    "no_barrier_after_combine",
+    "full_parity",             # consumers wait with the page index as parity
+    "ring_parity",             # producer waits on the slot's current phase
+)
+
+_CHUNK = 256
+
+
+def simulate_cc(num_pages, d, gc, kv8, seed=0, mutation=None):
+    """One CTA over `num_pages` cached pages (head size d, gc query heads per
+    CTA, E4M3 cache if kv8).  Raises ProtocolError on any violation."""
+    assert num_pages >= 1 and d in (64, 128) and gc in (1, 2, 4, 8)
+    stages = 6 if kv8 else 3
+    row_bytes = d * (1 if kv8 else 2)
+    tile_bytes = 64 * row_bytes
+    cmb_m = 4 * gc * d * 4
+    cmb_l = cmb_m + 4 * gc * 4
+    assert cmb_l + 4 * gc * 4 <= 2 * stages * tile_bytes
+    sim = _Sim(seed)
+    rng = sim.rng
+    for s in range(stages):
+        sim.bar(f"full{s}")
+        sim.bar(f"empty{s}", 3 if mutation == "empty_three_arrivals" else 4)
+    sim.bar("named", 4)
+
+    def chunks(lo, hi):          # K-ring chunks covering bytes [lo, hi)
+        return [f"k{c}" for c in range(lo // _CHUNK, (hi + _CHUNK - 1) // _CHUNK)]
+
+    def rows(st, w):             # warp w's 16 token rows of slot st
+        lo = st * tile_bytes + w * 16 * row_bytes
+        return chunks(lo, lo + 16 * row_bytes)
+
+    def producer():
+        for i in range(num_pages):
+            st = i % stages
+            phase = i // stages if mutation == "ring_parity" else i // stages - 1
+            yield ("wait", f"empty{st}", phase)
+            # one byte count for both copies; each piece of the page lands on its own
+            parts = [(c, ("K", i)) for w in range(4) for c in rows(st, w)] + \
+                    [(f"v{st}_{w}", ("V", i)) for w in range(4)]
+            yield ("expect_tx", f"full{st}", len(parts))
+            for res, tag in parts:
+                yield ("tma", f"full{st}", 1, res, tag)
+            yield ("delay", rng.uniform(0.0, 0.2))
+
+    def cmb_parts(w):
+        o = chunks(w * gc * d * 4, (w + 1) * gc * d * 4)
+        m = chunks(cmb_m + w * gc * 4, cmb_m + (w + 1) * gc * 4)
+        l = chunks(cmb_l + w * gc * 4, cmb_l + (w + 1) * gc * 4)
+        return sorted(set(o + m + l))
+
+    def consumer(w):
+        syncs = 0
+
+        def named_sync():
+            nonlocal syncs
+            yield ("arrive", "named")
+            yield ("wait", "named", syncs)
+            syncs += 1
+
+        for i in range(num_pages):
+            st = i % stages
+            yield ("wait", f"full{st}", i if mutation == "full_parity" else i // stages)
+            for c in rows(st, w):
+                yield ("read", c, ("K", i))
+            yield ("delay", rng.uniform(0.2, 1.5))              # q . k for the warp's rows
+            for c in rows(st, w):
+                yield ("read", c, ("K", i))
+            if mutation == "release_before_pv":
+                yield ("arrive", f"empty{st}")
+            yield ("read", f"v{st}_{w}", ("V", i))
+            yield ("delay", rng.uniform(0.2, 1.5))              # softmax and P V
+            yield ("read", f"v{st}_{w}", ("V", i))
+            if mutation != "release_before_pv":
+                yield ("arrive", f"empty{st}")
+        if mutation != "no_barrier_before_combine":
+            yield from named_sync()
+        yield ("delay", rng.uniform(0.0, 0.5))
+        for c in cmb_parts(w):
+            yield ("write", c, ("combine",))
+        if mutation != "no_barrier_after_combine":
+            yield from named_sync()
+        yield ("delay", rng.uniform(0.0, 0.3))
+        for v in range(4):
+            for c in cmb_parts(v):
+                yield ("read", c, ("combine",))
+
+    sim.add_role("producer", producer())
+    for w in range(4):
+        sim.add_role(f"consumer{w}", consumer(w))
+    sim.run()
+
+
+def random_cc_case(seed):
+    """(num_pages, d, gc, kv8) over the kernel's configurations."""
+    import random
+    r = random.Random(2000 + seed)
+    return r.choice([1, 2, 3, 4, 5, 6, 7, 9, 13, 20]), r.choice([64, 128]), r.choice([1, 2, 4, 8]), \
+        r.random() < 0.5
