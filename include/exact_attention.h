@@ -83,7 +83,8 @@ typedef struct {
   int chunk_tokens;      /* keys per split; a multiple of page_size */
   int max_splits;        /* splits of the longest planned request */
   int heads_per_cta;     /* query heads of one kv head packed into a CTA */
-  int num_work_items;    /* non-empty (request, kv-head group, split) items */
+  int num_work_items;    /* (request, kv-head group, split) CTAs that run: each split of a
+                            request, and one for an empty request (it writes O = 0, LSE = -inf) */
   int max_seqlen;        /* longest planned cache length */
   size_t workspace_bytes;
   int kv_dtype;          /* fa_kv_dtype the plan was made for */
