@@ -113,7 +113,9 @@ typedef struct {
  *   scale: score multiplier; NaN means 1/sqrt(d).  Must be > 0 otherwise.
  *   out  [T, Hq, d] bf16 (written); lse [T, Hq] fp32 natural-log LSE, or NULL.
  * Supported: d in {64, 128}; Hq % Hkv == 0; each sequence length >= 1;
- * T < 2^31 / (Hq*d).  Output rows of different sequences never mix.
+ * T * Hq * d < 2^40 (else FA_ERR_UNSUPPORTED; the kernels index q, out and
+ * lse with 64-bit offsets, and T itself is an int32 as cu_seqlens are).
+ * Output rows of different sequences never mix.
  *
  * Schedule (plan-stage load balancing: wsisp.com "FIA / FlashAttention",
  * section 二).  The work is cut into items of two 128-row query tiles that read

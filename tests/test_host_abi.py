@@ -246,6 +246,12 @@ def test_prefill_validation_before_any_cuda_call(lib):
     assert call(cuh=bad.ctypes.data_as(ctypes.c_void_p)) == fa.FA_ERR_INVALID_ARG
     bad2 = np.array([5, 10], dtype=np.int32)                        # must start at 0
     assert call(cuh=bad2.ctypes.data_as(ctypes.c_void_p)) == fa.FA_ERR_INVALID_ARG
+    # T * Hq * d must stay below 2^40: two 2^22-token sequences, 1024 heads, d = 128
+    big = np.array([0, 1 << 22, 1 << 23], dtype=np.int32)
+    big_call = lambda hq: lib.fa_prefill(_fake(A), _fake(A), _fake(A), _fake(A),
+                                         big.ctypes.data_as(ctypes.c_void_p), 2, hq, hq, 128, 1,
+                                         float("nan"), _fake(A), None, None)
+    assert big_call(1024) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_decode_validation_before_any_cuda_call(lib):
